@@ -1,0 +1,412 @@
+// DFlash draft-step oracle: a plain, slow, double-precision CPU implementation.
+//
+// TEST INFRASTRUCTURE ONLY.  This file is the correctness reference that the
+// GPU library is checked against.  Only the test suite, the package smoke
+// check and the benchmark's CPU-baseline leg may load it.  It shares no code,
+// header, table or constant generator with the CUDA library, and the CUDA
+// library never calls it.
+//
+// What it computes follows the DFlash technical summaries ("DFlash – Block
+// Diffusion for Flash Speculative Decoding", gist.science ja/nl pages):
+//   * §2.2 (inference design), context-feature bullet: hidden states of a fixed,
+//     uniformly spaced set of target layers are concatenated and projected into
+//     one compact context feature                         -> oracle_fuse_context
+//   * §2.2, KV-injection bullet: that feature enters the key/value projection of
+//     every draft layer and is kept in the draft KV cache   -> oracle_inject_kv
+//   * §2.2, parallel block diffusion bullet: one forward pass predicts a block of
+//     masked positions; §2.3 random-anchor bullet: the block starts from the
+//     target's clean token; §2.3 architecture bullet: embedding and LM head are
+//     shared with the target                               -> oracle_draft_block
+//   * §5 (claims), lossless verification: drafts are kept only while they equal
+//     the target's own greedy tokens                      -> oracle_accept
+//   * §2.3 loss-weighting bullet: w_k = exp(-(k-1)/gamma)  -> oracle_loss_weights
+//
+// The summaries give no layer equations.  The layer internals used here
+// (pre-norm RMSNorm, rotate-half RoPE, grouped-query attention without a mask,
+// SwiGLU MLP, a final norm before the LM head) and the bf16 storage points R()
+// are the plain reading of a standard decoder layer; the CUDA library states
+// the same reading in its header.  R() is round-to-nearest-even to bf16 when
+// storage is bf16 and the identity when storage is fp32.  Every accumulation is
+// fp64.  No blocking, fusion or reordering is done beyond what the definitions
+// state: plain loops, parallelised over independent outputs only.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#include <algorithm>
+#include <limits>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+extern "C" {
+
+struct oracle_config {
+    int hidden, n_layers, n_q_heads, n_kv_heads, head_dim, intermediate, vocab;
+    int n_sel, target_hidden, mask_id;
+    int storage;            // 0: fp32 storage, R() is the identity. 1: bf16 storage.
+    double rope_theta, rms_eps;
+};
+
+// All matrices are [out, in] row-major in the storage type (uint16 bf16 bit
+// patterns, or float).  lm_head may alias embed (tied embedding / LM head).
+struct oracle_weights {
+    const void* w_fc;      // [hidden, n_sel*target_hidden]
+    const void* g_fc;      // [hidden]
+    const void* embed;     // [vocab, hidden]
+    const void* lm_head;   // [vocab, hidden]
+    const void* g_final;   // [hidden]
+    const void* g_in[16];
+    const void* wq[16];    // [n_q_heads*head_dim, hidden]
+    const void* wk[16];    // [n_kv_heads*head_dim, hidden]
+    const void* wv[16];    // [n_kv_heads*head_dim, hidden]
+    const void* wo[16];    // [hidden, n_q_heads*head_dim]
+    const void* g_post[16];
+    const void* w_gate[16];  // [intermediate, hidden]
+    const void* w_up[16];    // [intermediate, hidden]
+    const void* w_down[16];  // [hidden, intermediate]
+};
+
+// ---------------------------------------------------------------------------
+// Storage-type helpers
+// ---------------------------------------------------------------------------
+
+static inline double bf16_bits_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+static inline double load(const void* p, long i, int storage) {
+    if (storage == 1) return bf16_bits_to_double(((const uint16_t*)p)[i]);
+    return (double)((const float*)p)[i];
+}
+
+// Round-to-nearest-even of a double to the nearest bf16 value (8 significant
+// bits, exponent range of fp32, gradual underflow).  Direct rounding from the
+// double, not via fp32, so there is no double rounding.
+double oracle_round_bf16(double x) {
+    if (std::isnan(x) || std::isinf(x) || x == 0.0) return x;
+    int e;
+    std::frexp(x, &e);                 // |x| = m * 2^e, m in [0.5, 1)
+    int E = e - 1;                     // |x| in [2^E, 2^(E+1))
+    if (E < -126) E = -126;            // subnormal range: fixed quantum 2^-133
+    double quantum = std::ldexp(1.0, E - 7);
+    double q = std::nearbyint(x / quantum);   // default FP env rounds half to even
+    double r = q * quantum;
+    if (std::fabs(r) >= std::ldexp(1.0, 128)) return x > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
+void oracle_round_bf16_array(const double* x, double* y, long n) {
+    for (long i = 0; i < n; ++i) y[i] = oracle_round_bf16(x[i]);
+}
+
+static inline double R(double x, int storage) {
+    return storage == 1 ? oracle_round_bf16(x) : x;
+}
+
+// ---------------------------------------------------------------------------
+// Building blocks (each exported so the tests can pin it on its own)
+// ---------------------------------------------------------------------------
+
+// y = x / sqrt(mean(x^2) + eps) * g      (no rounding)
+void oracle_rmsnorm(const double* x, const double* g, int n, double eps, double* y) {
+    double ss = 0.0;
+    for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+    double inv = 1.0 / std::sqrt(ss / n + eps);
+    for (int i = 0; i < n; ++i) y[i] = x[i] * inv * g[i];
+}
+
+// Rotate-half rotary embedding of one head vector v[0..d) at position pos:
+// pairs (i, i + d/2), angle pos * theta^(-2i/d).
+void oracle_rope(double* v, int d, long pos, double theta) {
+    int h = d / 2;
+    for (int i = 0; i < h; ++i) {
+        double inv_freq = std::pow(theta, -2.0 * i / d);
+        double ang = (double)pos * inv_freq;
+        double c = std::cos(ang), s = std::sin(ang);
+        double a = v[i], b = v[i + h];
+        v[i] = a * c - b * s;
+        v[i + h] = b * c + a * s;
+    }
+}
+
+// Multi-head attention without a mask.  q: [nrow][nq][d]; k, v: [nkv][n][d];
+// o: [nrow][nq][d].  Query head hq reads key/value head hq / (nq/nkv).
+// Scores are scaled by 1/sqrt(d); softmax is the two-pass max / sum form.  With
+// round_p != 0 the probabilities are rounded to bf16 before they weight V.
+// The output is not rounded here.
+void oracle_attention(const double* q, int nrow, int nq, const double* k, const double* v,
+                      int n, int nkv, int d, int round_p, double* o) {
+    int G = nq / nkv;
+    double scale = 1.0 / std::sqrt((double)d);
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int r = 0; r < nrow; ++r) {
+        for (int hq = 0; hq < nq; ++hq) {
+            int g = hq / G;
+            const double* qv = q + ((long)r * nq + hq) * d;
+            const double* kh = k + (long)g * n * d;
+            const double* vh = v + (long)g * n * d;
+            std::vector<double> s(n > 0 ? n : 1);
+            double m = -INFINITY;
+            for (int i = 0; i < n; ++i) {
+                double acc = 0.0;
+                for (int t = 0; t < d; ++t) acc += qv[t] * kh[(long)i * d + t];
+                s[i] = acc * scale;
+                if (s[i] > m) m = s[i];
+            }
+            double Z = 0.0;
+            for (int i = 0; i < n; ++i) { s[i] = std::exp(s[i] - m); Z += s[i]; }
+            double* ov = o + ((long)r * nq + hq) * d;
+            for (int t = 0; t < d; ++t) ov[t] = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double p = s[i] / Z;
+                if (round_p) p = oracle_round_bf16(p);
+                for (int t = 0; t < d; ++t) ov[t] += p * vh[(long)i * d + t];
+            }
+        }
+    }
+}
+
+// y[m][n] = sum_k x[m][k] * W[n][k]; W in storage type, [N, K] row-major.
+static void linear(const double* x, int M, int K, const void* W, int N, int storage, double* y) {
+    #pragma omp parallel
+    {
+        std::vector<double> wrow(K);
+        #pragma omp for schedule(static)
+        for (int nn = 0; nn < N; ++nn) {
+            for (int kk = 0; kk < K; ++kk) wrow[kk] = load(W, (long)nn * K + kk, storage);
+            for (int mm = 0; mm < M; ++mm) {
+                const double* xr = x + (long)mm * K;
+                double acc = 0.0;
+                // fp64 dot product; the simd reduction only changes the order
+                // in which fp64 partial sums are added.
+                #pragma omp simd reduction(+:acc)
+                for (int kk = 0; kk < K; ++kk) acc += xr[kk] * wrow[kk];
+                y[(long)mm * N + nn] = acc;
+            }
+        }
+    }
+}
+
+static void load_vec(const void* p, int n, int storage, double* out) {
+    for (int i = 0; i < n; ++i) out[i] = load(p, i, storage);
+}
+
+// Uniformly spaced target layers, shallow to deep (reading of §2.2's
+// context-feature bullet; the pages name no indices): l_i = round(i*(L_t-1)/(n_sel-1)).
+void oracle_layer_ids(int n_target_layers, int n_sel, int* ids) {
+    for (int i = 0; i < n_sel; ++i) {
+        if (n_sel == 1) { ids[i] = n_target_layers - 1; continue; }
+        double t = (double)i * (n_target_layers - 1) / (n_sel - 1);
+        ids[i] = (int)std::floor(t + 0.5);
+    }
+}
+
+// §2.3 loss-weighting bullet: w_k = exp(-(k-1)/gamma), k = 1..gamma.
+void oracle_loss_weights(int gamma, double* w) {
+    for (int k = 1; k <= gamma; ++k) w[k - 1] = std::exp(-(double)(k - 1) / gamma);
+}
+
+// ---------------------------------------------------------------------------
+// a1: fuse the context feature.
+// ctx_r = R( RMSNorm( R( concat_i h_i[r] . W_fc^T ) ) * g_fc )
+// hiddens[i] points at n_sel arrays of [rows, target_hidden] (row stride in
+// elements), concatenated in ascending layer order along the feature axis.
+// ---------------------------------------------------------------------------
+void oracle_fuse_context(const oracle_config* c, const oracle_weights* w,
+                         const void* const* hiddens, long row_stride, int rows, double* ctx_out) {
+    int S = c->storage, H = c->hidden, Ht = c->target_hidden, Kc = c->n_sel * Ht;
+    std::vector<double> cat((size_t)rows * Kc);
+    for (int r = 0; r < rows; ++r)
+        for (int i = 0; i < c->n_sel; ++i)
+            for (int t = 0; t < Ht; ++t)
+                cat[(size_t)r * Kc + (size_t)i * Ht + t] = load(hiddens[i], (long)r * row_stride + t, S);
+    std::vector<double> y((size_t)rows * H);
+    linear(cat.data(), rows, Kc, w->w_fc, H, S, y.data());
+    std::vector<double> g(H);
+    load_vec(w->g_fc, H, S, g.data());
+    std::vector<double> tmp(H);
+    for (int r = 0; r < rows; ++r) {
+        double* yr = y.data() + (size_t)r * H;
+        for (int t = 0; t < H; ++t) yr[t] = R(yr[t], S);
+        oracle_rmsnorm(yr, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) ctx_out[(size_t)r * H + t] = R(tmp[t], S);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a2: inject the context feature into every draft layer's K/V cache.
+// For layer l and row r at absolute position p = pos0 + r:
+//   K_l[p] = R( RoPE_p( ctx_r . W_k,l^T ) ),  V_l[p] = R( ctx_r . W_v,l^T )
+// Cache layout (this oracle's own): k_cache/v_cache [L][nkv][cap][d].
+// ---------------------------------------------------------------------------
+void oracle_inject_kv(const oracle_config* c, const oracle_weights* w, const double* ctx,
+                      int rows, int pos0, double* k_cache, double* v_cache, int cap) {
+    int S = c->storage, H = c->hidden, d = c->head_dim, nkv = c->n_kv_heads, Nkv = nkv * d;
+    std::vector<double> kk((size_t)rows * Nkv), vv((size_t)rows * Nkv);
+    for (int l = 0; l < c->n_layers; ++l) {
+        linear(ctx, rows, H, w->wk[l], Nkv, S, kk.data());
+        linear(ctx, rows, H, w->wv[l], Nkv, S, vv.data());
+        for (int r = 0; r < rows; ++r) {
+            long p = (long)pos0 + r;
+            for (int g = 0; g < nkv; ++g) {
+                double* kh = kk.data() + (size_t)r * Nkv + (size_t)g * d;
+                double* vh = vv.data() + (size_t)r * Nkv + (size_t)g * d;
+                oracle_rope(kh, d, p, c->rope_theta);
+                size_t base = (((size_t)l * nkv + g) * cap + p) * d;
+                for (int t = 0; t < d; ++t) {
+                    k_cache[base + t] = R(kh[t], S);
+                    v_cache[base + t] = R(vh[t], S);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3..a7: draft one block of gamma positions in one forward pass.
+// Position 0 holds the clean anchor token, positions 1..gamma-1 the mask
+// token; block position j sits at absolute position len + j.  Every block
+// query sees the whole committed context [0, len) and every block position
+// (no mask).  The block's own K/V are used for this pass only and are not
+// written to the cache.  Mask position j predicts the token at len + j:
+// drafts[j-1] = argmax of its logits (ties to the lowest index), j = 1..gamma-1.
+// logits (optional): [(gamma-1), vocab], margin (optional): top1 - top2 per row.
+// ---------------------------------------------------------------------------
+void oracle_draft_block(const oracle_config* c, const oracle_weights* w,
+                        const double* k_cache, const double* v_cache, int cap, int len,
+                        int anchor, int gamma, int* drafts, double* logits, double* margin) {
+    int S = c->storage, H = c->hidden, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
+    int Nq = nq * d, Nkv = nkv * d, I = c->intermediate, V = c->vocab;
+    int n = len + gamma;
+
+    // a3: embedding of [anchor, mask, ..., mask] (exact copies of table rows).
+    std::vector<double> x((size_t)gamma * H);
+    for (int j = 0; j < gamma; ++j) {
+        int tok = (j == 0) ? anchor : c->mask_id;
+        for (int t = 0; t < H; ++t) x[(size_t)j * H + t] = load(w->embed, (long)tok * H + t, S);
+    }
+
+    std::vector<double> g(H), h((size_t)gamma * H), tmp(H);
+    std::vector<double> q((size_t)gamma * Nq), kb((size_t)gamma * Nkv), vb((size_t)gamma * Nkv);
+    std::vector<double> K((size_t)nkv * n * d), Vv((size_t)nkv * n * d), o((size_t)gamma * Nq);
+    std::vector<double> y((size_t)gamma * H);
+    std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I);
+
+    for (int l = 0; l < c->n_layers; ++l) {
+        // a4: h = R(RMSNorm(x) * g_in); q, k with RoPE at len + j; v.
+        load_vec(w->g_in[l], H, S, g.data());
+        for (int j = 0; j < gamma; ++j) {
+            oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+            for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
+        }
+        linear(h.data(), gamma, H, w->wq[l], Nq, S, q.data());
+        linear(h.data(), gamma, H, w->wk[l], Nkv, S, kb.data());
+        linear(h.data(), gamma, H, w->wv[l], Nkv, S, vb.data());
+        for (int j = 0; j < gamma; ++j) {
+            long p = (long)len + j;
+            for (int hq = 0; hq < nq; ++hq) oracle_rope(q.data() + (size_t)j * Nq + (size_t)hq * d, d, p, c->rope_theta);
+            for (int g2 = 0; g2 < nkv; ++g2) oracle_rope(kb.data() + (size_t)j * Nkv + (size_t)g2 * d, d, p, c->rope_theta);
+        }
+        for (auto& e : q) e = R(e, S);
+        for (auto& e : kb) e = R(e, S);
+        for (auto& e : vb) e = R(e, S);
+
+        // a5: keys/values = injected context rows [0, len) then the block rows.
+        for (int g2 = 0; g2 < nkv; ++g2) {
+            for (int i = 0; i < len; ++i)
+                for (int t = 0; t < d; ++t) {
+                    size_t src = (((size_t)l * nkv + g2) * cap + i) * d + t;
+                    K[((size_t)g2 * n + i) * d + t] = k_cache[src];
+                    Vv[((size_t)g2 * n + i) * d + t] = v_cache[src];
+                }
+            for (int j = 0; j < gamma; ++j)
+                for (int t = 0; t < d; ++t) {
+                    K[((size_t)g2 * n + len + j) * d + t] = kb[(size_t)j * Nkv + (size_t)g2 * d + t];
+                    Vv[((size_t)g2 * n + len + j) * d + t] = vb[(size_t)j * Nkv + (size_t)g2 * d + t];
+                }
+        }
+        oracle_attention(q.data(), gamma, nq, K.data(), Vv.data(), n, nkv, d, S == 1, o.data());
+        for (auto& e : o) e = R(e, S);
+
+        // a6: x = R(x + o.Wo^T); h2 = R(RMSNorm(x) * g_post);
+        //     m = R(silu(h2.Wg^T) * (h2.Wu^T)); x = R(x + m.Wd^T)
+        linear(o.data(), gamma, Nq, w->wo[l], H, S, y.data());
+        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
+        load_vec(w->g_post[l], H, S, g.data());
+        for (int j = 0; j < gamma; ++j) {
+            oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+            for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
+        }
+        linear(h.data(), gamma, H, w->w_gate[l], I, S, gt.data());
+        linear(h.data(), gamma, H, w->w_up[l], I, S, up.data());
+        for (size_t i = 0; i < mm.size(); ++i) {
+            double a = gt[i];
+            double silu = a / (1.0 + std::exp(-a));
+            mm[i] = R(silu * up[i], S);
+        }
+        linear(mm.data(), gamma, I, w->w_down[l], H, S, y.data());
+        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
+    }
+
+    // a7: final norm of the mask positions, shared LM head, argmax.
+    int nd = gamma - 1;
+    if (nd <= 0) return;
+    load_vec(w->g_final, H, S, g.data());
+    std::vector<double> hf((size_t)nd * H);
+    for (int j = 1; j < gamma; ++j) {
+        oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) hf[(size_t)(j - 1) * H + t] = R(tmp[t], S);
+    }
+    std::vector<double> lg((size_t)nd * V);
+    linear(hf.data(), nd, H, w->lm_head, V, S, lg.data());
+    for (int r = 0; r < nd; ++r) {
+        const double* row = lg.data() + (size_t)r * V;
+        int best = 0;
+        for (int vv = 1; vv < V; ++vv) if (row[vv] > row[best]) best = vv;
+        double second = -INFINITY;
+        for (int vv = 0; vv < V; ++vv) if (vv != best && row[vv] > second) second = row[vv];
+        drafts[r] = best;
+        if (margin) margin[r] = (V > 1) ? row[best] - second : INFINITY;
+    }
+    if (logits) std::memcpy(logits, lg.data(), sizeof(double) * lg.size());
+}
+
+// ---------------------------------------------------------------------------
+// a8: greedy lossless acceptance for one request.
+// a = largest k <= gamma-1 with drafts[i] == target[i] for all i < k;
+// next_anchor = target[a]; committed += a + 1; len = min(len, committed).
+// Returns 0, or -7 (token out of range: nothing is changed, outputs are -1).
+// ---------------------------------------------------------------------------
+int oracle_accept(int gamma, int vocab, const int* drafts, const int* target,
+                  int* accept_len, int* next_anchor, int* len, int* committed) {
+    for (int i = 0; i < gamma; ++i) {
+        if (target[i] < 0 || target[i] >= vocab) {
+            *accept_len = -1;
+            *next_anchor = -1;
+            return -7;
+        }
+    }
+    int a = 0;
+    while (a < gamma - 1 && drafts[a] == target[a]) ++a;
+    *accept_len = a;
+    *next_anchor = target[a];
+    *committed += a + 1;
+    if (*len > *committed) *len = *committed;
+    return 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+}  // extern "C"

@@ -1,0 +1,218 @@
+"""Python wrapper of the CPU oracle (test infrastructure only).
+
+Loads liboracle.so (built from dflash_oracle.cpp) and marshals numpy arrays.
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+use this module; the GPU library never imports it.  It imports nothing from
+the GPU package either: callers pass numpy arrays (bf16 tensors as uint16 bit
+patterns, fp32 as float32) and a plain dict of shapes.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class _Cfg(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("n_layers", C.c_int), ("n_q_heads", C.c_int),
+                ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("intermediate", C.c_int),
+                ("vocab", C.c_int), ("n_sel", C.c_int), ("target_hidden", C.c_int),
+                ("mask_id", C.c_int), ("storage", C.c_int),
+                ("rope_theta", C.c_double), ("rms_eps", C.c_double)]
+
+
+class _W(C.Structure):
+    _fields_ = [("w_fc", C.c_void_p), ("g_fc", C.c_void_p), ("embed", C.c_void_p),
+                ("lm_head", C.c_void_p), ("g_final", C.c_void_p)] + \
+               [(n, C.c_void_p * 16) for n in ("g_in", "wq", "wk", "wv", "wo", "g_post",
+                                                "w_gate", "w_up", "w_down")]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        dp = C.POINTER(C.c_double)
+        ip = C.POINTER(C.c_int)
+        L.oracle_round_bf16.restype = C.c_double
+        L.oracle_round_bf16.argtypes = [C.c_double]
+        L.oracle_round_bf16_array.argtypes = [dp, dp, C.c_long]
+        L.oracle_rmsnorm.argtypes = [dp, dp, C.c_int, C.c_double, dp]
+        L.oracle_rope.argtypes = [dp, C.c_int, C.c_long, C.c_double]
+        L.oracle_attention.argtypes = [dp, C.c_int, C.c_int, dp, dp, C.c_int, C.c_int, C.c_int, C.c_int, dp]
+        L.oracle_layer_ids.argtypes = [C.c_int, C.c_int, ip]
+        L.oracle_loss_weights.argtypes = [C.c_int, dp]
+        L.oracle_fuse_context.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.POINTER(C.c_void_p),
+                                          C.c_long, C.c_int, dp]
+        L.oracle_inject_kv.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, C.c_int, dp, dp, C.c_int]
+        L.oracle_draft_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, dp, C.c_int, C.c_int,
+                                         C.c_int, C.c_int, ip, dp, dp]
+        L.oracle_accept.restype = C.c_int
+        L.oracle_accept.argtypes = [C.c_int, C.c_int, ip, ip, ip, ip, ip, ip]
+        L.oracle_num_threads.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _dp(a: np.ndarray):
+    assert a.dtype == np.float64 and a.flags.c_contiguous
+    return a.ctypes.data_as(C.POINTER(C.c_double))
+
+
+def _ip(a: np.ndarray):
+    assert a.dtype == np.int32 and a.flags.c_contiguous
+    return a.ctypes.data_as(C.POINTER(C.c_int))
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+# ---------------------------------------------------------------------------
+# Building blocks
+# ---------------------------------------------------------------------------
+
+def round_bf16(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    lib().oracle_round_bf16_array(_dp(x), _dp(y), x.size)
+    return y
+
+
+def rmsnorm(x, g, eps: float) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    y = np.empty_like(x)
+    lib().oracle_rmsnorm(_dp(x), _dp(g), x.size, eps, _dp(y))
+    return y
+
+
+def rope(v, pos: int, theta: float) -> np.ndarray:
+    v = np.array(v, dtype=np.float64, copy=True)
+    lib().oracle_rope(_dp(v), v.size, pos, theta)
+    return v
+
+
+def attention(q, k, v, round_p: bool = False) -> np.ndarray:
+    """q: [nrow, nq, d]; k, v: [nkv, n, d] -> o [nrow, nq, d]."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    nrow, nq, d = q.shape
+    nkv, n, _ = k.shape
+    o = np.empty_like(q)
+    lib().oracle_attention(_dp(q), nrow, nq, _dp(k), _dp(v), n, nkv, d, int(round_p), _dp(o))
+    return o
+
+
+def layer_ids(n_target_layers: int, n_sel: int) -> List[int]:
+    out = np.zeros(n_sel, dtype=np.int32)
+    lib().oracle_layer_ids(n_target_layers, n_sel, _ip(out))
+    return [int(v) for v in out]
+
+
+def loss_weights(gamma: int) -> np.ndarray:
+    w = np.zeros(gamma, dtype=np.float64)
+    lib().oracle_loss_weights(gamma, _dp(w))
+    return w
+
+
+# ---------------------------------------------------------------------------
+# The draft step
+# ---------------------------------------------------------------------------
+
+class OracleDrafter:
+    """The oracle's drafter.  ``shape`` keys: hidden, n_layers, n_q_heads,
+    n_kv_heads, head_dim, intermediate, vocab, n_sel, target_hidden, mask_id,
+    storage ("bf16" | "f32"), rope_theta, rms_eps.  ``weights``: numpy arrays
+    (uint16 bf16 bits or float32) named like the GPU library's weight table:
+    w_fc, g_fc, embed, lm_head, g_final, and per layer (list ``layers``) g_in,
+    wq, wk, wv, wo, g_post, w_gate, w_up, w_down."""
+
+    def __init__(self, shape: Dict, weights: Dict):
+        self.shape = dict(shape)
+        st = 1 if shape["storage"] == "bf16" else 0
+        self._np_dtype = np.uint16 if st == 1 else np.float32
+        self.cfg = _Cfg(shape["hidden"], shape["n_layers"], shape["n_q_heads"], shape["n_kv_heads"],
+                        shape["head_dim"], shape["intermediate"], shape["vocab"], shape["n_sel"],
+                        shape["target_hidden"], shape["mask_id"], st,
+                        float(shape["rope_theta"]), float(shape["rms_eps"]))
+        self._keep = []
+        w = _W()
+
+        def ptr(a):
+            a = np.ascontiguousarray(a)
+            assert a.dtype == self._np_dtype, (a.dtype, self._np_dtype)
+            self._keep.append(a)
+            return a.ctypes.data
+
+        w.w_fc = ptr(weights["w_fc"])
+        w.g_fc = ptr(weights["g_fc"])
+        w.embed = ptr(weights["embed"])
+        w.lm_head = ptr(weights["lm_head"])
+        w.g_final = ptr(weights["g_final"])
+        for l, lw in enumerate(weights["layers"]):
+            for name in ("g_in", "wq", "wk", "wv", "wo", "g_post", "w_gate", "w_up", "w_down"):
+                getattr(w, name)[l] = ptr(lw[name])
+        self.w = w
+
+    # -- cache of one request: k, v [L, nkv, cap, d] fp64 -------------------
+    def new_cache(self, cap: int):
+        s = self.shape
+        k = np.zeros((s["n_layers"], s["n_kv_heads"], cap, s["head_dim"]), dtype=np.float64)
+        return {"k": k, "v": np.zeros_like(k), "cap": cap, "len": 0, "committed": 0}
+
+    def fuse_context(self, hiddens: Sequence[np.ndarray]) -> np.ndarray:
+        """hiddens: n_sel arrays [rows, target_hidden] -> ctx [rows, hidden] fp64."""
+        hs = [np.ascontiguousarray(h) for h in hiddens]
+        for h in hs:
+            assert h.dtype == self._np_dtype
+        rows = hs[0].shape[0]
+        arr = (C.c_void_p * len(hs))(*[h.ctypes.data for h in hs])
+        out = np.empty((rows, self.shape["hidden"]), dtype=np.float64)
+        lib().oracle_fuse_context(C.byref(self.cfg), C.byref(self.w), arr, hs[0].shape[1], rows, _dp(out))
+        return out
+
+    def inject_kv(self, cache: Dict, ctx: np.ndarray) -> None:
+        ctx = np.ascontiguousarray(ctx, dtype=np.float64)
+        rows = ctx.shape[0]
+        if cache["len"] + rows > cache["cap"]:
+            raise ValueError("capacity")
+        lib().oracle_inject_kv(C.byref(self.cfg), C.byref(self.w), _dp(ctx), rows, cache["len"],
+                               _dp(cache["k"]), _dp(cache["v"]), cache["cap"])
+        cache["len"] += rows
+
+    def draft_block(self, cache: Dict, anchor: int, gamma: int, want_logits: bool = False):
+        """Returns (drafts [gamma-1] int32, margin [gamma-1], logits or None)."""
+        if cache["len"] + gamma > cache["cap"]:
+            raise ValueError("capacity")
+        nd = max(gamma - 1, 0)
+        drafts = np.zeros(max(nd, 1), dtype=np.int32)
+        margin = np.zeros(max(nd, 1), dtype=np.float64)
+        logits = np.zeros((max(nd, 1), self.shape["vocab"]), dtype=np.float64) if want_logits else None
+        lib().oracle_draft_block(C.byref(self.cfg), C.byref(self.w), _dp(cache["k"]), _dp(cache["v"]),
+                                 cache["cap"], cache["len"], int(anchor), int(gamma), _ip(drafts),
+                                 _dp(logits) if logits is not None else None, _dp(margin))
+        return drafts[:nd], margin[:nd], (logits[:nd] if logits is not None else None)
+
+    def accept(self, cache: Dict, drafts, target) -> tuple:
+        """Returns (status, accept_len, next_anchor) and updates cache lengths."""
+        target = np.ascontiguousarray(target, dtype=np.int32)
+        gamma = target.size
+        d = np.ascontiguousarray(drafts, dtype=np.int32)
+        if d.size == 0:
+            d = np.zeros(1, dtype=np.int32)
+        a = np.zeros(1, dtype=np.int32)
+        nxt = np.zeros(1, dtype=np.int32)
+        ln = np.array([cache["len"]], dtype=np.int32)
+        cm = np.array([cache["committed"]], dtype=np.int32)
+        st = lib().oracle_accept(gamma, self.shape["vocab"], _ip(d), _ip(target), _ip(a), _ip(nxt), _ip(ln), _ip(cm))
+        cache["len"], cache["committed"] = int(ln[0]), int(cm[0])
+        return st, int(a[0]), int(nxt[0])
