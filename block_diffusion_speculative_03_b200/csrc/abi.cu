@@ -1,0 +1,942 @@
+// C ABI of libdflash (include/dflash.h): argument validation, workspace and
+// cache layout, tensor-map encoding, and the launch sequence of each call.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/dflash.h"
+#include "../../include/dflash_diag.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+using namespace df;
+
+namespace {
+
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled_t get_encode() {
+    static PFN_encodeTiled_t fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_encodeTiled_t)p;
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `rows` rows of
+// `stride` elements, box {64, box_rows}, 128-byte swizzle, zero fill out of bounds.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                    uint32_t box_rows) {
+    PFN_encodeTiled_t enc = get_encode();
+    if (!enc || rows == 0 || inner == 0) return false;
+    if (((uintptr_t)base & 15) || ((stride * 2) & 15)) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {stride * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline size_t al(size_t v, size_t a = 1024) { return (v + a - 1) / a * a; }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+constexpr int kMaxCtas = 160;   // >= SMs of any B200 part
+
+struct WsLayout {
+    size_t status, rope, x, h, q, o, act, hf, y, y32, lgs, part_o, part_ml, req_ok, gpart, gcnt, rec, total;
+    int nt_max;
+    long long n_counters;
+};
+
+int m_tiles_for(int M) { return M <= 0 ? 0 : cdiv(M, pick_nt(M)); }
+
+void make_layout(const dflash_config& c, WsLayout& L) {
+    const bool bf = c.dtype == DFLASH_BF16;
+    const size_t es = bf ? 2 : 4;
+    const long long H = c.hidden, d = c.head_dim, Nq = (long long)c.n_q_heads * d, Nkv = (long long)c.n_kv_heads * d;
+    const long long I = c.intermediate, V = c.vocab;
+    const long long Mmax = (long long)c.max_batch * c.max_gamma;
+    const long long Mlm = std::max(1LL, (long long)c.max_batch * (c.max_gamma - 1));
+    const long long R = std::max(1, c.max_rows);
+    size_t off = 0;
+    L.status = off; off += 1024;
+    L.rope = off; off = al(off + (size_t)c.max_position * (d / 2) * sizeof(float2));
+    L.x = off; off = al(off + Mmax * H * es);
+    L.h = off; off = al(off + Mmax * H * es);
+    L.q = off; off = al(off + Mmax * Nq * es);
+    L.o = off; off = al(off + Mmax * Nq * es);
+    L.act = off; off = al(off + Mmax * I * es);
+    L.hf = off; off = al(off + Mlm * H * es);
+    L.y = off; off = al(off + R * H * es);
+    L.req_ok = off; off = al(off + (size_t)c.max_batch * 4);
+    L.y32 = L.lgs = L.part_o = L.part_ml = L.gpart = L.gcnt = L.rec = off;
+    L.nt_max = 0;
+    L.n_counters = 0;
+    if (!bf) {
+        long long y32 = std::max(std::max(Mmax * (Nq + 2 * Nkv), Mmax * 2 * I), std::max(Mmax * H, R * 2 * Nkv));
+        L.y32 = off; off = al(off + (size_t)y32 * 4);
+        L.lgs = off; off = al(off + (size_t)Mlm * V * 4);
+    } else {
+        const long long parts = kAttnTargetCtas + (long long)c.max_batch * c.n_kv_heads;
+        L.part_o = off; off = al(off + (size_t)parts * 64 * d * 4);
+        L.part_ml = off; off = al(off + (size_t)parts * 64 * sizeof(float2));
+        L.nt_max = pick_nt((int)std::max(std::max(Mmax, Mlm), R));
+        L.gpart = off; off = al(off + gemm_partial_bytes(kMaxCtas, L.nt_max));
+        const long long t_layer = std::max(std::max((long long)cdiv(Nq, 128) + 2 * cdiv(Nkv, 128), (long long)cdiv(H, 128)),
+                                           I / 64);
+        const long long t_big = std::max((long long)cdiv(H, 128), 10LL * cdiv(Nkv, 128));
+        L.n_counters = std::max(std::max(t_layer * m_tiles_for((int)Mmax), (long long)cdiv(V, 128) * m_tiles_for((int)Mlm)),
+                                t_big * m_tiles_for((int)R));
+        L.gcnt = off; off = al(off + (size_t)L.n_counters * 4);
+        L.rec = off; off = al(off + (size_t)cdiv(V, 128) * Mlm * sizeof(float4));
+    }
+    L.total = off;
+}
+
+int validate_config(const dflash_config* c) {
+    if (!c) return DFLASH_INVALID_ARG;
+    if (c->hidden <= 0 || c->n_layers < 0 || c->n_layers > DFLASH_MAX_LAYERS || c->n_q_heads <= 0 ||
+        c->n_kv_heads <= 0 || c->head_dim <= 0 || c->intermediate <= 0 || c->vocab <= 0 || c->n_sel <= 0 ||
+        c->target_hidden <= 0 || c->max_gamma < 1 || c->max_batch < 1 || c->max_rows < 0 || c->max_position < 2 ||
+        !(c->rope_theta > 0) || !(c->rms_eps >= 0))
+        return DFLASH_INVALID_ARG;
+    if (c->mask_id < 0 || c->mask_id >= c->vocab) return DFLASH_INVALID_ARG;
+    if (c->n_q_heads % c->n_kv_heads) return DFLASH_INVALID_ARG;
+    if (c->dtype != DFLASH_BF16 && c->dtype != DFLASH_F32) return DFLASH_INVALID_ARG;
+    if (c->max_gamma > 32 || c->n_sel > 8 || (c->head_dim & 1)) return DFLASH_UNSUPPORTED;
+    if (c->hidden % 8 || c->target_hidden % 8) return DFLASH_UNSUPPORTED;
+    if (c->dtype == DFLASH_BF16) {
+        if (c->head_dim != 64 && c->head_dim != 128) return DFLASH_UNSUPPORTED;
+        if (c->hidden % 64 || c->intermediate % 64 || c->target_hidden % 64) return DFLASH_UNSUPPORTED;
+        if ((c->n_q_heads / c->n_kv_heads) * c->max_gamma > 64) return DFLASH_UNSUPPORTED;
+    } else {
+        if (c->max_position > 12000) return DFLASH_UNSUPPORTED;   // fp32 attention keeps a row of scores in smem
+    }
+    return DFLASH_OK;
+}
+
+}  // namespace
+
+struct dflash_handle {
+    dflash_config cfg;
+    dflash_weights w;
+    int num_sms;
+    uint8_t* ws;
+    size_t ws_bytes;
+    WsLayout L;
+    int* status;
+    float2* rope;
+    void *x, *h, *q, *o, *act, *hf, *y;
+    float *y32, *lgs, *part_o, *gpart;
+    float2* part_ml;
+    int *req_ok, *gcnt;
+    float4* rec;
+    CUtensorMap tm_wfc, tm_lm;
+    CUtensorMap tm_wq[DFLASH_MAX_LAYERS], tm_wk[DFLASH_MAX_LAYERS], tm_wv[DFLASH_MAX_LAYERS], tm_wo[DFLASH_MAX_LAYERS];
+    CUtensorMap tm_wg[DFLASH_MAX_LAYERS], tm_wu[DFLASH_MAX_LAYERS], tm_wd[DFLASH_MAX_LAYERS];
+    long long launches;
+    // Diagnostic timing (dflash_diag_timing_*): event pairs around launches.
+    std::vector<cudaEvent_t> ev;
+    std::vector<int> ev_kind;
+    int ev_used = 0;
+    bool timing = false;
+};
+
+struct dflash_cache {
+    const dflash_handle* h;
+    uint8_t* mem;
+    size_t bytes;
+    int batch, capacity;
+    int* status;
+    int* len;
+    int* committed;
+    void* slab;
+    long long s_kv, s_kind, s_layer, s_req;
+    CUtensorMap tm_slab;
+};
+
+namespace {
+
+struct CacheLayout {
+    size_t len, committed, slab, total;
+};
+void cache_layout(const dflash_config& c, int batch, int capacity, CacheLayout& L) {
+    const size_t es = c.dtype == DFLASH_BF16 ? 2 : 4;
+    L.len = 256;
+    L.committed = L.len + al((size_t)batch * 4, 256);
+    L.slab = al(L.committed + al((size_t)batch * 4, 256), 1024);
+    L.total = L.slab + (size_t)batch * c.n_layers * 2 * c.n_kv_heads * (size_t)capacity * c.head_dim * es;
+}
+
+inline cudaStream_t S(dflash_stream s) { return (cudaStream_t)s; }
+inline cudaStream_t st_of(dflash_stream s) { return (cudaStream_t)s; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? DFLASH_OK : DFLASH_CUDA; }
+
+bool aligned16(const void* p) { return p && (((uintptr_t)p) & 15) == 0; }
+
+// Launch groups reported by the diagnostic timer.
+enum TimedKind {
+    TK_EMBED = 0, TK_RMSNORM, TK_GEMM_QKV, TK_ATTENTION, TK_GEMM_O, TK_GEMM_SWIGLU, TK_GEMM_DOWN, TK_GEMM_LMHEAD,
+    TK_LM_REDUCE, TK_GEMM_FUSE, TK_GEMM_INJECT, TK_INJECT_FINALIZE, TK_ACCEPT, TK_SET_LEN, TK_SIMT_F32, TK_COUNT
+};
+const char* kTimedNames[TK_COUNT] = {"embed", "rmsnorm", "gemm_qkv", "attention", "gemm_o", "gemm_swiglu",
+                                     "gemm_down", "gemm_lmhead", "lm_reduce", "gemm_fuse", "gemm_inject",
+                                     "inject_finalize", "accept", "set_len", "simt_f32"};
+
+// Records a CUDA event before and after the launches in its scope when the
+// handle's diagnostic timer is on (events on the launch stream).
+struct Timed {
+    dflash_handle* h;
+    cudaStream_t st;
+    int slot = -1;
+    Timed(dflash_handle* h_, int kind, cudaStream_t st_) : h(h_), st(st_) {
+        if (h->timing && h->ev_used + 2 <= (int)h->ev.size()) {
+            slot = h->ev_used;
+            h->ev_used += 2;
+            h->ev_kind[slot / 2] = kind;
+            cudaEventRecord(h->ev[slot], st);
+        }
+    }
+    ~Timed() {
+        if (slot >= 0) cudaEventRecord(h->ev[slot + 1], st);
+    }
+};
+
+// Common GEMM plumbing.
+void gemm_common(dflash_handle* h, GemmParams& p) {
+    p.partial = h->gpart;
+    p.counters = h->gcnt;
+    p.status = h->status;
+    p.ctas = 0;
+}
+
+int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st) {
+    gemm_common(h, p);
+    int e = launch_gemm_tc(p, nt, std::min(h->num_sms, kMaxCtas), st);
+    h->launches += p.units > 0 ? 1 : 0;
+    return e == 0 ? DFLASH_OK : DFLASH_CUDA;
+}
+
+// Activation operand map: rows x K bf16 with row stride `stride`, box rows nt.
+bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride, int nt) {
+    return encode_bf16_2d(m, base, (uint64_t)K, (uint64_t)rows, (uint64_t)stride, (uint32_t)nt);
+}
+
+void attn_plan(int B, int nkv, int cap, int& splits, int& chunk) {
+    int s = cdiv(kAttnTargetCtas, (long long)B * nkv);
+    s = std::max(1, std::min(s, cdiv(cap, 64)));
+    chunk = cdiv(cdiv(cap, s), 64) * 64;
+    splits = cdiv(cap, chunk);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dflash_status_string(int s) {
+    switch (s) {
+    case DFLASH_OK: return "ok";
+    case DFLASH_INVALID_ARG: return "invalid argument";
+    case DFLASH_UNSUPPORTED: return "unsupported shape";
+    case DFLASH_CUDA: return "CUDA error";
+    case DFLASH_WORKSPACE: return "workspace or cache memory too small";
+    case DFLASH_CAPACITY: return "cache capacity exceeded";
+    case DFLASH_STATE: return "cache state: len != committed";
+    case DFLASH_TOKEN_RANGE: return "token id out of range";
+    case DFLASH_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int dflash_workspace_bytes(const dflash_config* cfg, size_t* bytes) {
+    int v = validate_config(cfg);
+    if (v) return v;
+    if (!bytes) return DFLASH_INVALID_ARG;
+    WsLayout L;
+    make_layout(*cfg, L);
+    *bytes = L.total;
+    return DFLASH_OK;
+}
+
+int dflash_create(const dflash_config* cfg, const dflash_weights* w, void* workspace, size_t ws_bytes,
+                  dflash_handle** out) {
+    int v = validate_config(cfg);
+    if (v) return v;
+    if (!w || !workspace || !out) return DFLASH_INVALID_ARG;
+    if ((uintptr_t)workspace & 1023) return DFLASH_INVALID_ARG;
+    const dflash_config& c = *cfg;
+    if (!w->w_fc || !w->g_fc || !w->embed || !w->lm_head || !w->g_final) return DFLASH_INVALID_ARG;
+    for (int l = 0; l < c.n_layers; ++l)
+        if (!w->g_in[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->g_post[l] || !w->w_gate[l] ||
+            !w->w_up[l] || !w->w_down[l])
+            return DFLASH_INVALID_ARG;
+    WsLayout L;
+    make_layout(c, L);
+    if (ws_bytes < L.total) return DFLASH_WORKSPACE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DFLASH_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DFLASH_CUDA;
+    if (prop.major != 10) return DFLASH_UNSUPPORTED;   // built for sm_100a only
+
+    dflash_handle* h = new (std::nothrow) dflash_handle();
+    if (!h) return DFLASH_CUDA;
+    h->cfg = c;
+    h->w = *w;
+    h->num_sms = prop.multiProcessorCount;
+    h->ws = (uint8_t*)workspace;
+    h->ws_bytes = ws_bytes;
+    h->L = L;
+    uint8_t* b = h->ws;
+    h->status = (int*)(b + L.status);
+    h->rope = (float2*)(b + L.rope);
+    h->x = b + L.x;
+    h->h = b + L.h;
+    h->q = b + L.q;
+    h->o = b + L.o;
+    h->act = b + L.act;
+    h->hf = b + L.hf;
+    h->y = b + L.y;
+    h->y32 = (float*)(b + L.y32);
+    h->lgs = (float*)(b + L.lgs);
+    h->part_o = (float*)(b + L.part_o);
+    h->part_ml = (float2*)(b + L.part_ml);
+    h->req_ok = (int*)(b + L.req_ok);
+    h->gpart = (float*)(b + L.gpart);
+    h->gcnt = (int*)(b + L.gcnt);
+    h->rec = (float4*)(b + L.rec);
+    h->launches = 0;
+
+    // RoPE table: angle p * theta^(-2i/d) in fp64, stored as fp32 (cos, sin).
+    const int half = c.head_dim / 2;
+    std::vector<float2> tab((size_t)c.max_position * half);
+    for (int i = 0; i < half; ++i) {
+        const double inv_freq = std::pow(c.rope_theta, -2.0 * i / c.head_dim);
+        for (long long pos = 0; pos < c.max_position; ++pos) {
+            const double ang = (double)pos * inv_freq;
+            tab[(size_t)pos * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+        }
+    }
+    cudaError_t e = cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(h->status, 0, 1024);
+    if (e == cudaSuccess) e = cudaMemset(h->req_ok, 0, (size_t)c.max_batch * 4);
+    if (e == cudaSuccess && L.n_counters > 0) e = cudaMemset(h->gcnt, 0, (size_t)L.n_counters * 4);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) {
+        delete h;
+        return DFLASH_CUDA;
+    }
+    if (c.dtype == DFLASH_BF16) {
+        const int H = c.hidden, d = c.head_dim, Nq = c.n_q_heads * d, Nkv = c.n_kv_heads * d, I = c.intermediate;
+        bool ok = encode_bf16_2d(&h->tm_wfc, w->w_fc, (uint64_t)c.n_sel * c.target_hidden, H,
+                                 (uint64_t)c.n_sel * c.target_hidden, 128) &&
+                  encode_bf16_2d(&h->tm_lm, w->lm_head, H, c.vocab, H, 128);
+        for (int l = 0; ok && l < c.n_layers; ++l) {
+            ok = encode_bf16_2d(&h->tm_wq[l], w->wq[l], H, Nq, H, 128) &&
+                 encode_bf16_2d(&h->tm_wk[l], w->wk[l], H, Nkv, H, 128) &&
+                 encode_bf16_2d(&h->tm_wv[l], w->wv[l], H, Nkv, H, 128) &&
+                 encode_bf16_2d(&h->tm_wo[l], w->wo[l], Nq, H, Nq, 128) &&
+                 encode_bf16_2d(&h->tm_wg[l], w->w_gate[l], H, I, H, 64) &&
+                 encode_bf16_2d(&h->tm_wu[l], w->w_up[l], H, I, H, 64) &&
+                 encode_bf16_2d(&h->tm_wd[l], w->w_down[l], I, H, I, 128);
+        }
+        if (!ok) {
+            delete h;
+            return get_encode() ? DFLASH_INVALID_ARG : DFLASH_CUDA;
+        }
+    }
+    *out = h;
+    return DFLASH_OK;
+}
+
+void dflash_destroy(dflash_handle* h) {
+    if (!h) return;
+    for (auto e : h->ev) cudaEventDestroy(e);
+    delete h;
+}
+
+int64_t dflash_launch_count(const dflash_handle* h) { return h ? h->launches : 0; }
+
+int dflash_cache_bytes(const dflash_handle* h, int batch, int capacity, size_t* bytes) {
+    if (!h || !bytes || batch < 1 || batch > h->cfg.max_batch || capacity < 1 || capacity > h->cfg.max_position)
+        return DFLASH_INVALID_ARG;
+    CacheLayout L;
+    cache_layout(h->cfg, batch, capacity, L);
+    *bytes = L.total;
+    return DFLASH_OK;
+}
+
+int dflash_cache_init(const dflash_handle* h, void* mem, size_t bytes, int batch, int capacity, dflash_cache** out,
+                      dflash_stream stream) {
+    if (!h || !mem || !out || batch < 1 || batch > h->cfg.max_batch || capacity < 1 ||
+        capacity > h->cfg.max_position)
+        return DFLASH_INVALID_ARG;
+    if ((uintptr_t)mem & 1023) return DFLASH_INVALID_ARG;
+    CacheLayout L;
+    cache_layout(h->cfg, batch, capacity, L);
+    if (bytes < L.total) return DFLASH_WORKSPACE;
+    const dflash_config& c = h->cfg;
+    dflash_cache* cc = new (std::nothrow) dflash_cache();
+    if (!cc) return DFLASH_CUDA;
+    cc->h = h;
+    cc->mem = (uint8_t*)mem;
+    cc->bytes = bytes;
+    cc->batch = batch;
+    cc->capacity = capacity;
+    cc->status = (int*)mem;
+    cc->len = (int*)((uint8_t*)mem + L.len);
+    cc->committed = (int*)((uint8_t*)mem + L.committed);
+    cc->slab = (uint8_t*)mem + L.slab;
+    cc->s_kv = (long long)capacity * c.head_dim;
+    cc->s_kind = cc->s_kv * c.n_kv_heads;
+    cc->s_layer = cc->s_kind * 2;
+    cc->s_req = cc->s_layer * c.n_layers;
+    if (c.dtype == DFLASH_BF16 && c.n_layers > 0) {
+        const uint64_t rows = (uint64_t)batch * cc->s_req / c.head_dim;
+        if (!encode_bf16_2d(&cc->tm_slab, cc->slab, c.head_dim, rows, c.head_dim, 64)) {
+            delete cc;
+            return DFLASH_CUDA;
+        }
+    }
+    if (cudaMemsetAsync(mem, 0, L.slab, S(stream)) != cudaSuccess) {
+        delete cc;
+        return DFLASH_CUDA;
+    }
+    *out = cc;
+    return DFLASH_OK;
+}
+
+void dflash_cache_release(dflash_cache* c) { delete c; }
+
+int dflash_cache_get_info(const dflash_cache* c, dflash_cache_info* info) {
+    if (!c || !info) return DFLASH_INVALID_ARG;
+    info->batch = c->batch;
+    info->capacity = c->capacity;
+    info->status = c->status;
+    info->len = c->len;
+    info->committed = c->committed;
+    info->slab = c->slab;
+    info->stride_kv = c->s_kv;
+    info->stride_kind = c->s_kind;
+    info->stride_layer = c->s_layer;
+    info->stride_request = c->s_req;
+    return DFLASH_OK;
+}
+
+int dflash_cache_set_len(dflash_cache* c, const int32_t* lens, dflash_stream stream) {
+    if (!c || !lens) return DFLASH_INVALID_ARG;
+    launch_set_len(lens, c->batch, c->capacity, c->len, c->committed, c->status, S(stream));
+    const_cast<dflash_handle*>(c->h)->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+int dflash_cache_status(dflash_handle* h, dflash_cache* c, dflash_stream stream) {
+    if (!h || !c || c->h != h) return DFLASH_INVALID_ARG;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DFLASH_CUDA;
+    int hs = 0, cs = 0;
+    if (cudaMemcpy(&hs, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return DFLASH_CUDA;
+    if (cudaMemcpy(&cs, c->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return DFLASH_CUDA;
+    if (cudaMemset(c->status, 0, 4) != cudaSuccess) return DFLASH_CUDA;
+    if (hs && cudaMemset(h->status, 0, 4) != cudaSuccess) return DFLASH_CUDA;
+    if (cudaStreamSynchronize(0) != cudaSuccess) return DFLASH_CUDA;
+    return hs ? hs : cs;
+}
+
+// ---------------------------------------------------------------------------
+// a1: fuse context
+// ---------------------------------------------------------------------------
+int dflash_fuse_context(dflash_handle* h, const void* const* hiddens, int64_t row_stride, int total_rows,
+                        void* ctx_out, dflash_stream stream) {
+    if (!h || !hiddens || !ctx_out || total_rows < 0 || total_rows > h->cfg.max_rows) return DFLASH_INVALID_ARG;
+    const dflash_config& c = h->cfg;
+    if (row_stride < c.target_hidden) return DFLASH_INVALID_ARG;
+    for (int i = 0; i < c.n_sel; ++i)
+        if (!hiddens[i]) return DFLASH_INVALID_ARG;
+    if (total_rows == 0) return DFLASH_OK;
+    cudaStream_t st = S(stream);
+    const int H = c.hidden;
+    if (c.dtype == DFLASH_BF16) {
+        if ((row_stride * 2) % 16 || !aligned16(ctx_out)) return DFLASH_INVALID_ARG;
+        for (int i = 0; i < c.n_sel; ++i)
+            if (!aligned16(hiddens[i])) return DFLASH_INVALID_ARG;
+        GemmParams p;
+        std::memset(&p, 0, sizeof(p));
+        const int nt = pick_nt(total_rows);
+        p.ta[0] = h->tm_wfc;
+        p.n_amat = 1;
+        p.amat[0].rows = H;
+        for (int i = 0; i < c.n_sel; ++i)
+            if (!act_map(&p.tb[i], hiddens[i], total_rows, c.target_hidden, row_stride, nt)) return DFLASH_INVALID_ARG;
+        p.kb_per_b = c.target_hidden / 64;
+        p.M = total_rows;
+        p.K = c.n_sel * c.target_hidden;
+        p.epi = EPI_BF16;
+        p.out = h->y;
+        p.ldo = H;
+        {
+            Timed t(h, TK_GEMM_FUSE, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+        Timed t(h, TK_RMSNORM, st);
+        launch_rmsnorm<__nv_bfloat16>((const __nv_bfloat16*)h->y, (const __nv_bfloat16*)h->w.g_fc,
+                                      (__nv_bfloat16*)ctx_out, total_rows, H, (float)c.rms_eps, total_rows, 0, 0, st);
+    } else {
+        Timed t(h, TK_SIMT_F32, st);
+        XSegs xs;
+        std::memset(&xs, 0, sizeof(xs));
+        for (int i = 0; i < c.n_sel; ++i) xs.ptr[i] = (const float*)hiddens[i];
+        xs.stride = row_stride;
+        xs.width = c.target_hidden;
+        launch_gemm_f32(xs, (const float*)h->w.w_fc, (float*)h->y, total_rows, H, c.n_sel * c.target_hidden, H, 0, st);
+        launch_rmsnorm<float>((const float*)h->y, (const float*)h->w.g_fc, (float*)ctx_out, total_rows, H,
+                              (float)c.rms_eps, total_rows, 0, 0, st);
+        h->launches += 1;
+    }
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// a2: inject KV
+// ---------------------------------------------------------------------------
+int dflash_inject_kv(dflash_handle* h, dflash_cache* cc, const void* ctx, const int32_t* row_start,
+                     const int32_t* row_count, int total_rows, dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !ctx || !row_start || !row_count || total_rows < 0 ||
+        total_rows > h->cfg.max_rows)
+        return DFLASH_INVALID_ARG;
+    if (total_rows == 0) return DFLASH_OK;
+    const dflash_config& c = h->cfg;
+    cudaStream_t st = S(stream);
+    const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
+    if (c.dtype == DFLASH_BF16) {
+        if (!aligned16(ctx)) return DFLASH_INVALID_ARG;
+        const int nt = pick_nt(total_rows);
+        CUtensorMap tb;
+        if (!act_map(&tb, ctx, total_rows, H, H, nt)) return DFLASH_INVALID_ARG;
+        for (int l0 = 0; l0 < c.n_layers; l0 += kMaxAMats / 2) {
+            const int nl = std::min(kMaxAMats / 2, c.n_layers - l0);
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            for (int i = 0; i < nl; ++i) {
+                p.ta[2 * i] = h->tm_wk[l0 + i];
+                p.ta[2 * i + 1] = h->tm_wv[l0 + i];
+                p.amat[2 * i].rows = Nkv;
+                p.amat[2 * i + 1].rows = Nkv;
+            }
+            p.n_amat = 2 * nl;
+            p.tb[0] = tb;
+            p.kb_per_b = cdiv(H, 64);
+            p.M = total_rows;
+            p.K = H;
+            p.epi = EPI_INJECT;
+            p.d = d;
+            p.cap = cc->capacity;
+            p.layer = l0;
+            p.batch = cc->batch;
+            p.len = cc->len;
+            p.rope = h->rope;
+            p.slab = (__nv_bfloat16*)cc->slab;
+            p.s_req = cc->s_req;
+            p.s_layer = cc->s_layer;
+            p.s_kind = cc->s_kind;
+            p.s_kv = cc->s_kv;
+            p.row_start = row_start;
+            p.row_count = row_count;
+            Timed t(h, TK_GEMM_INJECT, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+    } else {
+        Timed t(h, TK_SIMT_F32, st);
+        XSegs xs;
+        std::memset(&xs, 0, sizeof(xs));
+        xs.ptr[0] = (const float*)ctx;
+        xs.stride = H;
+        xs.width = H;
+        for (int l = 0; l < c.n_layers; ++l) {
+            launch_gemm_f32(xs, (const float*)h->w.wk[l], h->y32, total_rows, Nkv, H, 2 * Nkv, 0, st);
+            launch_gemm_f32(xs, (const float*)h->w.wv[l], h->y32, total_rows, Nkv, H, 2 * Nkv, Nkv, st);
+            launch_epi_inject_f32(h->y32, total_rows, Nkv, d, row_start, row_count, cc->batch, cc->len, cc->capacity,
+                                  h->rope, (float*)cc->slab, cc->s_req, cc->s_layer, cc->s_kind, cc->s_kv, l, st);
+            h->launches += 3;
+        }
+    }
+    Timed t(h, TK_INJECT_FINALIZE, st);
+    launch_inject_finalize(row_count, cc->batch, cc->capacity, cc->len, cc->status, st);
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// a3..a7: draft block
+// ---------------------------------------------------------------------------
+static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* drafts, float* logits, float* margin,
+                      cudaStream_t st) {
+    const dflash_config& c = h->cfg;
+    const int B = cc->batch, M = B * gamma, Mlm = B * (gamma - 1);
+    const int H = c.hidden, d = c.head_dim, Nq = c.n_q_heads * d, Nkv = c.n_kv_heads * d, I = c.intermediate;
+    typedef __nv_bfloat16 bf;
+    const int nt = pick_nt(M);
+    CUtensorMap tm_h, tm_o, tm_act, tm_hf;
+    if (!act_map(&tm_h, h->h, M, H, H, nt) || !act_map(&tm_o, h->o, M, Nq, Nq, nt) ||
+        !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)))
+        return DFLASH_CUDA;
+    int splits, chunk;
+    attn_plan(B, c.n_kv_heads, cc->capacity, splits, chunk);
+    AttnParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    ap.tmap = cc->tm_slab;
+    ap.q = (const bf*)h->q;
+    ap.len = cc->len;
+    ap.req_ok = h->req_ok;
+    ap.part_o = h->part_o;
+    ap.part_ml = h->part_ml;
+    ap.gamma = gamma;
+    ap.G = c.n_q_heads / c.n_kv_heads;
+    ap.nq = c.n_q_heads;
+    ap.nkv = c.n_kv_heads;
+    ap.splits = splits;
+    ap.chunk = chunk;
+    ap.rows_kv = cc->s_kv / d;
+    ap.rows_kind = cc->s_kind / d;
+    ap.rows_layer = cc->s_layer / d;
+    ap.rows_req = cc->s_req / d;
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    ap.status = h->status;
+
+    for (int l = 0; l < c.n_layers; ++l) {
+        {
+            Timed t(h, TK_RMSNORM, st);
+            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_in[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st);
+            h->launches += 1;
+        }
+        {   // QKV + RoPE; block K/V to cache scratch rows [len, len + gamma)
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            p.ta[0] = h->tm_wq[l];
+            p.ta[1] = h->tm_wk[l];
+            p.ta[2] = h->tm_wv[l];
+            p.amat[0].rows = Nq;
+            p.amat[1].rows = Nkv;
+            p.amat[2].rows = Nkv;
+            p.n_amat = 3;
+            p.tb[0] = tm_h;
+            p.kb_per_b = cdiv(H, 64);
+            p.M = M;
+            p.K = H;
+            p.epi = EPI_QKV;
+            p.out = h->q;
+            p.ldo = Nq;
+            p.d = d;
+            p.gamma = gamma;
+            p.cap = cc->capacity;
+            p.layer = l;
+            p.batch = B;
+            p.len = cc->len;
+            p.req_ok = h->req_ok;
+            p.rope = h->rope;
+            p.slab = (bf*)cc->slab;
+            p.s_req = cc->s_req;
+            p.s_layer = cc->s_layer;
+            p.s_kind = cc->s_kind;
+            p.s_kv = cc->s_kv;
+            Timed t(h, TK_GEMM_QKV, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+        ap.layer = l;
+        {
+            Timed t(h, TK_ATTENTION, st);
+            int e = launch_attention(ap, d, B, st, (bf*)h->o, &h->launches);
+            if (e) return DFLASH_CUDA;
+        }
+        {   // O-proj + residual
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            p.ta[0] = h->tm_wo[l];
+            p.amat[0].rows = H;
+            p.n_amat = 1;
+            p.tb[0] = tm_o;
+            p.kb_per_b = cdiv(Nq, 64);
+            p.M = M;
+            p.K = Nq;
+            p.epi = EPI_RESID;
+            p.out = h->x;
+            p.ldo = H;
+            Timed t(h, TK_GEMM_O, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+        {
+            Timed t(h, TK_RMSNORM, st);
+            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_post[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st);
+            h->launches += 1;
+        }
+        {   // gate/up + SwiGLU
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            p.ta[0] = h->tm_wg[l];
+            p.ta[1] = h->tm_wu[l];
+            p.n_amat = 2;
+            p.swiglu = 1;
+            p.n_tiles = I / 64;
+            p.tb[0] = tm_h;
+            p.kb_per_b = cdiv(H, 64);
+            p.M = M;
+            p.K = H;
+            p.epi = EPI_SWIGLU;
+            p.out = h->act;
+            p.ldo = I;
+            Timed t(h, TK_GEMM_SWIGLU, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+        {   // down + residual
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            p.ta[0] = h->tm_wd[l];
+            p.amat[0].rows = H;
+            p.n_amat = 1;
+            p.tb[0] = tm_act;
+            p.kb_per_b = cdiv(I, 64);
+            p.M = M;
+            p.K = I;
+            p.epi = EPI_RESID;
+            p.out = h->x;
+            p.ldo = H;
+            Timed t(h, TK_GEMM_DOWN, st);
+            int r = run_gemm(h, p, nt, st);
+            if (r) return r;
+        }
+    }
+    {
+        Timed t(h, TK_RMSNORM, st);
+        launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_final, (bf*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1,
+                           gamma, 1, st);
+        h->launches += 1;
+    }
+    {   // shared LM head + per-tile top-2
+        GemmParams p;
+        std::memset(&p, 0, sizeof(p));
+        p.ta[0] = h->tm_lm;
+        p.amat[0].rows = c.vocab;
+        p.n_amat = 1;
+        p.tb[0] = tm_hf;
+        p.kb_per_b = cdiv(H, 64);
+        p.M = Mlm;
+        p.K = H;
+        p.epi = EPI_LMHEAD;
+        p.vocab = c.vocab;
+        p.logits = logits;
+        p.records = h->rec;
+        Timed t(h, TK_GEMM_LMHEAD, st);
+        int r = run_gemm(h, p, pick_nt(Mlm), st);
+        if (r) return r;
+    }
+    Timed t(h, TK_LM_REDUCE, st);
+    launch_lm_reduce(h->rec, cdiv(c.vocab, 128), Mlm, gamma - 1, h->req_ok, drafts, margin, st);
+    h->launches += 1;
+    return DFLASH_OK;
+}
+
+static int draft_f32(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* drafts, float* logits, float* margin,
+                     cudaStream_t st) {
+    const dflash_config& c = h->cfg;
+    const int B = cc->batch, M = B * gamma, Mlm = B * (gamma - 1);
+    const int H = c.hidden, d = c.head_dim, Nq = c.n_q_heads * d, Nkv = c.n_kv_heads * d, I = c.intermediate;
+    const int ldq = Nq + 2 * Nkv;
+    Timed t(h, TK_SIMT_F32, st);
+    float *x = (float*)h->x, *hh = (float*)h->h, *q = (float*)h->q, *o = (float*)h->o, *act = (float*)h->act;
+    XSegs xh{}, xo{}, xa{}, xf{};
+    xh.ptr[0] = hh; xh.stride = H; xh.width = H;
+    xo.ptr[0] = o; xo.stride = Nq; xo.width = Nq;
+    xa.ptr[0] = act; xa.stride = I; xa.width = I;
+    xf.ptr[0] = (float*)h->hf; xf.stride = H; xf.width = H;
+    for (int l = 0; l < c.n_layers; ++l) {
+        launch_rmsnorm<float>(x, (const float*)h->w.g_in[l], hh, M, H, (float)c.rms_eps, M, 0, 0, st);
+        launch_gemm_f32(xh, (const float*)h->w.wq[l], h->y32, M, Nq, H, ldq, 0, st);
+        launch_gemm_f32(xh, (const float*)h->w.wk[l], h->y32, M, Nkv, H, ldq, Nq, st);
+        launch_gemm_f32(xh, (const float*)h->w.wv[l], h->y32, M, Nkv, H, ldq, Nq + Nkv, st);
+        launch_epi_qkv_f32(h->y32, M, Nq, Nkv, d, gamma, cc->len, h->req_ok, h->rope, q, (float*)cc->slab, cc->s_req,
+                           cc->s_layer, cc->s_kind, cc->s_kv, l, st);
+        int e = launch_attn_f32(q, (const float*)cc->slab, cc->len, h->req_ok, o, B, gamma, c.n_q_heads,
+                                c.n_q_heads / c.n_kv_heads, d, cc->s_req, cc->s_layer, cc->s_kind, cc->s_kv, l,
+                                cc->capacity, st);
+        if (e) return DFLASH_CUDA;
+        launch_gemm_f32(xo, (const float*)h->w.wo[l], h->y32, M, H, Nq, H, 0, st);
+        launch_resid_f32(x, h->y32, (long long)M * H, st);
+        launch_rmsnorm<float>(x, (const float*)h->w.g_post[l], hh, M, H, (float)c.rms_eps, M, 0, 0, st);
+        launch_gemm_f32(xh, (const float*)h->w.w_gate[l], h->y32, M, I, H, 2 * I, 0, st);
+        launch_gemm_f32(xh, (const float*)h->w.w_up[l], h->y32, M, I, H, 2 * I, I, st);
+        launch_swiglu_f32(h->y32, act, M, I, st);
+        launch_gemm_f32(xa, (const float*)h->w.w_down[l], h->y32, M, H, I, H, 0, st);
+        launch_resid_f32(x, h->y32, (long long)M * H, st);
+        h->launches += 14;
+    }
+    launch_rmsnorm<float>(x, (const float*)h->w.g_final, (float*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1, gamma, 1,
+                          st);
+    float* lg = logits ? logits : h->lgs;
+    launch_gemm_f32(xf, (const float*)h->w.lm_head, lg, Mlm, c.vocab, H, c.vocab, 0, st);
+    launch_top2_rows(lg, Mlm, c.vocab, gamma - 1, h->req_ok, drafts, margin, st);
+    h->launches += 3;
+    return DFLASH_OK;
+}
+
+int dflash_draft_block(dflash_handle* h, dflash_cache* cc, const int32_t* anchor, int gamma, int32_t* drafts,
+                       float* logits_opt, float* margin_opt, dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !anchor || gamma < 1 || gamma > h->cfg.max_gamma) return DFLASH_INVALID_ARG;
+    if (gamma > 1 && !drafts) return DFLASH_INVALID_ARG;
+    const dflash_config& c = h->cfg;
+    cudaStream_t st = S(stream);
+    {
+    Timed t(h, TK_EMBED, st);
+    if (c.dtype == DFLASH_BF16)
+        launch_embed<__nv_bfloat16>((const __nv_bfloat16*)h->w.embed, anchor, c.mask_id, cc->batch, gamma, c.hidden,
+                                    c.vocab, cc->len, cc->committed, cc->capacity, (__nv_bfloat16*)h->x, h->req_ok,
+                                    cc->status, st);
+    else
+        launch_embed<float>((const float*)h->w.embed, anchor, c.mask_id, cc->batch, gamma, c.hidden, c.vocab, cc->len,
+                            cc->committed, cc->capacity, (float*)h->x, h->req_ok, cc->status, st);
+    h->launches += 1;
+    }
+    if (gamma == 1) return cuda_status(cudaGetLastError());
+    int r = c.dtype == DFLASH_BF16 ? draft_bf16(h, cc, gamma, drafts, logits_opt, margin_opt, st)
+                                   : draft_f32(h, cc, gamma, drafts, logits_opt, margin_opt, st);
+    if (r) return r;
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// a8: accept
+// ---------------------------------------------------------------------------
+int dflash_accept(dflash_handle* h, dflash_cache* cc, const int32_t* drafts, const int32_t* target, int gamma,
+                  int32_t* accept_len, int32_t* next_anchor, dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !target || !accept_len || !next_anchor || gamma < 1 || gamma > h->cfg.max_gamma)
+        return DFLASH_INVALID_ARG;
+    if (gamma > 1 && !drafts) return DFLASH_INVALID_ARG;
+    Timed t(h, TK_ACCEPT, st_of(stream));
+    launch_accept(drafts ? drafts : target, target, cc->batch, gamma, h->cfg.vocab, cc->len, cc->committed, accept_len,
+                  next_anchor, cc->status, S(stream));
+    h->launches += 1;
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostics
+// ---------------------------------------------------------------------------
+const char* dflash_diag_arch(void) { return "sm_100a"; }
+
+int dflash_diag_partition(int64_t units, int kb, int ctas, int64_t tile, int* first_cta, int* n_contrib) {
+    if (units <= 0 || kb <= 0 || units % kb || ctas <= 0 || ctas > units || tile < 0 || tile * kb >= units || !first_cta ||
+        !n_contrib)
+        return DFLASH_INVALID_ARG;
+    *first_cta = sk_first_cta(tile, kb, units, ctas);
+    *n_contrib = sk_n_contrib(tile, kb, units, ctas);
+    return DFLASH_OK;
+}
+
+int dflash_diag_gemm_scratch_bytes(int M, int N, int K, size_t* bytes) {
+    if (!bytes || M < 1 || M > 4096 || N < 1 || K < 8 || K % 8) return DFLASH_INVALID_ARG;
+    const int nt = pick_nt(M);
+    const size_t counters = (size_t)cdiv(N, 128) * cdiv(M, nt) * 4;
+    *bytes = al(counters, 256) + gemm_partial_bytes(kMaxCtas, nt);
+    return DFLASH_OK;
+}
+
+int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
+                          size_t scratch_bytes, int grid, dflash_stream stream) {
+    size_t need = 0;
+    if (dflash_diag_gemm_scratch_bytes(M, N, K, &need) != DFLASH_OK) return DFLASH_INVALID_ARG;
+    if (!X || !W || !Y || !scratch || ((uintptr_t)scratch & 255)) return DFLASH_INVALID_ARG;
+    if (scratch_bytes < need) return DFLASH_WORKSPACE;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFLASH_CUDA;
+    const int nt = pick_nt(M);
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!encode_bf16_2d(&p.ta[0], W, K, N, K, 128) || !encode_bf16_2d(&p.tb[0], X, K, M, K, nt))
+        return DFLASH_INVALID_ARG;
+    p.amat[0].rows = N;
+    p.n_amat = 1;
+    p.kb_per_b = cdiv(K, 64);
+    p.M = M;
+    p.K = K;
+    p.epi = EPI_F32;
+    p.out = Y;
+    p.ldo = N;
+    const size_t counters = al((size_t)cdiv(N, 128) * cdiv(M, nt) * 4, 256);
+    p.counters = (int*)scratch;
+    p.partial = (float*)((uint8_t*)scratch + counters);
+    p.status = nullptr;
+    p.ctas = grid > 0 ? std::min(grid, kMaxCtas) : 0;
+    int e = launch_gemm_tc(p, nt, std::min(sms, kMaxCtas), S(stream));
+    return e == 0 ? DFLASH_OK : DFLASH_CUDA;
+}
+
+int dflash_diag_synth_target(const int32_t* drafts, const int32_t* a_plan, const int32_t* rand_tokens, int batch,
+                             int gamma, int vocab, int32_t* target, dflash_stream stream) {
+    if (!a_plan || !rand_tokens || !target || batch < 1 || gamma < 1 || vocab < 2) return DFLASH_INVALID_ARG;
+    if (gamma > 1 && !drafts) return DFLASH_INVALID_ARG;
+    launch_synth_target(drafts ? drafts : a_plan, a_plan, rand_tokens, batch, gamma, vocab, target, S(stream));
+    return cuda_status(cudaGetLastError());
+}
+
+int dflash_diag_timing_enable(dflash_handle* h, int max_launches) {
+    if (!h || max_launches < 1 || max_launches > (1 << 20)) return DFLASH_INVALID_ARG;
+    for (auto e : h->ev) cudaEventDestroy(e);
+    h->ev.assign(2 * (size_t)max_launches, nullptr);
+    h->ev_kind.assign(max_launches, -1);
+    for (auto& e : h->ev)
+        if (cudaEventCreate(&e) != cudaSuccess) return DFLASH_CUDA;
+    h->ev_used = 0;
+    h->timing = true;
+    return DFLASH_OK;
+}
+
+int dflash_diag_timing_read(dflash_handle* h, dflash_stream stream, int* kinds, float* ms, int max_entries,
+                            int* n_entries) {
+    if (!h || !kinds || !ms || !n_entries || max_entries < 0) return DFLASH_INVALID_ARG;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DFLASH_CUDA;
+    const int n = std::min(h->ev_used / 2, max_entries);
+    for (int i = 0; i < n; ++i) {
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, h->ev[2 * i], h->ev[2 * i + 1]) != cudaSuccess) return DFLASH_CUDA;
+        kinds[i] = h->ev_kind[i];
+        ms[i] = t;
+    }
+    *n_entries = n;
+    h->ev_used = 0;
+    return DFLASH_OK;
+}
+
+int dflash_diag_timing_disable(dflash_handle* h) {
+    if (!h) return DFLASH_INVALID_ARG;
+    h->timing = false;
+    for (auto e : h->ev) cudaEventDestroy(e);
+    h->ev.clear();
+    h->ev_kind.clear();
+    h->ev_used = 0;
+    return DFLASH_OK;
+}
+
+const char* dflash_diag_timed_name(int kind) { return (kind >= 0 && kind < TK_COUNT) ? kTimedNames[kind] : "?"; }
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+// Persistent split-K tensor-core GEMM of libdflash: parameters, the work
+// partition (shared by host and device), and the launcher's interface.
+//
+// Every projection of the draft step is Y[m, n] = sum_k X[m, k] W[n, k] with
+// the weights W streamed from HBM once and the tokens X few (16 rows at batch
+// 1).  The kernel computes it "swap-AB": a 128-row weight tile is the tcgen05 A
+// operand (M = 128), NT tokens are the B operand (N = NT), the fp32 tile lives
+// in TMEM.  Work units are k-blocks of 64 along K of every output tile; the
+// grid's CTAs take equal contiguous ranges of units (a range may start or end
+// inside a tile), so all SMs stream the same number of weight bytes whatever
+// the shape.  A tile split across CTAs is finished by the CTA that arrives
+// last on the tile's counter; it adds the fp32 partials in contributor order,
+// so the result does not depend on arrival order.  No CTA ever waits for
+// another.
+#pragma once
+#include "common.cuh"
+
+namespace df {
+
+enum EpiKind : int {
+    EPI_F32 = 0,     // out fp32[m, n] = acc
+    EPI_BF16 = 1,    // out bf16[m, n] = R(acc)
+    EPI_RESID = 2,   // out bf16[m, n] = R(out + acc)            (O-proj, down-proj)
+    EPI_QKV = 3,     // q = R(RoPE(acc)) -> q buffer; k = R(RoPE(acc)), v = R(acc) -> cache scratch
+    EPI_SWIGLU = 4,  // out bf16[m, f] = R(silu(gate) * up)     (A tile = 64 gate rows + 64 up rows)
+    EPI_INJECT = 5,  // K = R(RoPE(acc)), V = R(acc) -> cache rows of the owning request
+    EPI_LMHEAD = 6,  // per 128-vocab tile and token: top-1 (value, id) and top-2 value; optional fp32 logits
+};
+
+constexpr int kMaxAMats = 10;   // weight matrices stacked in one A operand
+constexpr int kMaxBMaps = 8;    // activation tensor maps concatenated along K
+
+struct GemmAMat {
+    int rows;    // rows of this weight matrix
+    int tile0;   // first n-tile of this matrix
+    int ntiles;  // n-tiles of this matrix
+    int feat0;   // unused by the kernel; global feature offset for callers
+};
+
+struct GemmParams {
+    CUtensorMap ta[kMaxAMats];   // weight maps, box {64, 128} (SwiGLU: {64, 64})
+    CUtensorMap tb[kMaxBMaps];   // activation maps, box {64, NT}
+    GemmAMat amat[kMaxAMats];
+    int n_amat;
+    int swiglu;                  // A = rows [64t, 64t+64) of ta[0] then of ta[1]
+    int kb_per_b;                // k-blocks served by one activation map
+    int M, K, KB;                // tokens, reduction length, k-blocks per tile
+    int n_tiles, m_tiles;
+    long long units;             // n_tiles * m_tiles * KB
+    int ctas;
+    float* partial;              // [2 * ctas][NT][128] fp32 split-tile partials
+    int* counters;               // [n_tiles * m_tiles], zero between launches
+    int* status;                 // handle status word (DFLASH_TIMEOUT)
+    int epi;
+    void* out;                   // EPI_F32 / BF16 / RESID / SWIGLU output, EPI_QKV q buffer
+    int ldo;                     // its row stride in elements
+    // EPI_QKV / EPI_INJECT
+    int d, gamma, cap, layer, batch;
+    const int* len;
+    const int* req_ok;
+    const float2* rope;          // [max_position][d/2] (cos, sin)
+    __nv_bfloat16* slab;
+    long long s_req, s_layer, s_kind, s_kv;
+    const int* row_start;
+    const int* row_count;
+    // EPI_LMHEAD
+    int vocab;
+    float* logits;               // [M, vocab] or null
+    float4* records;             // [n_tiles][M]: (top1, id bits, top2, 0)
+};
+
+// ---------------------------------------------------------------------------
+// Work partition.  CTA p owns units [begin(p), begin(p+1)), begin(p) = p*U/P.
+// Requires U >= P so that no CTA is empty.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline long long sk_begin(int p, long long U, int P) {
+    return (long long)p * U / P;
+}
+// The CTA that owns unit u: the largest p with begin(p) <= u, i.e.
+// p = ceil((u+1) P / U) - 1.
+__host__ __device__ inline int sk_owner(long long u, long long U, int P) {
+    return (int)(((u + 1) * (long long)P - 1) / U);
+}
+__host__ __device__ inline int sk_first_cta(long long tile, int KB, long long U, int P) {
+    return sk_owner(tile * KB, U, P);
+}
+__host__ __device__ inline int sk_n_contrib(long long tile, int KB, long long U, int P) {
+    return sk_owner((tile + 1) * KB - 1, U, P) - sk_owner(tile * KB, U, P) + 1;
+}
+// Partial slot of CTA p's segment of `tile`: a CTA has at most two split
+// segments, its first (slot 2p) and its last (slot 2p+1); every segment in
+// between covers a whole tile and needs no partial.
+__host__ __device__ inline int sk_slot(int p, long long tile, int KB, long long U, int P) {
+    long long first_tile = sk_begin(p, U, P) / KB;
+    return 2 * p + (tile == first_tile ? 0 : 1);
+}
+
+// Tokens per MMA tile for M rows.
+inline int pick_nt(int M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+// Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
+// ctas) and launches on `stream`.  Returns a cudaError_t.
+int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream);
+
+// Bytes of split-tile partial scratch for ctas CTAs at tile width nt.
+inline size_t gemm_partial_bytes(int ctas, int nt) { return (size_t)2 * ctas * nt * 128 * sizeof(float); }
+
+}  // namespace df

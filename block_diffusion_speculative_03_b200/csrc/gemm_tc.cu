@@ -1,0 +1,445 @@
+// Persistent split-K tcgen05 GEMM with fused epilogues (see gemm.cuh).
+//
+// CTA = 6 warps:  warp 0 lane 0 issues TMA loads of (weight tile, token tile)
+// pairs into an S-stage shared-memory ring; warp 1 lane 0 issues tcgen05.mma
+// (M=128, N=NT, K=16, bf16 in, fp32 accumulate) into one of two TMEM
+// accumulator buffers; warps 2..5 (128 threads, one TMEM lane each) drain a
+// finished accumulator with tcgen05.ld, resolve split tiles, and run the
+// epilogue while the next tile accumulates in the other buffer.
+#include "gemm.cuh"
+
+namespace df {
+
+template <int NT>
+struct GemmCfg {
+    static constexpr int A_BYTES = 128 * 128;            // 128 rows x 64 bf16
+    static constexpr int B_BYTES = NT * 128;             // NT rows x 64 bf16
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int CH = NT < 32 ? NT : 32;         // epilogue column chunk
+    static constexpr int XCH_FLOATS = 128 * 33;
+    static constexpr int MISC_BYTES = 4096;
+    static constexpr int BUDGET = 232448 - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
+    static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCH_FLOATS * 4 + MISC_BYTES;
+    static constexpr uint32_t TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
+};
+
+DF_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// Top-2 merge: a <- top2(a ∪ b); ties of the top value go to the lower id.
+DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
+    if (b1 > a1 || (b1 == a1 && bi < ai)) {
+        a2 = fmaxf(a1, b2);
+        a1 = b1;
+        ai = bi;
+    } else {
+        a2 = fmaxf(a2, b1);
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
+    using C = GemmCfg<NT>;
+    constexpr int S = C::STAGES;
+    constexpr int CH = C::CH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S * C::A_BYTES;
+    float* xch = (float*)(sB + S * C::B_BYTES);
+    uint64_t* full = (uint64_t*)(xch + C::XCH_FLOATS);
+    uint64_t* empty = full + S;
+    uint64_t* accf = empty + S;
+    uint64_t* acce = accf + 2;
+    uint64_t* drain = acce + 2;
+    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    int* s_flag = (int*)(tmem_slot + 2);
+    int* tok_b = s_flag + 1;          // [NT]
+    int* tok_pos = tok_b + NT;        // [NT]
+    float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < p.n_amat; ++i) tma_prefetch_desc(&p.ta[i]);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const long long U = p.units;
+    const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
+    const long long u_begin = sk_begin(cta, U, P), u_end = sk_begin(cta + 1, U, P);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol_w = make_l2_policy_evict_first();
+            int stage = 0;
+            uint32_t round = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const long long t = u / KB;
+                const int kb0 = (int)(u % KB);
+                const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+                const int n_tile = (int)(t / m_tiles), m_tile = (int)(t % m_tiles);
+                int mi = 0;
+                if (!p.swiglu)
+                    while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
+                const int arow = p.swiglu ? n_tile * 64 : (n_tile - p.amat[mi].tile0) * 128;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&empty[stage], (round & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                    uint8_t* a = sA + stage * C::A_BYTES;
+                    uint8_t* b = sB + stage * C::B_BYTES;
+                    if (p.swiglu) {
+                        tma_load_2d_hint(a, &p.ta[0], &full[stage], kb * 64, arow, pol_w);
+                        tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[stage], kb * 64, arow, pol_w);
+                    } else {
+                        tma_load_2d_hint(a, &p.ta[mi], &full[stage], kb * 64, arow, pol_w);
+                    }
+                    const int bm = kb / p.kb_per_b;
+                    tma_load_2d(b, &p.tb[bm], &full[stage], (kb - bm * p.kb_per_b) * 64, m_tile * NT);
+                    ++issued;
+                    if (++stage == S) { stage = 0; ++round; }
+                }
+                u += kb1 - kb0;
+            }
+            if (*abort_flag) {
+                // Let the copies already issued land before the CTA exits.
+                long long first = issued > S ? issued - S : 0;
+                for (long long i = first; i < issued; ++i) {
+                    volatile int never = 0;
+                    mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), &never, nullptr);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(128, NT);
+            int stage = 0, seg = 0;
+            uint32_t round = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const int kb0 = (int)(u % KB);
+                const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+                const int buf = seg & 1;
+                const uint32_t use = (uint32_t)(seg >> 1);
+                if (!mbar_wait(&acce[buf], (use & 1) ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * NT);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], round & 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+                    const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc_mma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    if (++stage == S) { stage = 0; ++round; }
+                }
+                if (!ok) break;
+                tc_commit(&accf[buf]);
+                ++seg;
+                u += kb1 - kb0;
+            }
+            if (*abort_flag) {
+                // Drain the MMAs already issued before TMEM is released.
+                tc_commit(drain);
+                volatile int never = 0;
+                mbar_wait(drain, 0, &never, nullptr);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quadrant of this warp
+        const int row = q * 32 + lane;          // weight-tile row = TMEM lane
+        const int e = threadIdx.x - 64;         // 0..127
+        int seg = 0;
+        for (long long u = u_begin; u < u_end;) {
+            const long long t = u / KB;
+            const int kb0 = (int)(u % KB);
+            const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+            const int n_tile = (int)(t / m_tiles), m_tile = (int)(t % m_tiles);
+            const int buf = seg & 1;
+            const uint32_t use = (uint32_t)(seg >> 1);
+            const bool ok = mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
+            if (named_bar_or(1, 128, !ok)) break;   // leave together: later named barriers stay matched
+            tc_fence_after();
+            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
+            const bool whole = (kb0 == 0 && kb1 == KB);
+            bool finish = true;
+            int first = cta, nc = 1;
+            if (!whole) {
+                first = sk_first_cta(t, KB, U, P);
+                nc = sk_n_contrib(t, KB, U, P);
+                float* dst = p.partial + (size_t)sk_slot(cta, t, KB, U, P) * NT * 128;
+#pragma unroll 1
+                for (int c0 = 0; c0 < NT; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tb + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) __stcg(dst + (c0 + i) * 128 + row, v[i]);
+                }
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (e == 0) {
+                    int old = atomicAdd(&p.counters[t], 1);
+                    *s_flag = (old == nc - 1) ? 1 : 0;
+                }
+                named_bar_sync(1, 128);
+                finish = (*s_flag != 0);
+                if (finish) __threadfence();
+            }
+            if (finish) {
+                // Weight-row -> output-feature mapping of this tile.
+                int mi = 0;
+                if (!p.swiglu)
+                    while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
+                const int lr = p.swiglu ? 0 : (n_tile - p.amat[mi].tile0) * 128 + row;
+                const bool row_ok = p.swiglu ? true : (lr < p.amat[mi].rows);
+                // Per-token request / position for the cache-writing epilogues.
+                if (p.epi == EPI_QKV || p.epi == EPI_INJECT) {
+                    named_bar_sync(1, 128);
+                    for (int te = e; te < NT; te += 128) {   // NT may exceed the 128 epilogue threads
+                        const int m = m_tile * NT + te;
+                        int b = -1, pos = -1;
+                        if (m < p.M) {
+                            if (p.epi == EPI_QKV) {
+                                const int bb = m / p.gamma;
+                                if (p.req_ok[bb]) { b = bb; pos = p.len[bb] + (m - bb * p.gamma); }
+                            } else {
+                                for (int bb = 0; bb < p.batch; ++bb) {
+                                    const int rs = p.row_start[bb], rc = p.row_count[bb];
+                                    if (m >= rs && m < rs + rc) {
+                                        const int L0 = p.len[bb];
+                                        if (L0 + rc <= p.cap) { b = bb; pos = L0 + (m - rs); }
+                                        break;
+                                    }
+                                }
+                            }
+                        }
+                        if (pos < 0 || pos >= p.cap) b = -1;   // never write outside the request's slab
+                        tok_b[te] = b;
+                        tok_pos[te] = pos;
+                    }
+                    named_bar_sync(1, 128);
+                }
+#pragma unroll 1
+                for (int c0 = 0; c0 < NT; c0 += CH) {
+                    float v[CH];
+#pragma unroll
+                    for (int h = 0; h < CH; h += 16) tmem_ld16(tb + c0 + h, v + h);
+                    if (!whole) {
+                        float acc[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) acc[i] = 0.0f;
+                        for (int ci = 0; ci < nc; ++ci) {
+                            const int pc = first + ci;
+                            if (pc == cta) {
+#pragma unroll
+                                for (int i = 0; i < CH; ++i) acc[i] += v[i];
+                            } else {
+                                const float* src = p.partial + (size_t)sk_slot(pc, t, KB, U, P) * NT * 128;
+#pragma unroll
+                                for (int i = 0; i < CH; ++i) acc[i] += __ldcg(src + (c0 + i) * 128 + row);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) v[i] = acc[i];
+                    }
+                    // ---------------------------------------------- epilogues
+                    const int mbase = m_tile * NT + c0;
+                    switch (p.epi) {
+                    case EPI_F32: {
+                        float* o = (float*)p.out;
+                        if (row_ok)
+                            for (int i = 0; i < CH; ++i)
+                                if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = v[i];
+                        break;
+                    }
+                    case EPI_BF16: {
+                        __nv_bfloat16* o = (__nv_bfloat16*)p.out;
+                        if (row_ok)
+                            for (int i = 0; i < CH; ++i)
+                                if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = f2bf(v[i]);
+                        break;
+                    }
+                    case EPI_RESID: {
+                        __nv_bfloat16* o = (__nv_bfloat16*)p.out;
+                        if (row_ok)
+                            for (int i = 0; i < CH; ++i)
+                                if (mbase + i < p.M) {
+                                    __nv_bfloat16* po = o + (size_t)(mbase + i) * p.ldo + lr;
+                                    *po = f2bf(bf2f(*po) + v[i]);
+                                }
+                        break;
+                    }
+                    case EPI_SWIGLU: {
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) xch[row * 33 + i] = v[i];
+                        named_bar_sync(1, 128);
+                        if (row < 64) {
+                            __nv_bfloat16* o = (__nv_bfloat16*)p.out;
+                            const int f = n_tile * 64 + row;
+                            for (int i = 0; i < CH; ++i)
+                                if (mbase + i < p.M) {
+                                    const float up = xch[(row + 64) * 33 + i];
+                                    o[(size_t)(mbase + i) * p.ldo + f] = f2bf(silu(v[i]) * up);
+                                }
+                        }
+                        named_bar_sync(1, 128);
+                        break;
+                    }
+                    case EPI_QKV:
+                    case EPI_INJECT: {
+                        // Section of this weight matrix: QKV -> 0 q, 1 k, 2 v;
+                        // inject -> (layer, kind) = (mi / 2, mi % 2).
+                        const bool is_q = (p.epi == EPI_QKV && mi == 0);
+                        const int kind = (p.epi == EPI_QKV) ? mi - 1 : (mi & 1);
+                        const int layer = (p.epi == EPI_QKV) ? p.layer : p.layer + (mi >> 1);
+                        const bool rotate = is_q || kind == 0;
+                        const int d = p.d, half = d >> 1;
+                        const int i_in = lr % d;
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) xch[row * 33 + i] = v[i];
+                        named_bar_sync(1, 128);
+                        const int prow = (i_in < half) ? row + half : row - half;
+                        if (row_ok) {
+                            for (int i = 0; i < CH; ++i) {
+                                const int b = tok_b[c0 + i];
+                                if (b < 0) continue;
+                                const int pos = tok_pos[c0 + i];
+                                float x = v[i];
+                                if (rotate) {
+                                    const float pr = xch[prow * 33 + i];
+                                    const float2 cs = p.rope[(size_t)pos * half + (i_in % half)];
+                                    x = (i_in < half) ? (x * cs.x - pr * cs.y) : (x * cs.x + pr * cs.y);
+                                }
+                                if (is_q) {
+                                    ((__nv_bfloat16*)p.out)[(size_t)(mbase + i) * p.ldo + lr] = f2bf(x);
+                                } else {
+                                    const int g = lr / d;
+                                    p.slab[(size_t)b * p.s_req + (size_t)layer * p.s_layer + (size_t)kind * p.s_kind +
+                                           (size_t)g * p.s_kv + (size_t)pos * d + i_in] = f2bf(x);
+                                }
+                            }
+                        }
+                        named_bar_sync(1, 128);
+                        break;
+                    }
+                    case EPI_LMHEAD: {
+                        const int vid = lr;   // vocab id (lm_head is one matrix)
+#pragma unroll 1
+                        for (int i = 0; i < CH; ++i) {
+                            const int m = mbase + i;
+                            if (p.logits && row_ok && m < p.M) p.logits[(size_t)m * p.vocab + vid] = v[i];
+                            float a1 = row_ok ? v[i] : -INFINITY, a2 = -INFINITY;
+                            int ai = row_ok ? vid : 0x7fffffff;
+#pragma unroll
+                            for (int off = 16; off > 0; off >>= 1) {
+                                const float b1 = __shfl_xor_sync(0xffffffffu, a1, off);
+                                const int bi = __shfl_xor_sync(0xffffffffu, ai, off);
+                                const float b2 = __shfl_xor_sync(0xffffffffu, a2, off);
+                                top2_merge(a1, ai, a2, b1, bi, b2);
+                            }
+                            if (lane == 0) {
+                                lmred[(q * CH + i) * 3 + 0] = a1;
+                                lmred[(q * CH + i) * 3 + 1] = __int_as_float(ai);
+                                lmred[(q * CH + i) * 3 + 2] = a2;
+                            }
+                        }
+                        named_bar_sync(1, 128);
+                        if (e < CH && mbase + e < p.M) {
+                            float a1 = lmred[e * 3 + 0], a2 = lmred[e * 3 + 2];
+                            int ai = __float_as_int(lmred[e * 3 + 1]);
+                            for (int qq = 1; qq < 4; ++qq)
+                                top2_merge(a1, ai, a2, lmred[(qq * CH + e) * 3 + 0],
+                                           __float_as_int(lmred[(qq * CH + e) * 3 + 1]), lmred[(qq * CH + e) * 3 + 2]);
+                            p.records[(size_t)n_tile * p.M + mbase + e] = make_float4(a1, __int_as_float(ai), a2, 0.0f);
+                        }
+                        named_bar_sync(1, 128);
+                        break;
+                    }
+                    default:
+                        break;
+                    }
+                }
+                if (!whole && e == 0) p.counters[t] = 0;
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[buf]);
+            ++seg;
+            u += kb1 - kb0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int NT>
+static int launch_nt(GemmParams& p, cudaStream_t stream) {
+    using C = GemmCfg<NT>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return (int)e;
+        attr_done = true;
+    }
+    k_gemm_tc<NT><<<p.ctas, 192, C::SMEM, stream>>>(p);
+    return (int)cudaGetLastError();
+}
+
+int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
+    p.KB = (p.K + 63) / 64;
+    p.m_tiles = (p.M + nt - 1) / nt;
+    if (p.swiglu) {
+        // n_tiles set by the caller (I / 64)
+    } else {
+        int nt_total = 0;
+        for (int i = 0; i < p.n_amat; ++i) {
+            p.amat[i].tile0 = nt_total;
+            p.amat[i].ntiles = (p.amat[i].rows + 127) / 128;
+            nt_total += p.amat[i].ntiles;
+        }
+        p.n_tiles = nt_total;
+    }
+    p.units = (long long)p.n_tiles * p.m_tiles * p.KB;
+    if (p.ctas <= 0 || p.ctas > num_sms) p.ctas = num_sms;
+    if ((long long)p.ctas > p.units) p.ctas = (int)p.units;
+    if (p.units == 0) return 0;
+    switch (nt) {
+    case 16: return launch_nt<16>(p, stream);
+    case 32: return launch_nt<32>(p, stream);
+    case 64: return launch_nt<64>(p, stream);
+    case 128: return launch_nt<128>(p, stream);
+    case 256: return launch_nt<256>(p, stream);
+    default: return (int)cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace df

@@ -1,0 +1,64 @@
+/*
+ * dflash_diag.h — diagnostic entry points of libdflash.
+ *
+ * These are not part of the DFlash draft step.  They expose single kernels of
+ * the library (for kernel-level tests), the host-side work partition of the
+ * tensor-core GEMM (for CPU tests), and a stand-in for the target model's
+ * verification pass that benchmarks and chained tests use to drive the
+ * draft/accept cycle with planned acceptance lengths.
+ */
+#ifndef DFLASH_DIAG_H_
+#define DFLASH_DIAG_H_
+
+#include "dflash.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Scratch bytes (device) that dflash_diag_gemm_bf16 needs for these sizes. */
+int dflash_diag_gemm_scratch_bytes(int M, int N, int K, size_t* bytes);
+
+/* Y[m, n] = sum_k X[m, k] * W[n, k] with the sm_100a tcgen05 GEMM (fp32
+ * accumulation, fp32 output).  X: device bf16 [M, K], W: device bf16 [N, K],
+ * Y: device fp32 [M, N]; K % 8 == 0, 1 <= M <= 4096.  scratch: device memory of
+ * dflash_diag_gemm_scratch_bytes, 256-byte aligned; it must be zero on the first
+ * call (the kernel leaves it zeroed again).  grid: persistent CTAs to use (0 = one
+ * per SM); a small grid forces the split-K fix-up path. */
+int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, int K,
+                          void* scratch, size_t scratch_bytes, int grid, dflash_stream stream);
+
+/* Work partition of the persistent split-K GEMM (host only, no CUDA call).
+ * `units` k-blocks in total, `kb` k-blocks per output tile, `ctas` CTAs.  For
+ * output tile `tile`: first_cta = first CTA contributing to it, n_contrib = the
+ * number of CTAs contributing.  Returns DFLASH_INVALID_ARG on bad sizes. */
+int dflash_diag_partition(int64_t units, int kb, int ctas, int64_t tile, int* first_cta, int* n_contrib);
+
+/* Stand-in for the target's greedy verification of one block per request:
+ * target[b, i] = drafts[b, i] for i < a_plan[b]; target[b, a_plan[b]] differs from
+ * drafts[b, a_plan[b]] when a_plan[b] < gamma-1; other entries are rand_tokens[b, i].
+ * All pointers are device int32: drafts [batch, gamma-1], a_plan [batch] (values
+ * in [0, gamma-1]), rand_tokens and target [batch, gamma].  A draft of -1 (skipped
+ * request) is treated like any other token. */
+int dflash_diag_synth_target(const int32_t* drafts, const int32_t* a_plan, const int32_t* rand_tokens,
+                             int batch, int gamma, int vocab, int32_t* target, dflash_stream stream);
+
+/* Diagnostic timer.  While enabled, the handle brackets each launch group of
+ * the four calls (a GEMM, an attention split + combine pair, a norm, ...) with
+ * two CUDA events recorded on the launch stream, up to max_launches groups.
+ * Not for use under CUDA-graph capture.  dflash_diag_timing_read synchronises
+ * `stream`, writes up to max_entries (kind, milliseconds) pairs in launch order,
+ * and restarts the log.  dflash_diag_timed_name names a kind. */
+int dflash_diag_timing_enable(dflash_handle* h, int max_launches);
+int dflash_diag_timing_read(dflash_handle* h, dflash_stream stream, int* kinds, float* ms, int max_entries,
+                            int* n_entries);
+int dflash_diag_timing_disable(dflash_handle* h);
+const char* dflash_diag_timed_name(int kind);
+
+/* "sm_100a" for this build. */
+const char* dflash_diag_arch(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFLASH_DIAG_H_ */

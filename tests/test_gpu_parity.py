@@ -1,0 +1,95 @@
+"""GPU path vs the CPU oracle, element by element, on reduced shapes that span
+several GEMM tiles and ragged tails: prefill (fuse + inject), then chained
+draft -> verify -> accept cycles with planned acceptance lengths.  The accept
+step consumes the oracle's drafts (teacher forcing) so both sides follow the
+same length trajectory; the GPU's own drafts are compared every cycle."""
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_speculative_03_b200 import inputs as I
+from tests.parity import Pair
+
+pytestmark = pytest.mark.gpu
+
+
+def _chain(name, cycles=None, order="speculative", gamma=None):
+    w = I.preset(name)
+    if cycles is not None:
+        w.cycles = cycles
+    g = gamma or w.gamma
+    pr = Pair(w)
+    pr.prefill()
+    anchors = I.make_anchors(w).numpy()
+    plan = I.plan_accept(w, w.cycles, gamma=g).numpy()
+    compared = 0
+    for cyc in range(w.cycles):
+        o_dr, g_dr, n = pr.draft(anchors, g)
+        compared += n
+        anchors = pr.verify_and_accept(o_dr, g, plan[cyc], cyc, order=order)
+        pr.check_cache()
+    return compared
+
+
+def test_tiny_fp32_chain():
+    # hidden 256, 2 layers, 4/2 heads, d 64, vocab 1024, 64 context rows, gamma 4
+    n = _chain("tiny", cycles=6)
+    assert n > 0
+
+
+def test_small_bf16_chain_speculative_order():
+    n = _chain("small_bf16")
+    assert n > 0
+
+
+def test_small_bf16_chain_commit_order():
+    _chain("small_bf16", cycles=2, order="commit")
+
+
+def test_small_bf16_untied_ragged_heads_and_empty_context():
+    # d 64, 3 kv heads (K/V sections not multiples of 128), vocab 2500, one
+    # request with an empty context, separate LM head
+    n = _chain("small_bf16_untied")
+    assert n > 0
+
+
+@pytest.mark.parametrize("gamma", [1, 2, 5, 8])
+def test_small_bf16_other_block_sizes(gamma):
+    w = I.preset("small_bf16")
+    pr = Pair(w)
+    pr.prefill(check=False)
+    anchors = I.make_anchors(w).numpy()
+    if gamma == 1:
+        drafts = torch.empty(w.batch, 1, dtype=torch.int32, device="cuda")
+        pr.gpu.draft_block(pr.cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"), 1, drafts=drafts)
+        torch.cuda.synchronize()
+        assert pr.cache.status() == 0
+        return
+    pr.draft(anchors, gamma)
+
+
+def test_inject_in_chunks_equals_all_at_once_on_gpu():
+    w = I.preset("small_bf16")
+    a = Pair(w)
+    a.prefill(check=False)
+    b = Pair(w, weights=a.W)
+    total = sum(w.context)
+    hid = I.make_hiddens(w, total)
+    ctx = b.gpu.fuse_context([h.cuda() for h in hid])
+    starts = np.cumsum([0] + w.context[:-1])
+    # inject each request's rows in two pieces of different sizes
+    for piece in range(2):
+        rs, rc = [], []
+        for r in range(w.batch):
+            T = w.context[r]
+            cut = T // 3
+            rs.append(int(starts[r]) + (0 if piece == 0 else cut))
+            rc.append(cut if piece == 0 else T - cut)
+        b.gpu.inject_kv(b.cache, ctx, torch.tensor(rs, dtype=torch.int32, device="cuda"),
+                        torch.tensor(rc, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(a.cache.len.cpu(), b.cache.len.cpu())
+    sa, sb = a.cache.slab(), b.cache.slab()
+    for r in range(w.batch):
+        T = w.context[r]
+        assert torch.equal(sa[r, :, :, :, :T], sb[r, :, :, :, :T])
