@@ -15,6 +15,19 @@
 
 using namespace df;
 
+namespace df {
+static bool g_pdl = true;
+void set_pdl(bool on) { g_pdl = on; }
+bool pdl_enabled() { return g_pdl; }
+void ensure_carveout(const void* fn) {
+    static std::vector<const void*> done;
+    for (const void* f : done)
+        if (f == fn) return;
+    cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    done.push_back(fn);
+}
+}  // namespace df
+
 namespace {
 
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -56,7 +69,7 @@ inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 constexpr int kMaxCtas = 160;   // >= SMs of any B200 part
 
 struct WsLayout {
-    size_t status, rope, x, h, q, o, act, hf, y, y32, lgs, part_o, part_ml, req_ok, gpart, gcnt, rec, total;
+    size_t status, rope, x, h, q, o, act, hf, y, y32, lgs, req_ok, gpart, gcnt, rec, total;
     int nt_max;
     long long n_counters;
 };
@@ -82,7 +95,7 @@ void make_layout(const dflash_config& c, WsLayout& L) {
     L.hf = off; off = al(off + Mlm * H * es);
     L.y = off; off = al(off + R * H * es);
     L.req_ok = off; off = al(off + (size_t)c.max_batch * 4);
-    L.y32 = L.lgs = L.part_o = L.part_ml = L.gpart = L.gcnt = L.rec = off;
+    L.y32 = L.lgs = L.gpart = L.gcnt = L.rec = off;
     L.nt_max = 0;
     L.n_counters = 0;
     if (!bf) {
@@ -90,9 +103,6 @@ void make_layout(const dflash_config& c, WsLayout& L) {
         L.y32 = off; off = al(off + (size_t)y32 * 4);
         L.lgs = off; off = al(off + (size_t)Mlm * V * 4);
     } else {
-        const long long parts = kAttnTargetCtas + (long long)c.max_batch * c.n_kv_heads;
-        L.part_o = off; off = al(off + (size_t)parts * 64 * d * 4);
-        L.part_ml = off; off = al(off + (size_t)parts * 64 * sizeof(float2));
         L.nt_max = pick_nt((int)std::max(std::max(Mmax, Mlm), R));
         L.gpart = off; off = al(off + gemm_partial_bytes(kMaxCtas, L.nt_max));
         const long long t_layer = std::max(std::max((long long)cdiv(Nq, 128) + 2 * cdiv(Nkv, 128), (long long)cdiv(H, 128)),
@@ -140,8 +150,7 @@ struct dflash_handle {
     int* status;
     float2* rope;
     void *x, *h, *q, *o, *act, *hf, *y;
-    float *y32, *lgs, *part_o, *gpart;
-    float2* part_ml;
+    float *y32, *lgs, *gpart;
     int *req_ok, *gcnt;
     float4* rec;
     CUtensorMap tm_wfc, tm_lm;
@@ -236,12 +245,6 @@ bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride
     return encode_bf16_2d(m, base, (uint64_t)K, (uint64_t)rows, (uint64_t)stride, (uint32_t)nt);
 }
 
-void attn_plan(int B, int nkv, int cap, int& splits, int& chunk) {
-    int s = cdiv(kAttnTargetCtas, (long long)B * nkv);
-    s = std::max(1, std::min(s, cdiv(cap, 64)));
-    chunk = cdiv(cdiv(cap, s), 64) * 64;
-    splits = cdiv(cap, chunk);
-}
 
 }  // namespace
 
@@ -314,8 +317,6 @@ int dflash_create(const dflash_config* cfg, const dflash_weights* w, void* works
     h->y = b + L.y;
     h->y32 = (float*)(b + L.y32);
     h->lgs = (float*)(b + L.lgs);
-    h->part_o = (float*)(b + L.part_o);
-    h->part_ml = (float2*)(b + L.part_ml);
     h->req_ok = (int*)(b + L.req_ok);
     h->gpart = (float*)(b + L.gpart);
     h->gcnt = (int*)(b + L.gcnt);
@@ -598,15 +599,14 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
         !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)))
         return DFLASH_CUDA;
     int splits, chunk;
-    attn_plan(B, c.n_kv_heads, cc->capacity, splits, chunk);
+    attn_plan(B, c.n_kv_heads, cc->capacity, h->num_sms, splits, chunk);
     AttnParams ap;
     std::memset(&ap, 0, sizeof(ap));
     ap.tmap = cc->tm_slab;
     ap.q = (const bf*)h->q;
+    ap.out = (bf*)h->o;
     ap.len = cc->len;
     ap.req_ok = h->req_ok;
-    ap.part_o = h->part_o;
-    ap.part_ml = h->part_ml;
     ap.gamma = gamma;
     ap.G = c.n_q_heads / c.n_kv_heads;
     ap.nq = c.n_q_heads;
@@ -663,7 +663,7 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
         ap.layer = l;
         {
             Timed t(h, TK_ATTENTION, st);
-            int e = launch_attention(ap, d, B, st, (bf*)h->o, &h->launches);
+            int e = launch_attention(ap, d, B, st, &h->launches);
             if (e) return DFLASH_CUDA;
         }
         {   // O-proj + residual
@@ -934,6 +934,57 @@ int dflash_diag_timing_disable(dflash_handle* h) {
     h->ev.clear();
     h->ev_kind.clear();
     h->ev_used = 0;
+    return DFLASH_OK;
+}
+
+int dflash_diag_attention(dflash_handle* h, dflash_cache* cc, const void* q, void* out, int layer, int gamma,
+                          dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || gamma < 1 ||
+        gamma > h->cfg.max_gamma || h->cfg.dtype != DFLASH_BF16)
+        return DFLASH_INVALID_ARG;
+    const dflash_config& c = h->cfg;
+    const int d = c.head_dim;
+    // all requests are attended (req_ok = 1): the caller keeps len + gamma <= capacity
+    std::vector<int> ones(cc->batch, 1);
+    if (cudaMemcpyAsync(h->req_ok, ones.data(), cc->batch * sizeof(int), cudaMemcpyHostToDevice, S(stream)) !=
+        cudaSuccess)
+        return DFLASH_CUDA;
+    AttnParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    int splits, chunk;
+    attn_plan(cc->batch, c.n_kv_heads, cc->capacity, h->num_sms, splits, chunk);
+    ap.tmap = cc->tm_slab;
+    ap.q = (const __nv_bfloat16*)q;
+    ap.out = (__nv_bfloat16*)out;
+    ap.len = cc->len;
+    ap.req_ok = h->req_ok;
+    ap.gamma = gamma;
+    ap.G = c.n_q_heads / c.n_kv_heads;
+    ap.nq = c.n_q_heads;
+    ap.nkv = c.n_kv_heads;
+    ap.layer = layer;
+    ap.splits = splits;
+    ap.chunk = chunk;
+    ap.rows_kv = cc->s_kv / d;
+    ap.rows_kind = cc->s_kind / d;
+    ap.rows_layer = cc->s_layer / d;
+    ap.rows_req = cc->s_req / d;
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    ap.status = h->status;
+    const int e = launch_attention(ap, d, cc->batch, S(stream), &h->launches);
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DFLASH_CUDA;
+    return e == 0 ? DFLASH_OK : DFLASH_CUDA;
+}
+
+int dflash_diag_wait_selftest(dflash_handle* h, int32_t* out, dflash_stream stream) {
+    if (!h || !out) return DFLASH_INVALID_ARG;
+    const int e = launch_wait_selftest(h->status, out, S(stream));
+    h->launches += 1;
+    return e == 0 ? DFLASH_OK : DFLASH_CUDA;
+}
+
+int dflash_diag_set_launch_mode(int programmatic) {
+    set_pdl(programmatic != 0);
     return DFLASH_OK;
 }
 

@@ -1,20 +1,25 @@
-// Block attention of the draft step (bf16 storage), split over the key axis.
+// Block attention of the draft step (bf16 storage), split over the key axis
+// across the CTAs of one thread-block cluster.
 //
 // For request b and kv head g, the G*gamma query rows (G = query heads per kv
 // head) attend to every cached row [0, len) plus the gamma block rows that the
-// QKV epilogue wrote at [len, len+gamma): no mask.  CTA (split s, g, b) takes
-// key rows [s*chunk, (s+1)*chunk): K/V tiles of 64 rows x d arrive by TMA
-// (128-byte swizzle, no multicast) into a 2-stage ring; each warp owns 16
-// query rows (and a share of each tile's keys when there are fewer than 64
+// QKV epilogue wrote at [len, len+gamma): no mask.  The `splits` CTAs of a
+// cluster (b, g) each take one key range: K/V tiles of 64 rows x d arrive by
+// TMA (128-byte swizzle, no multicast) into a 3-stage ring; each warp owns 16
+// query rows (and a share of every tile's keys when there are fewer than 64
 // rows), computes S = Q K^T and O += P V with mma.sync m16n8k16 (bf16 in, fp32
 // accumulate), and keeps the online-softmax row max / sum with quad shuffles.
-// Partials (m, l, O) per split are merged by k_attn_combine.
+// Each CTA leaves its partial (m, l, O) in its own shared memory; after a
+// cluster barrier every CTA merges a slice of the rows by reading all partials
+// through distributed shared memory, and writes the bf16 output.  No partial
+// goes through global memory and no second kernel is needed.
+#include <cooperative_groups.h>
+
 #include "attn.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace df {
-
-
-
 
 // Byte offset of element (r, c) in a [64 rows][D] bf16 tile stored as D/64
 // column blocks of [64 rows][128 B] with the 128-byte swizzle (16-byte chunk
@@ -24,7 +29,7 @@ DF_DEV uint32_t sw_off(int r, int c) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ AttnParams p) {
     constexpr int TILE_BYTES = 64 * D * 2;
     constexpr int NDT = D / 8;     // n-tiles of the output
     extern __shared__ uint8_t smem_raw[];
@@ -33,16 +38,41 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
     uint8_t* sK = sQ + TILE_BYTES;                   // [stages]
     uint8_t* sV = sK + kAttnStages * TILE_BYTES;     // [stages]
     uint64_t* bars = (uint64_t*)(sV + kAttnStages * TILE_BYTES);
+    // After the key loop the ring is reused: per-warp results, then the CTA's partial.
+    float* mo = (float*)(smem + TILE_BYTES);         // [4 warps][16][D]
+    float2* mml = (float2*)(mo + 4 * 16 * D);        // [4 warps][16] (m, l)
+    float* po = (float*)(mml + 4 * 16);              // [64][D]  partial O of this CTA
+    float2* pml = (float2*)(po + 64 * D);            // [64]     (m, l) of this CTA
+    float* wts = (float*)(pml + 64);                 // [64][4]  in-CTA merge weights
+    float* cm = wts + 64 * 4;                        // [64][splits] peers' row max
+    float* cl = cm + 64 * kAttnMaxSplits;            // [64][splits] peers' row sum
+    float* cw = cl + 64 * kAttnMaxSplits;            // [64][splits] normalised merge weights
     __shared__ int s_abort;
 
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int nsplit = p.splits;
+    const int g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (!p.req_ok[b]) return;
+    if (tid == 0) tma_prefetch_desc(&p.tmap);
+    griddep_wait();
+    griddep_launch();
+
+    const int R = p.G * p.gamma;
+    const int rows_per = (R + nsplit - 1) / nsplit;
+    const int r_lo = rank * rows_per, r_hi = min(R, r_lo + rows_per);
+    if (!p.req_ok[b]) {   // skipped request: zero output rows, no cluster traffic
+        for (int r = r_lo; r < r_hi; ++r) {
+            const int j = r / p.G, hh = r % p.G;
+            __nv_bfloat16* dst = p.out + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D;
+            for (int c = tid; c < D; c += 128) dst[c] = f2bf(0.f);
+        }
+        return;
+    }
     const int n = p.len[b] + p.gamma;
-    const int kv0 = s * p.chunk;
+    const int kv0 = rank * p.chunk;
     const int kv1 = min(n, kv0 + p.chunk);
     const int ntiles = kv1 > kv0 ? (kv1 - kv0 + 63) / 64 : 0;
-    const int R = p.G * p.gamma;
     int RT = (R + 15) / 16;
     if (RT == 3) RT = 4;
     const int NKS = 4 / RT;
@@ -58,7 +88,6 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
     }
     __syncthreads();
     if (tid == 0) {
-        tma_prefetch_desc(&p.tmap);
         for (int it = 0; it < min(ntiles, kAttnStages); ++it) {
             mbar_arrive_expect_tx(&bars[it], 2 * TILE_BYTES);
             for (int h = 0; h < D / 64; ++h) {
@@ -91,7 +120,10 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
         }
     }
 
-    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+    // Base-2 online softmax with an integer base: m_t = running max of the
+    // log2-scaled scores, m_r = floor(m_t).  Every rescale is 2^(integer), so
+    // bf16(2^(t - m_r)) rescaled later equals bf16(2^(t - final base)) exactly.
+    float m_t[2] = {-INFINITY, -INFINITY}, m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
     float o[NDT][4];
 #pragma unroll
     for (int i = 0; i < NDT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
@@ -138,8 +170,8 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
                 const int kv = kvbase + nt * 8 + 2 * (lane & 3);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const bool valid = (kv + (c & 1)) < kv1;
-                    sc[nt][c] = valid ? sc[nt][c] * p.scale_log2 : -INFINITY;
+                    const bool valid_k = (kv + (c & 1)) < kv1;
+                    sc[nt][c] = valid_k ? sc[nt][c] * p.scale_log2 : -INFINITY;
                 }
                 mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
                 mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
@@ -149,12 +181,14 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m_r[0], mx0), mn1 = fmaxf(m_r[1], mx1);
-        const float base0 = (mn0 == -INFINITY) ? 0.f : mn0;
-        const float base1 = (mn1 == -INFINITY) ? 0.f : mn1;
-        const float corr0 = exp2f(m_r[0] - base0), corr1 = exp2f(m_r[1] - base1);
-        m_r[0] = mn0;
-        m_r[1] = mn1;
+        m_t[0] = fmaxf(m_t[0], mx0);
+        m_t[1] = fmaxf(m_t[1], mx1);
+        const float nb0 = floorf(m_t[0]), nb1 = floorf(m_t[1]);      // -inf stays -inf
+        const float base0 = (nb0 == -INFINITY) ? 0.f : nb0;
+        const float base1 = (nb1 == -INFINITY) ? 0.f : nb1;
+        const float corr0 = exp2f(m_r[0] - base0), corr1 = exp2f(m_r[1] - base1);   // 0 while m_r is -inf
+        m_r[0] = nb0;
+        m_r[1] = nb1;
         float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
@@ -206,148 +240,137 @@ __global__ void __launch_bounds__(128) k_attn_split(const __grid_constant__ Attn
             }
         }
     }
-    // Quad-reduce the row sums.
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 1);
         l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 2);
     }
-    __syncthreads();
-    // Merge the key shares of warps that hold the same query rows.
-    float* mo = (float*)(smem + TILE_BYTES);          // reuse the K/V ring: [4 warps][16][D]
-    float* mml = mo + 4 * 16 * D;                     // [4 warps][16][2]
-    if (NKS > 1) {
+    __syncthreads();   // the ring is free from here on
+
+    // ---- this CTA's partial: merge the key shares of the warps of each row tile
+    {
         const int r0 = lane >> 2, c0 = 2 * (lane & 3);
 #pragma unroll
         for (int nd = 0; nd < NDT; ++nd) {
-            mo[(warp * 16 + r0) * D + nd * 8 + c0] = o[nd][0];
-            mo[(warp * 16 + r0) * D + nd * 8 + c0 + 1] = o[nd][1];
-            mo[(warp * 16 + r0 + 8) * D + nd * 8 + c0] = o[nd][2];
-            mo[(warp * 16 + r0 + 8) * D + nd * 8 + c0 + 1] = o[nd][3];
+            *reinterpret_cast<float2*>(&mo[(warp * 16 + r0) * D + nd * 8 + c0]) = make_float2(o[nd][0], o[nd][1]);
+            *reinterpret_cast<float2*>(&mo[(warp * 16 + r0 + 8) * D + nd * 8 + c0]) = make_float2(o[nd][2], o[nd][3]);
         }
         if ((lane & 3) == 0) {
-            mml[(warp * 16 + r0) * 2] = m_r[0];
-            mml[(warp * 16 + r0) * 2 + 1] = l_r[0];
-            mml[(warp * 16 + r0 + 8) * 2] = m_r[1];
-            mml[(warp * 16 + r0 + 8) * 2 + 1] = l_r[1];
-        }
-        __syncthreads();
-        if (ks == 0) {
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int r = (lane >> 2) + hr * 8;
-                float M = -INFINITY;
-                for (int k2 = 0; k2 < NKS; ++k2) M = fmaxf(M, mml[((rt + k2 * RT) * 16 + r) * 2]);
-                const float base = (M == -INFINITY) ? 0.f : M;
-                float L = 0.f;
-                float sc2[4];
-                for (int k2 = 0; k2 < NKS; ++k2) {
-                    sc2[k2] = exp2f(mml[((rt + k2 * RT) * 16 + r) * 2] - base);
-                    L += sc2[k2] * mml[((rt + k2 * RT) * 16 + r) * 2 + 1];
-                }
-#pragma unroll
-                for (int nd = 0; nd < NDT; ++nd) {
-                    for (int cc = 0; cc < 2; ++cc) {
-                        float acc = 0.f;
-                        for (int k2 = 0; k2 < NKS; ++k2)
-                            acc += sc2[k2] * mo[((rt + k2 * RT) * 16 + r) * D + nd * 8 + 2 * (lane & 3) + cc];
-                        o[nd][hr * 2 + cc] = acc;
-                    }
-                }
-                m_r[hr] = M;
-                l_r[hr] = L;
-            }
+            mml[warp * 16 + r0] = make_float2(m_r[0], l_r[0]);
+            mml[warp * 16 + r0 + 8] = make_float2(m_r[1], l_r[1]);
         }
     }
-    if (ks == 0) {
-        const size_t base = ((size_t)(b * p.nkv + g) * p.splits + s) * 64;
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int r = rt * 16 + (lane >> 2) + hr * 8;
-            if (r < R) {
-                float* dst = p.part_o + (base + r) * D;
-#pragma unroll
-                for (int nd = 0; nd < NDT; ++nd)
-                    *reinterpret_cast<float2*>(dst + nd * 8 + 2 * (lane & 3)) = make_float2(o[nd][hr * 2], o[nd][hr * 2 + 1]);
-                if ((lane & 3) == 0) p.part_ml[base + r] = make_float2(m_r[hr], l_r[hr]);
-            }
+    __syncthreads();
+    for (int r = tid; r < R; r += 128) {
+        const int t = r >> 4, rr = r & 15;
+        float M = -INFINITY;
+        for (int k2 = 0; k2 < NKS; ++k2) M = fmaxf(M, mml[(t + k2 * RT) * 16 + rr].x);
+        const float base = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f;
+        for (int k2 = 0; k2 < NKS; ++k2) {
+            const float2 ml = mml[(t + k2 * RT) * 16 + rr];
+            const float wk = exp2f(ml.x - base);
+            wts[r * 4 + k2] = wk;
+            L += wk * ml.y;
         }
+        pml[r] = make_float2(M, L);
     }
+    __syncthreads();
+    for (int idx = tid; idx < R * D; idx += 128) {
+        const int r = idx / D, c = idx % D, t = r >> 4, rr = r & 15;
+        float acc = 0.f;
+        for (int k2 = 0; k2 < NKS; ++k2) acc += wts[r * 4 + k2] * mo[((t + k2 * RT) * 16 + rr) * D + c];
+        po[r * D + c] = acc;
+    }
+
+    // ---- merge the cluster's partials through distributed shared memory
+    cluster.sync();
+    const float* rpo[kAttnMaxSplits];
+    const float2* rpml[kAttnMaxSplits];
+#pragma unroll
+    for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+        rpo[s2] = s2 < nsplit ? cluster.map_shared_rank(po, s2) : po;
+        rpml[s2] = s2 < nsplit ? cluster.map_shared_rank(pml, s2) : pml;
+    }
+    const int nr = r_hi - r_lo;
+    for (int idx = tid; idx < nr * nsplit; idx += 128) {
+        const int r = r_lo + idx / nsplit, s2 = idx % nsplit;
+        const float2 ml = rpml[s2][r];
+        cm[idx] = ml.x;
+        cl[idx] = ml.y;
+    }
+    __syncthreads();
+    for (int rr = tid; rr < nr; rr += 128) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, cm[rr * nsplit + s2]);
+        const float base = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f;
+        for (int s2 = 0; s2 < nsplit; ++s2) {
+            const float l = cl[rr * nsplit + s2];
+            const float wv = l > 0.f ? exp2f(cm[rr * nsplit + s2] - base) : 0.f;
+            cw[rr * nsplit + s2] = wv;
+            L += wv * l;
+        }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        for (int s2 = 0; s2 < nsplit; ++s2) cw[rr * nsplit + s2] *= inv;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < nr * D; idx += 128) {
+        const int rr = idx / D, c = idx % D, r = r_lo + rr;
+        float v[kAttnMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) v[s2] = s2 < nsplit ? rpo[s2][r * D + c] : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
+            if (s2 < nsplit) acc += cw[rr * nsplit + s2] * v[s2];
+        const int j = r / p.G, hh = r % p.G;
+        p.out[((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c] = f2bf(acc);
+    }
+    cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
 }
 
-// Merge the split partials: one warp per (request, block position, query head).
-template <int D>
-__global__ void k_attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
-                               __nv_bfloat16* __restrict__ out, const int* __restrict__ req_ok, int B, int gamma,
-                               int G, int nq, int nkv, int splits) {
-    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (wid >= B * gamma * nq) return;
-    const int hq = wid % nq, j = (wid / nq) % gamma, b = wid / (nq * gamma);
-    const int g = hq / G, r = j * G + (hq % G);
-    constexpr int PER = D / 32;
-    float acc[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    __nv_bfloat16* dst = out + ((size_t)(b * gamma + j) * nq + hq) * D;
-    if (!req_ok[b]) {
-        for (int i = 0; i < PER; ++i) dst[lane + 32 * i] = f2bf(0.f);
-        return;
-    }
-    const size_t base = (size_t)(b * nkv + g) * splits * 64 + r;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[base + (size_t)s * 64].x);
-    const float mb = (M == -INFINITY) ? 0.f : M;
-    float L = 0.f;
-    for (int s = 0; s < splits; ++s) {
-        const float2 ml = part_ml[base + (size_t)s * 64];
-        if (ml.y == 0.f) continue;
-        const float w = exp2f(ml.x - mb);
-        L += w * ml.y;
-        const float* po = part_o + (base + (size_t)s * 64) * D;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) acc[i] += w * po[lane + 32 * i];
-    }
-    const float inv = L > 0.f ? 1.0f / L : 0.f;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) dst[lane + 32 * i] = f2bf(acc[i] * inv);
+int attn_smem_bytes(int d) {
+    return 1024 + (1 + 2 * kAttnStages) * 64 * d * 2 + 64;
 }
 
-int attn_smem_bytes(int d) { return 1024 + (1 + 2 * kAttnStages) * 64 * d * 2 + 64; }
+void attn_plan(int B, int nkv, int cap, int num_sms, int& splits, int& chunk) {
+    const int tiles = (cap + 63) / 64;
+    int s = (num_sms + B * nkv - 1) / (B * nkv);
+    s = s < 1 ? 1 : (s > kAttnMaxSplits ? kAttnMaxSplits : s);
+    if (s > tiles) s = tiles;
+    chunk = ((tiles + s - 1) / s) * 64;
+    splits = (cap + chunk - 1) / chunk;
+}
 
-int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, __nv_bfloat16* out,
-                     long long* launches) {
-    dim3 grid(p.splits, p.nkv, B);
+int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, long long* launches) {
     const int smem = attn_smem_bytes(d);
-    cudaError_t e;
-    if (d == 128) {
-        static bool done = false;
-        if (!done) {
-            e = cudaFuncSetAttribute(k_attn_split<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return (int)e;
-            done = true;
-        }
-        k_attn_split<128><<<grid, 128, smem, stream>>>(p);
-    } else {
-        static bool done = false;
-        if (!done) {
-            e = cudaFuncSetAttribute(k_attn_split<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return (int)e;
-            done = true;
-        }
-        k_attn_split<64><<<grid, 128, smem, stream>>>(p);
+    void (*kern)(AttnParams) = (d == 128) ? k_attn_cluster<128> : k_attn_cluster<64>;
+    static bool done128 = false, done64 = false;
+    bool& done = (d == 128) ? done128 : done64;
+    if (!done) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return (int)e;
+        ensure_carveout((const void*)kern);
+        done = true;
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return (int)e;
-    const int warps = B * p.gamma * p.nq;
-    const int blocks = (warps * 32 + 255) / 256;
-    if (d == 128)
-        k_attn_combine<128><<<blocks, 256, 0, stream>>>(p.part_o, p.part_ml, out, p.req_ok, B, p.gamma, p.G, p.nq,
-                                                        p.nkv, p.splits);
-    else
-        k_attn_combine<64><<<blocks, 256, 0, stream>>>(p.part_o, p.part_ml, out, p.req_ok, B, p.gamma, p.G, p.nq,
-                                                       p.nkv, p.splits);
-    *launches += 2;
-    return (int)cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.splits, p.nkv, B);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    *launches += 1;
+    return (int)e;
 }
 
 }  // namespace df

@@ -107,6 +107,38 @@ DF_DEV bool named_bar_or(int id, int nthreads, bool pred) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library calls
+// griddep_wait() before its first global-memory access that may depend on (or
+// race with) the previous kernel in the stream, and griddep_launch() early so
+// the next kernel can be scheduled while this one drains.
+// ---------------------------------------------------------------------------
+DF_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DF_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Host: launch with the programmatic-stream-serialization attribute when
+// enabled (set_pdl), else as a plain stream-ordered launch.
+void set_pdl(bool on);
+bool pdl_enabled();
+// Give every kernel the same (maximal) shared-memory carveout, once per
+// kernel, so consecutive kernels never make an SM re-partition L1 / shared.
+void ensure_carveout(const void* fn);
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    ensure_carveout((const void*)kern);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ((KArgs)args)...);
+}
+
+// ---------------------------------------------------------------------------
 // TMA (bulk tensor copies, no multicast)
 // ---------------------------------------------------------------------------
 DF_DEV void tma_prefetch_desc(const CUtensorMap* m) {

@@ -87,10 +87,36 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
     const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
     const long long u_begin = sk_begin(cta, U, P), u_end = sk_begin(cta + 1, U, P);
 
+    griddep_launch();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol_w = make_l2_policy_evict_first();
+            // Weights never depend on the previous kernel: start streaming the
+            // first S weight tiles before waiting for it to finish.
+            int pre = 0;
+            for (long long u = u_begin; u < u_end && pre < S;) {
+                const long long t = u / KB;
+                const int kb0 = (int)(u % KB);
+                const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+                const int n_tile = (int)(t / m_tiles);
+                int mi = 0;
+                if (!p.swiglu)
+                    while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
+                const int arow = p.swiglu ? n_tile * 64 : (n_tile - p.amat[mi].tile0) * 128;
+                for (int kb = kb0; kb < kb1 && pre < S; ++kb, ++pre) {
+                    mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+                    uint8_t* a = sA + pre * C::A_BYTES;
+                    if (p.swiglu) {
+                        tma_load_2d_hint(a, &p.ta[0], &full[pre], kb * 64, arow, pol_w);
+                        tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[pre], kb * 64, arow, pol_w);
+                    } else {
+                        tma_load_2d_hint(a, &p.ta[mi], &full[pre], kb * 64, arow, pol_w);
+                    }
+                }
+                u += kb1 - kb0;
+            }
+            griddep_wait();
             int stage = 0;
             uint32_t round = 0;
             long long issued = 0;
@@ -105,15 +131,17 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                     while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
                 const int arow = p.swiglu ? n_tile * 64 : (n_tile - p.amat[mi].tile0) * 128;
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(&empty[stage], (round & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
                     uint8_t* a = sA + stage * C::A_BYTES;
                     uint8_t* b = sB + stage * C::B_BYTES;
-                    if (p.swiglu) {
-                        tma_load_2d_hint(a, &p.ta[0], &full[stage], kb * 64, arow, pol_w);
-                        tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[stage], kb * 64, arow, pol_w);
-                    } else {
-                        tma_load_2d_hint(a, &p.ta[mi], &full[stage], kb * 64, arow, pol_w);
+                    if (issued >= pre) {
+                        if (!mbar_wait(&empty[stage], (round & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                        if (p.swiglu) {
+                            tma_load_2d_hint(a, &p.ta[0], &full[stage], kb * 64, arow, pol_w);
+                            tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[stage], kb * 64, arow, pol_w);
+                        } else {
+                            tma_load_2d_hint(a, &p.ta[mi], &full[stage], kb * 64, arow, pol_w);
+                        }
                     }
                     const int bm = kb / p.kb_per_b;
                     tma_load_2d(b, &p.tb[bm], &full[stage], (kb - bm * p.kb_per_b) * 64, m_tile * NT);
@@ -133,6 +161,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        griddep_wait();
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_bf16_f32(128, NT);
             int stage = 0, seg = 0;
@@ -171,6 +200,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        griddep_wait();
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const int row = q * 32 + lane;          // weight-tile row = TMEM lane
         const int e = threadIdx.x - 64;         // 0..127
@@ -218,29 +248,35 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                 const int lr = p.swiglu ? 0 : (n_tile - p.amat[mi].tile0) * 128 + row;
                 const bool row_ok = p.swiglu ? true : (lr < p.amat[mi].rows);
                 // Per-token request / position for the cache-writing epilogues.
-                if (p.epi == EPI_QKV || p.epi == EPI_INJECT) {
+                if (p.epi == EPI_QKV) {
                     named_bar_sync(1, 128);
                     for (int te = e; te < NT; te += 128) {   // NT may exceed the 128 epilogue threads
                         const int m = m_tile * NT + te;
                         int b = -1, pos = -1;
                         if (m < p.M) {
-                            if (p.epi == EPI_QKV) {
-                                const int bb = m / p.gamma;
-                                if (p.req_ok[bb]) { b = bb; pos = p.len[bb] + (m - bb * p.gamma); }
-                            } else {
-                                for (int bb = 0; bb < p.batch; ++bb) {
-                                    const int rs = p.row_start[bb], rc = p.row_count[bb];
-                                    if (m >= rs && m < rs + rc) {
-                                        const int L0 = p.len[bb];
-                                        if (L0 + rc <= p.cap) { b = bb; pos = L0 + (m - rs); }
-                                        break;
-                                    }
-                                }
-                            }
+                            const int bb = m / p.gamma;
+                            if (p.req_ok[bb]) { b = bb; pos = p.len[bb] + (m - bb * p.gamma); }
                         }
                         if (pos < 0 || pos >= p.cap) b = -1;   // never write outside the request's slab
                         tok_b[te] = b;
                         tok_pos[te] = pos;
+                    }
+                    named_bar_sync(1, 128);
+                } else if (p.epi == EPI_INJECT) {
+                    // One thread per request marks the rows it owns in this m-tile
+                    // (independent loads; no per-token search over the batch).
+                    named_bar_sync(1, 128);
+                    for (int te = e; te < NT; te += 128) tok_b[te] = -1;
+                    named_bar_sync(1, 128);
+                    const int m0 = m_tile * NT;
+                    for (int bb = e; bb < p.batch; bb += 128) {
+                        const int rs = p.row_start[bb], rc = p.row_count[bb], L0 = p.len[bb];
+                        if (rc <= 0 || L0 < 0 || L0 + rc > p.cap) continue;
+                        const int lo = max(rs, m0), hi = min(min(rs + rc, m0 + NT), p.M);
+                        for (int m = lo; m < hi; ++m) {
+                            tok_b[m - m0] = bb;
+                            tok_pos[m - m0] = L0 + (m - rs);
+                        }
                     }
                     named_bar_sync(1, 128);
                 }
@@ -273,6 +309,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                     case EPI_F32: {
                         float* o = (float*)p.out;
                         if (row_ok)
+#pragma unroll
                             for (int i = 0; i < CH; ++i)
                                 if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = v[i];
                         break;
@@ -280,18 +317,22 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                     case EPI_BF16: {
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
                         if (row_ok)
+#pragma unroll
                             for (int i = 0; i < CH; ++i)
                                 if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = f2bf(v[i]);
                         break;
                     }
                     case EPI_RESID: {
+                        // All residual loads of the chunk first, then the stores,
+                        // so the loads are not serialised behind the stores.
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
-                        if (row_ok)
-                            for (int i = 0; i < CH; ++i)
-                                if (mbase + i < p.M) {
-                                    __nv_bfloat16* po = o + (size_t)(mbase + i) * p.ldo + lr;
-                                    *po = f2bf(bf2f(*po) + v[i]);
-                                }
+                        float rv[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i)
+                            rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+#pragma unroll
+                        for (int i = 0; i < CH; ++i)
+                            if (row_ok && mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = f2bf(rv[i] + v[i]);
                         break;
                     }
                     case EPI_SWIGLU: {
@@ -301,6 +342,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                         if (row < 64) {
                             __nv_bfloat16* o = (__nv_bfloat16*)p.out;
                             const int f = n_tile * 64 + row;
+#pragma unroll
                             for (int i = 0; i < CH; ++i)
                                 if (mbase + i < p.M) {
                                     const float up = xch[(row + 64) * 33 + i];
@@ -325,6 +367,15 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                         named_bar_sync(1, 128);
                         const int prow = (i_in < half) ? row + half : row - half;
                         if (row_ok) {
+                            // cos/sin of every column first (independent loads), then the stores
+                            float2 cs[CH];
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) {
+                                const int b = tok_b[c0 + i];
+                                cs[i] = (rotate && b >= 0) ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
+                                                           : make_float2(1.f, 0.f);
+                            }
+#pragma unroll
                             for (int i = 0; i < CH; ++i) {
                                 const int b = tok_b[c0 + i];
                                 if (b < 0) continue;
@@ -332,8 +383,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                                 float x = v[i];
                                 if (rotate) {
                                     const float pr = xch[prow * 33 + i];
-                                    const float2 cs = p.rope[(size_t)pos * half + (i_in % half)];
-                                    x = (i_in < half) ? (x * cs.x - pr * cs.y) : (x * cs.x + pr * cs.y);
+                                    x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
                                 }
                                 if (is_q) {
                                     ((__nv_bfloat16*)p.out)[(size_t)(mbase + i) * p.ldo + lr] = f2bf(x);
@@ -410,7 +460,8 @@ static int launch_nt(GemmParams& p, cudaStream_t stream) {
         if (e != cudaSuccess) return (int)e;
         attr_done = true;
     }
-    k_gemm_tc<NT><<<p.ctas, 192, C::SMEM, stream>>>(p);
+    cudaError_t e = launch_k(k_gemm_tc<NT>, dim3(p.ctas), dim3(192), (size_t)C::SMEM, stream, p);
+    if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
 }
 

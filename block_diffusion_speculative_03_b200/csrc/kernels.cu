@@ -14,6 +14,8 @@ template <typename T>
 __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anchor, int mask_id, int gamma, int H,
                         int V, const int* __restrict__ len, const int* __restrict__ committed, int cap,
                         T* __restrict__ x, int* __restrict__ req_ok, int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch();
     const int m = blockIdx.x, b = m / gamma, j = m % gamma;
     const int L0 = len[b], a = anchor[b];
     int err = 0;
@@ -45,14 +47,24 @@ __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anc
 template <typename T>
 __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* __restrict__ y, int H, float eps,
                           int grp, int gstride, int goff) {
+    griddep_wait();
+    griddep_launch();
+    constexpr int VEC = 16 / sizeof(T);          // elements per 16-byte access
     const int o = blockIdx.x;
     const int in = (o / grp) * gstride + goff + o % grp;
-    const T* xr = x + (size_t)in * H;
-    T* yr = y + (size_t)o * H;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)in * H);
+    const uint4* gr = reinterpret_cast<const uint4*>(g);
+    uint4* yr = reinterpret_cast<uint4*>(y + (size_t)o * H);
+    const int nv = H / VEC;
     float ss = 0.f;
-    for (int i = threadIdx.x; i < H; i += blockDim.x) {
-        const float v = ldf(xr + i);
-        ss += v * v;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+        const uint4 u = xr[i];
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+            const float v = ldf(e + k);
+            ss += v * v;
+        }
     }
     __shared__ float red[32];
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -65,7 +77,16 @@ __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* _
     }
     __syncthreads();
     const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-    for (int i = threadIdx.x; i < H; i += blockDim.x) stf(yr + i, ldf(xr + i) * inv * ldf(g + i));
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+        const uint4 u = xr[i], gu = gr[i];
+        const T* e = reinterpret_cast<const T*>(&u);
+        const T* ge = reinterpret_cast<const T*>(&gu);
+        uint4 out;
+        T* oe = reinterpret_cast<T*>(&out);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) stf(oe + k, ldf(e + k) * inv * ldf(ge + k));
+        yr[i] = out;
+    }
 }
 
 // Top-2 merge with ties of the top value to the lower id.
@@ -85,6 +106,8 @@ DF_DEV void top2m(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
 // ---------------------------------------------------------------------------
 __global__ void k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M, int gm1, const int* __restrict__ req_ok,
                             int* __restrict__ drafts, float* __restrict__ margin) {
+    griddep_wait();
+    griddep_launch();
     const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (m >= M) return;
     float a1 = -INFINITY, a2 = -INFINITY;
@@ -109,6 +132,8 @@ __global__ void k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M, int
 // fp32 path: top-2 over the fp32 logits of each row; one CTA per row.
 __global__ void k_top2_rows(const float* __restrict__ logits, int V, int gm1, const int* __restrict__ req_ok,
                             int* __restrict__ drafts, float* __restrict__ margin) {
+    griddep_wait();
+    griddep_launch();
     const int m = blockIdx.x;
     const float* row = logits + (size_t)m * V;
     float a1 = -INFINITY, a2 = -INFINITY;
@@ -140,6 +165,8 @@ __global__ void k_top2_rows(const float* __restrict__ logits, int V, int gm1, co
 __global__ void k_accept(const int* __restrict__ drafts, const int* __restrict__ target, int B, int gamma, int V,
                          int* __restrict__ len, int* __restrict__ committed, int* __restrict__ accept_len,
                          int* __restrict__ next_anchor, int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch();
     const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (b >= B) return;
     const int tg = lane < gamma ? target[(size_t)b * gamma + lane] : 0;
@@ -167,6 +194,8 @@ __global__ void k_accept(const int* __restrict__ drafts, const int* __restrict__
 // After an injection: len[b] += row_count[b] for every request that fitted.
 __global__ void k_inject_finalize(const int* __restrict__ row_count, int B, int cap, int* __restrict__ len,
                                   int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     const int rc = row_count[b];
@@ -177,6 +206,8 @@ __global__ void k_inject_finalize(const int* __restrict__ row_count, int B, int 
 
 __global__ void k_set_len(const int* __restrict__ lens, int B, int cap, int* __restrict__ len,
                           int* __restrict__ committed, int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     const int v = lens[b];
@@ -188,6 +219,8 @@ __global__ void k_set_len(const int* __restrict__ lens, int B, int cap, int* __r
 // Stand-in for the target's greedy verification (diagnostic).
 __global__ void k_synth_target(const int* __restrict__ drafts, const int* __restrict__ a_plan,
                                const int* __restrict__ rnd, int B, int gamma, int V, int* __restrict__ target) {
+    griddep_wait();
+    griddep_launch();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= B * gamma) return;
     const int b = idx / gamma, i = idx % gamma;
@@ -202,6 +235,23 @@ __global__ void k_synth_target(const int* __restrict__ drafts, const int* __rest
     target[idx] = t;
 }
 
+// Self-test of the bounded pipeline wait: one thread waits on an mbarrier that
+// nothing ever arrives at; the wait gives up after its limit, records
+// DFLASH_TIMEOUT in *status and the kernel returns normally.
+__global__ void k_wait_selftest(int* status, int* out) {
+    griddep_wait();
+    griddep_launch();
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        const bool ok = mbar_wait(&bar, 0, (volatile int*)&abort_flag, status);
+        *out = ok ? 1 : 0;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // fp32 SIMT path
 // ---------------------------------------------------------------------------
@@ -211,6 +261,8 @@ __global__ void k_synth_target(const int* __restrict__ drafts, const int* __rest
 // with row stride xs.stride and xs.width columns.
 __global__ void k_gemm_f32(XSegs xs, const float* __restrict__ W, float* __restrict__ Y, int M, int N, int K,
                            int ldy, int ycol0) {
+    griddep_wait();
+    griddep_launch();
     const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (wid >= (long long)M * N) return;
@@ -231,6 +283,8 @@ __global__ void k_epi_qkv_f32(const float* __restrict__ Y, int M, int Nq, int Nk
                               const int* __restrict__ len, const int* __restrict__ req_ok,
                               const float2* __restrict__ rope, float* __restrict__ q, float* __restrict__ slab,
                               long long s_req, long long s_layer, long long s_kind, long long s_kv, int layer) {
+    griddep_wait();
+    griddep_launch();
     const int ld = Nq + 2 * Nkv;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)M * ld) return;
@@ -262,6 +316,8 @@ __global__ void k_epi_inject_f32(const float* __restrict__ Y, int rows, int Nkv,
                                  const int* __restrict__ row_count, int B, const int* __restrict__ len, int cap,
                                  const float2* __restrict__ rope, float* __restrict__ slab, long long s_req,
                                  long long s_layer, long long s_kind, long long s_kv, int layer) {
+    griddep_wait();
+    griddep_launch();
     const int ld = 2 * Nkv;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)rows * ld) return;
@@ -292,12 +348,16 @@ __global__ void k_epi_inject_f32(const float* __restrict__ Y, int rows, int Nkv,
 
 // x += Y (fp32 residual), elementwise over [M, H].
 __global__ void k_resid_f32(float* __restrict__ x, const float* __restrict__ Y, long long n) {
+    griddep_wait();
+    griddep_launch();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) x[i] += Y[i];
 }
 
 // act = silu(gate) * up with Y = [gate | up] of width 2I.
 __global__ void k_swiglu_f32(const float* __restrict__ Y, float* __restrict__ act, int M, int I) {
+    griddep_wait();
+    griddep_launch();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)M * I) return;
     const int m = (int)(i / I), f = (int)(i % I);
@@ -310,6 +370,8 @@ __global__ void k_swiglu_f32(const float* __restrict__ Y, float* __restrict__ ac
 __global__ void k_attn_f32(const float* __restrict__ q, const float* __restrict__ slab, const int* __restrict__ len,
                            const int* __restrict__ req_ok, float* __restrict__ o, int gamma, int nq, int G, int d,
                            long long s_req, long long s_layer, long long s_kind, long long s_kv, int layer, float scale) {
+    griddep_wait();
+    griddep_launch();
     extern __shared__ float sh[];     // [n] scores, then [d] query
     const int j = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int m = b * gamma + j;
@@ -370,13 +432,13 @@ __global__ void k_attn_f32(const float* __restrict__ q, const float* __restrict_
 template <typename T>
 void launch_embed(const T* embed, const int* anchor, int mask_id, int B, int gamma, int H, int V, const int* len,
                   const int* committed, int cap, T* x, int* req_ok, int* status, cudaStream_t st) {
-    k_embed<T><<<B * gamma, 128, 0, st>>>(embed, anchor, mask_id, gamma, H, V, len, committed, cap, x, req_ok, status);
+    launch_k(k_embed<T>, dim3(B * gamma), dim3(128), 0, st, embed, anchor, mask_id, gamma, H, V, len, committed, cap, x, req_ok, status);
 }
 template <typename T>
 void launch_rmsnorm(const T* x, const T* g, T* y, int rows, int H, float eps, int grp, int gstride, int goff,
                     cudaStream_t st) {
     if (rows <= 0) return;
-    k_rmsnorm<T><<<rows, 256, 0, st>>>(x, g, y, H, eps, grp, gstride, goff);
+    launch_k(k_rmsnorm<T>, dim3(rows), dim3(H / (16 / (int)sizeof(T)) >= 256 ? 256 : 128), 0, st, x, g, y, H, eps, grp, gstride, goff);
 }
 template void launch_embed<float>(const float*, const int*, int, int, int, int, int, const int*, const int*, int,
                                   float*, int*, int*, cudaStream_t);
@@ -388,38 +450,41 @@ template void launch_rmsnorm<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfl
 
 void launch_lm_reduce(const float4* rec, int n_vt, int M, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st) {
-    k_lm_reduce<<<(M * 32 + 255) / 256, 256, 0, st>>>(rec, n_vt, M, gm1, req_ok, drafts, margin);
+    launch_k(k_lm_reduce, dim3((M * 32 + 255) / 256), dim3(256), 0, st, rec, n_vt, M, gm1, req_ok, drafts, margin);
 }
 void launch_top2_rows(const float* logits, int M, int V, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st) {
-    k_top2_rows<<<M, 256, 0, st>>>(logits, V, gm1, req_ok, drafts, margin);
+    launch_k(k_top2_rows, dim3(M), dim3(256), 0, st, logits, V, gm1, req_ok, drafts, margin);
 }
 void launch_accept(const int* drafts, const int* target, int B, int gamma, int V, int* len, int* committed,
                    int* accept_len, int* next_anchor, int* status, cudaStream_t st) {
-    k_accept<<<(B * 32 + 127) / 128, 128, 0, st>>>(drafts, target, B, gamma, V, len, committed, accept_len,
+    launch_k(k_accept, dim3((B * 32 + 127) / 128), dim3(128), 0, st, drafts, target, B, gamma, V, len, committed, accept_len,
                                                    next_anchor, status);
 }
 void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st) {
-    k_inject_finalize<<<(B + 127) / 128, 128, 0, st>>>(row_count, B, cap, len, status);
+    launch_k(k_inject_finalize, dim3((B + 127) / 128), dim3(128), 0, st, row_count, B, cap, len, status);
 }
 void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st) {
-    k_set_len<<<(B + 127) / 128, 128, 0, st>>>(lens, B, cap, len, committed, status);
+    launch_k(k_set_len, dim3((B + 127) / 128), dim3(128), 0, st, lens, B, cap, len, committed, status);
 }
 void launch_synth_target(const int* drafts, const int* a_plan, const int* rnd, int B, int gamma, int V, int* target,
                          cudaStream_t st) {
-    k_synth_target<<<(B * gamma + 127) / 128, 128, 0, st>>>(drafts, a_plan, rnd, B, gamma, V, target);
+    launch_k(k_synth_target, dim3((B * gamma + 127) / 128), dim3(128), 0, st, drafts, a_plan, rnd, B, gamma, V, target);
+}
+int launch_wait_selftest(int* status, int* out, cudaStream_t st) {
+    return (int)launch_k(k_wait_selftest, dim3(1), dim3(32), 0, st, status, out);
 }
 void launch_gemm_f32(const XSegs& xs, const float* W, float* Y, int M, int N, int K, int ldy, int ycol0,
                      cudaStream_t st) {
     const long long warps = (long long)M * N;
     if (warps == 0) return;
-    k_gemm_f32<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(xs, W, Y, M, N, K, ldy, ycol0);
+    launch_k(k_gemm_f32, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st, xs, W, Y, M, N, K, ldy, ycol0);
 }
 void launch_epi_qkv_f32(const float* Y, int M, int Nq, int Nkv, int d, int gamma, const int* len, const int* req_ok,
                         const float2* rope, float* q, float* slab, long long s_req, long long s_layer, long long s_kind,
                         long long s_kv, int layer, cudaStream_t st) {
     const long long n = (long long)M * (Nq + 2 * Nkv);
-    k_epi_qkv_f32<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(Y, M, Nq, Nkv, d, gamma, len, req_ok, rope, q, slab,
+    launch_k(k_epi_qkv_f32, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, Y, M, Nq, Nkv, d, gamma, len, req_ok, rope, q, slab,
                                                                s_req, s_layer, s_kind, s_kv, layer);
 }
 void launch_epi_inject_f32(const float* Y, int rows, int Nkv, int d, const int* row_start, const int* row_count, int B,
@@ -427,15 +492,15 @@ void launch_epi_inject_f32(const float* Y, int rows, int Nkv, int d, const int* 
                            long long s_kind, long long s_kv, int layer, cudaStream_t st) {
     const long long n = (long long)rows * 2 * Nkv;
     if (n == 0) return;
-    k_epi_inject_f32<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(Y, rows, Nkv, d, row_start, row_count, B, len, cap,
+    launch_k(k_epi_inject_f32, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, Y, rows, Nkv, d, row_start, row_count, B, len, cap,
                                                                   rope, slab, s_req, s_layer, s_kind, s_kv, layer);
 }
 void launch_resid_f32(float* x, const float* Y, long long n, cudaStream_t st) {
-    k_resid_f32<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(x, Y, n);
+    launch_k(k_resid_f32, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, x, Y, n);
 }
 void launch_swiglu_f32(const float* Y, float* act, int M, int I, cudaStream_t st) {
     const long long n = (long long)M * I;
-    k_swiglu_f32<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(Y, act, M, I);
+    launch_k(k_swiglu_f32, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, Y, act, M, I);
 }
 int launch_attn_f32(const float* q, const float* slab, const int* len, const int* req_ok, float* o, int B, int gamma,
                     int nq, int G, int d, long long s_req, long long s_layer, long long s_kind, long long s_kv,
@@ -448,7 +513,7 @@ int launch_attn_f32(const float* q, const float* slab, const int* len, const int
         set_to = smem;
     }
     dim3 grid(gamma, nq, B);
-    k_attn_f32<<<grid, 128, smem, st>>>(q, slab, len, req_ok, o, gamma, nq, G, d, s_req, s_layer, s_kind, s_kv, layer,
+    launch_k(k_attn_f32, dim3(grid), dim3(128), smem, st, q, slab, len, req_ok, o, gamma, nq, G, d, s_req, s_layer, s_kind, s_kv, layer,
                                         1.0f / sqrtf((float)d));
     return (int)cudaGetLastError();
 }

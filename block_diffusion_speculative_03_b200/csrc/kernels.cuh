@@ -24,6 +24,7 @@ void launch_accept(const int* drafts, const int* target, int B, int gamma, int V
                    int* accept_len, int* next_anchor, int* status, cudaStream_t st);
 void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st);
 void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st);
+int launch_wait_selftest(int* status, int* out, cudaStream_t st);
 void launch_synth_target(const int* drafts, const int* a_plan, const int* rnd, int B, int gamma, int V, int* target,
                          cudaStream_t st);
 void launch_gemm_f32(const XSegs& xs, const float* W, float* Y, int M, int N, int K, int ldy, int ycol0,

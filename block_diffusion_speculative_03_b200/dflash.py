@@ -91,6 +91,9 @@ def lib():
         "dflash_diag_timing_read": (i32, [vp, vp, C.POINTER(i32), C.POINTER(C.c_float), i32, C.POINTER(i32)]),
         "dflash_diag_timing_disable": (i32, [vp]),
         "dflash_diag_timed_name": (C.c_char_p, [i32]),
+        "dflash_diag_set_launch_mode": (i32, [i32]),
+        "dflash_diag_wait_selftest": (i32, [vp, vp, vp]),
+        "dflash_diag_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -107,7 +110,8 @@ def exported_symbols() -> list:
             "dflash_status_string", "dflash_launch_count", "dflash_diag_gemm_scratch_bytes",
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
-            "dflash_diag_timed_name"]
+            "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_wait_selftest",
+            "dflash_diag_attention"]
 
 
 def _chk(st: int, where: str, check: bool = True) -> int:
@@ -246,3 +250,15 @@ def dflash_diag_timing_disable(h: int) -> int:
 
 def dflash_diag_timed_name(kind: int) -> str:
     return lib().dflash_diag_timed_name(kind).decode()
+
+
+def dflash_diag_set_launch_mode(programmatic: bool) -> int:
+    return _chk(lib().dflash_diag_set_launch_mode(1 if programmatic else 0), "dflash_diag_set_launch_mode")
+
+
+def dflash_diag_wait_selftest(h: int, out: int, stream: int = 0) -> int:
+    return _chk(lib().dflash_diag_wait_selftest(h, out, stream), "dflash_diag_wait_selftest")
+
+
+def dflash_diag_attention(h: int, c: int, q: int, out: int, layer: int, gamma: int, stream: int = 0) -> int:
+    return _chk(lib().dflash_diag_attention(h, c, q, out, layer, gamma, stream), "dflash_diag_attention")

@@ -55,6 +55,29 @@ int dflash_diag_timing_read(dflash_handle* h, dflash_stream stream, int* kinds, 
 int dflash_diag_timing_disable(dflash_handle* h);
 const char* dflash_diag_timed_name(int kind);
 
+/* The block-attention kernel alone (bf16 handles): for every request b and
+ * layer `layer`, q (device bf16 [batch*gamma, n_q_heads*head_dim], rows b*gamma+j)
+ * attends over cache rows [0, len[b] + gamma) of that layer (the caller writes
+ * the block's own K/V rows at [len, len+gamma) and keeps len + gamma <= capacity);
+ * out: device bf16, same layout as q.  Synchronises the stream. */
+int dflash_diag_attention(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
+                          dflash_stream stream);
+
+/* Self-test of the device-side bounded wait used by the pipelined kernels: a
+ * one-warp kernel waits on a shared-memory barrier that nothing arrives at.  The
+ * wait gives up after its limit (about 2 s), records DFLASH_TIMEOUT in the
+ * handle's status word and the kernel returns, leaving the context usable.
+ * out: device int32, set to 0 when the wait ran out (1 would mean it completed).
+ * dflash_cache_status then reports DFLASH_TIMEOUT once. */
+int dflash_diag_wait_selftest(dflash_handle* h, int32_t* out, dflash_stream stream);
+
+/* Launch mode of every kernel of the library (process-wide, default 1):
+ * 1 = programmatic dependent launch (a kernel may be scheduled while the
+ * previous kernel of the stream drains; each kernel waits for its predecessor's
+ * results in-kernel, and the GEMM streams its first weight tiles before that
+ * wait), 0 = plain stream-ordered launches. */
+int dflash_diag_set_launch_mode(int programmatic);
+
 /* "sm_100a" for this build. */
 const char* dflash_diag_arch(void);
 

@@ -48,6 +48,8 @@ struct oracle_config {
     int n_sel, target_hidden, mask_id;
     int storage;            // 0: fp32 storage, R() is the identity. 1: bf16 storage.
     double rope_theta, rms_eps;
+    int acc32;              // 1: accumulate dot products in fp32 instead of fp64
+                            //    (a timing / sensitivity variant; parity uses 0)
 };
 
 // All matrices are [out, in] row-major in the storage type (uint16 bf16 bit
@@ -137,13 +139,17 @@ void oracle_rope(double* v, int d, long pos, double theta) {
 
 // Multi-head attention without a mask.  q: [nrow][nq][d]; k, v: [nkv][n][d];
 // o: [nrow][nq][d].  Query head hq reads key/value head hq / (nq/nkv).
-// Scores are scaled by 1/sqrt(d); softmax is the two-pass max / sum form.  With
-// round_p != 0 the probabilities are rounded to bf16 before they weight V.
-// The output is not rounded here.
+// Scores are scaled by 1/sqrt(d).  The softmax is written in base 2 with an
+// integer shift: t_i = s_i * log2(e) / sqrt(d), B = floor(max_i t_i),
+// e_i = 2^(t_i - B), o = sum_i e_i v_i / sum_i e_i, which is the softmax.  With
+// round_p != 0 the weights e_i are rounded to bf16 before they multiply V (the
+// denominator keeps the unrounded e_i); shifting by an integer B makes that
+// rounding independent of how the keys are split into blocks.  The output is
+// not rounded here.
 void oracle_attention(const double* q, int nrow, int nq, const double* k, const double* v,
                       int n, int nkv, int d, int round_p, double* o) {
     int G = nq / nkv;
-    double scale = 1.0 / std::sqrt((double)d);
+    const double scale = 1.4426950408889634 / std::sqrt((double)d);   // log2(e) / sqrt(d)
     #pragma omp parallel for collapse(2) schedule(static)
     for (int r = 0; r < nrow; ++r) {
         for (int hq = 0; hq < nq; ++hq) {
@@ -151,28 +157,31 @@ void oracle_attention(const double* q, int nrow, int nq, const double* k, const 
             const double* qv = q + ((long)r * nq + hq) * d;
             const double* kh = k + (long)g * n * d;
             const double* vh = v + (long)g * n * d;
-            std::vector<double> s(n > 0 ? n : 1);
+            std::vector<double> t(n > 0 ? n : 1);
             double m = -INFINITY;
             for (int i = 0; i < n; ++i) {
                 double acc = 0.0;
-                for (int t = 0; t < d; ++t) acc += qv[t] * kh[(long)i * d + t];
-                s[i] = acc * scale;
-                if (s[i] > m) m = s[i];
+                for (int u = 0; u < d; ++u) acc += qv[u] * kh[(long)i * d + u];
+                t[i] = acc * scale;
+                if (t[i] > m) m = t[i];
             }
+            const double B = std::floor(m);
             double Z = 0.0;
-            for (int i = 0; i < n; ++i) { s[i] = std::exp(s[i] - m); Z += s[i]; }
+            for (int i = 0; i < n; ++i) { t[i] = std::exp2(t[i] - B); Z += t[i]; }
             double* ov = o + ((long)r * nq + hq) * d;
-            for (int t = 0; t < d; ++t) ov[t] = 0.0;
+            for (int u = 0; u < d; ++u) ov[u] = 0.0;
             for (int i = 0; i < n; ++i) {
-                double p = s[i] / Z;
-                if (round_p) p = oracle_round_bf16(p);
-                for (int t = 0; t < d; ++t) ov[t] += p * vh[(long)i * d + t];
+                double e = round_p ? oracle_round_bf16(t[i]) : t[i];
+                for (int u = 0; u < d; ++u) ov[u] += e * vh[(long)i * d + u];
             }
+            for (int u = 0; u < d; ++u) ov[u] /= Z;
         }
     }
 }
 
 // y[m][n] = sum_k x[m][k] * W[n][k]; W in storage type, [N, K] row-major.
+static int g_acc32 = 0;   // set from oracle_config.acc32 by each entry point
+
 static void linear(const double* x, int M, int K, const void* W, int N, int storage, double* y) {
     #pragma omp parallel
     {
@@ -182,6 +191,12 @@ static void linear(const double* x, int M, int K, const void* W, int N, int stor
             for (int kk = 0; kk < K; ++kk) wrow[kk] = load(W, (long)nn * K + kk, storage);
             for (int mm = 0; mm < M; ++mm) {
                 const double* xr = x + (long)mm * K;
+                if (g_acc32) {
+                    float acc = 0.0f;
+                    for (int kk = 0; kk < K; ++kk) acc += (float)xr[kk] * (float)wrow[kk];
+                    y[(long)mm * N + nn] = acc;
+                    continue;
+                }
                 double acc = 0.0;
                 // fp64 dot product; the simd reduction only changes the order
                 // in which fp64 partial sums are added.
@@ -220,6 +235,7 @@ void oracle_loss_weights(int gamma, double* w) {
 // ---------------------------------------------------------------------------
 void oracle_fuse_context(const oracle_config* c, const oracle_weights* w,
                          const void* const* hiddens, long row_stride, int rows, double* ctx_out) {
+    g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, Ht = c->target_hidden, Kc = c->n_sel * Ht;
     std::vector<double> cat((size_t)rows * Kc);
     for (int r = 0; r < rows; ++r)
@@ -247,6 +263,7 @@ void oracle_fuse_context(const oracle_config* c, const oracle_weights* w,
 // ---------------------------------------------------------------------------
 void oracle_inject_kv(const oracle_config* c, const oracle_weights* w, const double* ctx,
                       int rows, int pos0, double* k_cache, double* v_cache, int cap) {
+    g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, d = c->head_dim, nkv = c->n_kv_heads, Nkv = nkv * d;
     std::vector<double> kk((size_t)rows * Nkv), vv((size_t)rows * Nkv);
     for (int l = 0; l < c->n_layers; ++l) {
@@ -281,6 +298,7 @@ void oracle_inject_kv(const oracle_config* c, const oracle_weights* w, const dou
 void oracle_draft_block(const oracle_config* c, const oracle_weights* w,
                         const double* k_cache, const double* v_cache, int cap, int len,
                         int anchor, int gamma, int* drafts, double* logits, double* margin) {
+    g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
     int Nq = nq * d, Nkv = nkv * d, I = c->intermediate, V = c->vocab;
     int n = len + gamma;

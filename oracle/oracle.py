@@ -24,7 +24,7 @@ class _Cfg(C.Structure):
                 ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("intermediate", C.c_int),
                 ("vocab", C.c_int), ("n_sel", C.c_int), ("target_hidden", C.c_int),
                 ("mask_id", C.c_int), ("storage", C.c_int),
-                ("rope_theta", C.c_double), ("rms_eps", C.c_double)]
+                ("rope_theta", C.c_double), ("rms_eps", C.c_double), ("acc32", C.c_int)]
 
 
 class _W(C.Structure):
@@ -143,7 +143,7 @@ class OracleDrafter:
         self.cfg = _Cfg(shape["hidden"], shape["n_layers"], shape["n_q_heads"], shape["n_kv_heads"],
                         shape["head_dim"], shape["intermediate"], shape["vocab"], shape["n_sel"],
                         shape["target_hidden"], shape["mask_id"], st,
-                        float(shape["rope_theta"]), float(shape["rms_eps"]))
+                        float(shape["rope_theta"]), float(shape["rms_eps"]), int(shape.get("acc32", 0)))
         self._keep = []
         w = _W()
 

@@ -43,13 +43,19 @@ def check_float(w: I.Workload, got: np.ndarray, ref: np.ndarray, what: str, bf16
         assert same > 0.9, (what, same)
 
 
-def check_logits(w: I.Workload, got: np.ndarray, ref: np.ndarray):
+MAX_SEEN = {"logits": 0.0}
+
+
+def check_logits(w: I.Workload, got: np.ndarray, ref: np.ndarray, bf16_tol: float = BF16_LOGIT_ABS):
     if w.dtype == "f32":
         e = rel_err(got, ref)
         assert e <= F32_LOGIT_REL, ("logits rel", e)
     else:
         e = float(np.max(np.abs(got - ref)))
-        assert e <= BF16_LOGIT_ABS, ("logits abs", e)
+        assert e <= bf16_tol, ("logits abs", e, bf16_tol)
+    MAX_SEEN["logits"] = max(MAX_SEEN["logits"], e)
+    print("%s logits %s error %.3g" % (w.name, "max rel" if w.dtype == "f32" else "max abs", e))
+    return e
 
 
 def check_drafts(got: np.ndarray, ref: np.ndarray, margin: np.ndarray):

@@ -1,0 +1,162 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark
+uses: the GPU runs the whole batch; the oracle recomputes sampled requests.
+
+Logit tolerance at these sizes: five bf16-rounded layers of width 4096 are
+chaotic with respect to rounding, so two oracles that differ only in their
+accumulation precision (fp64 vs fp32) already disagree by ~0.06 in max logit
+(0.012 rms) on these inputs.  The GPU's logits must be within
+max(3e-2, 1.5 x that oracle-vs-oracle gap measured on the same request); the
+draft tokens must still match exactly wherever the oracle's top-1 margin
+exceeds 0.1, and every length exactly.
+
+The committed context of every request is filled with seeded K/V rows from the
+input generator (the spread of injected keys/values), so the oracle needs no
+million-row prefill; the oracle gets the same generator values.  Then, per
+cycle: draft_block for the whole batch (logits, margins and drafts of the
+sampled requests against the oracle), fuse + inject of gamma verified rows per
+request (sampled rows against the oracle), accept with planned acceptance
+lengths (lengths of every request exact).
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_speculative_03_b200 import inputs as I
+from block_diffusion_speculative_03_b200.drafter import Drafter, shape_from_workload
+from oracle import oracle as O
+from tests.helpers import oracle_drafter, oracle_weights, shape_of, synth_target, to_np
+from tests.parity import BF16_LOGIT_ABS, check_drafts, check_float, check_logits
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(name, sample, cycles, gammas=None):
+    w = I.preset(name)
+    B = w.batch
+    gammas = gammas or [w.gamma]
+    gmax = max(gammas)
+    W = I.make_weights(w, device="cuda")
+    if w.tied_lm_head:
+        W["lm_head"] = W["embed"]
+    cap = max(w.context) + (cycles + 1) * gmax + 8
+    dr = Drafter(shape_from_workload(w), W, max_batch=B, max_rows=B * gmax, max_position=cap, max_gamma=gmax)
+    cache = dr.new_cache(B, cap)
+    slab = cache.slab()
+    for b in range(B):
+        T = w.context[b]
+        for l in range(w.n_layers):
+            for kind in (0, 1):
+                slab[b, l, kind, :, :T] = I.synthetic_cache_rows(w, l, kind, b, T, device="cuda")
+    cache.set_len(torch.tensor(w.context, dtype=torch.int32))
+    torch.cuda.synchronize()
+    Wh = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in W.items() if k != "layers"}
+    Wh["layers"] = [{k: v.cpu() for k, v in lw.items()} for lw in W["layers"]]
+    od = oracle_drafter(w, Wh)
+    od32 = O.OracleDrafter(dict(shape_of(w), acc32=1), oracle_weights(Wh))   # sensitivity reference
+    del Wh
+    ocache = {}
+    for b in sample:
+        T = w.context[b]
+        oc = od.new_cache(cap)
+        oc["k"][:, :, :T] = slab[b, :, 0, :, :T].double().cpu().numpy()
+        oc["v"][:, :, :T] = slab[b, :, 1, :, :T].double().cpu().numpy()
+        oc["len"] = oc["committed"] = T
+        ocache[b] = oc
+
+    anchors = I.make_anchors(w).numpy()
+    compared = 0
+    for cyc in range(cycles):
+        for g in gammas:
+            nd = g - 1
+            logits = torch.empty(B, nd, w.vocab, dtype=torch.float32, device="cuda")
+            margin = torch.empty(B, nd, dtype=torch.float32, device="cuda")
+            drafts = dr.draft_block(cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"), g,
+                                    logits=logits, margin=margin)
+            torch.cuda.synchronize()
+            assert cache.status() == 0
+            g_dr = drafts.cpu().numpy()[:, :nd]
+            assert np.all((g_dr >= 0) & (g_dr < w.vocab))
+            o_drafts = {}
+            for b in sample:
+                d_o, m_o, l_o = od.draft_block(ocache[b], int(anchors[b]), g, want_logits=True)
+                _, _, l_32 = od32.draft_block(ocache[b], int(anchors[b]), g, want_logits=True)
+                gap = float(np.max(np.abs(l_32 - l_o)))
+                tol = max(BF16_LOGIT_ABS, 1.5 * gap)
+                print("%s b=%d gamma=%d: oracle fp64-vs-fp32-accumulation logit gap %.3g -> tolerance %.3g"
+                      % (name, b, g, gap, tol))
+                check_logits(w, logits[b].double().cpu().numpy(), l_o, bf16_tol=tol)
+                compared += check_drafts(g_dr[b], d_o, m_o)
+                o_drafts[b] = d_o
+        g = gammas[0]
+        nd = g - 1
+        # the last drafted block (gamma = gammas[-1]) is verified with gamma = gammas[0]
+        # only when they agree; re-draft at gammas[0] otherwise
+        if len(gammas) > 1:
+            drafts = dr.draft_block(cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"), g)
+            torch.cuda.synchronize()
+            g_dr = drafts.cpu().numpy()[:, :nd]
+            for b in sample:
+                o_drafts[b], _, _ = od.draft_block(ocache[b], int(anchors[b]), g)
+        # verification: targets from the oracle's drafts on sampled requests (teacher forcing)
+        plan = I.plan_accept(w, cycles, gamma=g).numpy()[cyc]
+        rnd = I.random_tokens(w, (B, g), stream=300 + cyc).numpy()
+        use = np.array([o_drafts[b] if b in o_drafts else g_dr[b] for b in range(B)], dtype=np.int32)
+        target = np.stack([synth_target(use[b], int(plan[b]), rnd[b], w.vocab) for b in range(B)])
+        hid = I.make_hiddens(w, B * g, stream=400 + cyc, device="cuda")
+        ctx = dr.fuse_context(hid)
+        dr.inject_kv(cache, ctx, torch.arange(0, B * g, g, dtype=torch.int32, device="cuda"),
+                     torch.full((B,), g, dtype=torch.int32, device="cuda"))
+        acc = torch.empty(B, dtype=torch.int32, device="cuda")
+        nxt = torch.empty(B, dtype=torch.int32, device="cuda")
+        lens_before = cache.len.cpu().numpy().copy()
+        dr.accept(cache, torch.tensor(use, dtype=torch.int32, device="cuda"),
+                  torch.tensor(target, dtype=torch.int32, device="cuda"), acc, nxt)
+        torch.cuda.synchronize()
+        assert cache.status() == 0
+        acc_np, nxt_np = acc.cpu().numpy(), nxt.cpu().numpy()
+        assert np.array_equal(acc_np, plan)
+        assert np.array_equal(nxt_np, target[np.arange(B), plan])
+        comm = cache.committed.cpu().numpy()
+        assert np.array_equal(cache.len.cpu().numpy(), comm)
+        assert np.array_equal(comm, lens_before - g + plan + 1)
+        ctx_np = ctx.double().cpu().numpy()
+        slab = cache.slab()
+        for b in sample:
+            T0 = ocache[b]["len"]
+            rows = [h[b * g:(b + 1) * g].cpu() for h in hid]
+            ctx_o = od.fuse_context([to_np(r) for r in rows])
+            check_float(w, ctx_np[b * g:(b + 1) * g], ctx_o, "ctx[%d]" % b)
+            od.inject_kv(ocache[b], ctx_o)
+            st, a, nx = od.accept(ocache[b], o_drafts[b], target[b])
+            assert st == 0 and a == plan[b] and nx == nxt_np[b]
+            new = slice(T0, T0 + a + 1)
+            gk = slab[b, :, 0, :, new].double().cpu().numpy()
+            gv = slab[b, :, 1, :, new].double().cpu().numpy()
+            check_float(w, gk, ocache[b]["k"][:, :, new], "K new rows [%d]" % b)
+            check_float(w, gv, ocache[b]["v"][:, :, new], "V new rows [%d]" % b)
+            assert ocache[b]["len"] == comm[b]
+        anchors = nxt_np
+    del dr, cache, W
+    gc.collect()
+    torch.cuda.empty_cache()
+    return compared
+
+
+def test_qwen3_8b_batch1_context2048():
+    assert _run("qwen3_8b", sample=[0], cycles=3) > 0
+
+
+def test_qwen3_8b_batch32_varlen():
+    w = I.preset("qwen3_8b_b32")
+    order = np.argsort(w.context)
+    assert _run("qwen3_8b_b32", sample=[int(order[0]), int(order[-1])], cycles=2) > 0
+
+
+def test_long_context_gamma_sweep():
+    assert _run("long_ctx", sample=[2], cycles=1, gammas=[16, 8, 4]) > 0
+
+
+def test_llama31_8b_batch16():
+    assert _run("llama31_8b", sample=[5], cycles=1) > 0

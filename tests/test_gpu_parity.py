@@ -93,3 +93,16 @@ def test_inject_in_chunks_equals_all_at_once_on_gpu():
     for r in range(w.batch):
         T = w.context[r]
         assert torch.equal(sa[r, :, :, :, :T], sb[r, :, :, :, :T])
+
+
+def test_small_bf16_long_context_multi_tile_splits():
+    # 2000 / 1500 context rows: every attention split holds several K/V tiles
+    import dataclasses
+    w = dataclasses.replace(I.preset("small_bf16"), context=[2000, 1500], cycles=2)
+    pr = Pair(w)
+    pr.prefill()
+    anchors = I.make_anchors(w).numpy()
+    plan = I.plan_accept(w, w.cycles).numpy()
+    for cyc in range(w.cycles):
+        o_dr, g_dr, n = pr.draft(anchors, w.gamma)
+        anchors = pr.verify_and_accept(o_dr, w.gamma, plan[cyc], cyc)
