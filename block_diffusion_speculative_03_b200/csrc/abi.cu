@@ -240,6 +240,20 @@ int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st) {
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
 }
 
+// q of the block as a 3-D bf16 map [positions][heads][d] with box {64, G, gamma}:
+// one box gathers the G query heads of kv head g for every block position.
+bool encode_q_map(CUtensorMap* m, const void* q, int positions, int nq, int d, int G, int gamma) {
+    PFN_encodeTiled_t enc = get_encode();
+    if (!enc || ((uintptr_t)q & 15)) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nq, (cuuint64_t)positions};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)nq * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)gamma};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Activation operand map: rows x K bf16 with row stride `stride`, box rows nt.
 bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride, int nt) {
     return encode_bf16_2d(m, base, (uint64_t)K, (uint64_t)rows, (uint64_t)stride, (uint32_t)nt);
@@ -599,10 +613,11 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
         !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)))
         return DFLASH_CUDA;
     int splits, chunk;
-    attn_plan(B, c.n_kv_heads, cc->capacity, h->num_sms, splits, chunk);
+    attn_plan(B, c.n_kv_heads, cc->capacity, h->num_sms, attn_max_cluster(d), splits, chunk);
     AttnParams ap;
     std::memset(&ap, 0, sizeof(ap));
     ap.tmap = cc->tm_slab;
+    if (!encode_q_map(&ap.tq, h->q, M, c.n_q_heads, d, c.n_q_heads / c.n_kv_heads, gamma)) return DFLASH_CUDA;
     ap.q = (const bf*)h->q;
     ap.out = (bf*)h->o;
     ap.len = cc->len;
@@ -859,8 +874,15 @@ int dflash_diag_gemm_scratch_bytes(int M, int N, int K, size_t* bytes) {
     return DFLASH_OK;
 }
 
+int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
+                                 size_t scratch_bytes, int grid, int64_t* trace, dflash_stream stream);
 int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
                           size_t scratch_bytes, int grid, dflash_stream stream) {
+    return dflash_diag_gemm_bf16_traced(X, W, Y, M, N, K, scratch, scratch_bytes, grid, nullptr, stream);
+}
+
+int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
+                                 size_t scratch_bytes, int grid, int64_t* trace, dflash_stream stream) {
     size_t need = 0;
     if (dflash_diag_gemm_scratch_bytes(M, N, K, &need) != DFLASH_OK) return DFLASH_INVALID_ARG;
     if (!X || !W || !Y || !scratch || ((uintptr_t)scratch & 255)) return DFLASH_INVALID_ARG;
@@ -886,6 +908,7 @@ int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, 
     p.counters = (int*)scratch;
     p.partial = (float*)((uint8_t*)scratch + counters);
     p.status = nullptr;
+    p.trace = (long long*)trace;
     p.ctas = grid > 0 ? std::min(grid, kMaxCtas) : 0;
     int e = launch_gemm_tc(p, nt, std::min(sms, kMaxCtas), S(stream));
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
@@ -937,8 +960,15 @@ int dflash_diag_timing_disable(dflash_handle* h) {
     return DFLASH_OK;
 }
 
+int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* cc, const void* q, void* out, int layer, int gamma,
+                                 int64_t* trace, int* splits_out, dflash_stream stream);
 int dflash_diag_attention(dflash_handle* h, dflash_cache* cc, const void* q, void* out, int layer, int gamma,
                           dflash_stream stream) {
+    return dflash_diag_attention_traced(h, cc, q, out, layer, gamma, nullptr, nullptr, stream);
+}
+
+int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* cc, const void* q, void* out, int layer, int gamma,
+                                 int64_t* trace, int* splits_out, dflash_stream stream) {
     if (!h || !cc || cc->h != h || !q || !out || layer < 0 || layer >= h->cfg.n_layers || gamma < 1 ||
         gamma > h->cfg.max_gamma || h->cfg.dtype != DFLASH_BF16)
         return DFLASH_INVALID_ARG;
@@ -952,8 +982,10 @@ int dflash_diag_attention(dflash_handle* h, dflash_cache* cc, const void* q, voi
     AttnParams ap;
     std::memset(&ap, 0, sizeof(ap));
     int splits, chunk;
-    attn_plan(cc->batch, c.n_kv_heads, cc->capacity, h->num_sms, splits, chunk);
+    attn_plan(cc->batch, c.n_kv_heads, cc->capacity, h->num_sms, attn_max_cluster(d), splits, chunk);
     ap.tmap = cc->tm_slab;
+    if (!encode_q_map(&ap.tq, q, cc->batch * gamma, c.n_q_heads, d, c.n_q_heads / c.n_kv_heads, gamma))
+        return DFLASH_INVALID_ARG;
     ap.q = (const __nv_bfloat16*)q;
     ap.out = (__nv_bfloat16*)out;
     ap.len = cc->len;
@@ -971,6 +1003,8 @@ int dflash_diag_attention(dflash_handle* h, dflash_cache* cc, const void* q, voi
     ap.rows_req = cc->s_req / d;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     ap.status = h->status;
+    ap.trace = (long long*)trace;
+    if (splits_out) *splits_out = splits;
     const int e = launch_attention(ap, d, cc->batch, S(stream), &h->launches);
     if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DFLASH_CUDA;
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;

@@ -1,18 +1,25 @@
-// Block attention of the draft step (bf16 storage), split over the key axis
-// across the CTAs of one thread-block cluster.
+// Block attention of the draft step (bf16 storage) on the 5th-generation
+// tensor cores, split over the key axis across the CTAs of one cluster.
 //
-// For request b and kv head g, the G*gamma query rows (G = query heads per kv
-// head) attend to every cached row [0, len) plus the gamma block rows that the
-// QKV epilogue wrote at [len, len+gamma): no mask.  The `splits` CTAs of a
-// cluster (b, g) each take one key range: K/V tiles of 64 rows x d arrive by
-// TMA (128-byte swizzle, no multicast) into a 3-stage ring; each warp owns 16
-// query rows (and a share of every tile's keys when there are fewer than 64
-// rows), computes S = Q K^T and O += P V with mma.sync m16n8k16 (bf16 in, fp32
-// accumulate), and keeps the online-softmax row max / sum with quad shuffles.
-// Each CTA leaves its partial (m, l, O) in its own shared memory; after a
+// For request b and kv head g, the R = G*gamma query rows (G = query heads per
+// kv head) attend to every cached row [0, len) plus the gamma block rows the
+// QKV epilogue wrote at [len, len+gamma): no mask.  CTA `rank` of the cluster
+// (b, g) takes keys [rank*chunk, (rank+1)*chunk).
+//
+//   warp 0   TMA: the Q tile once (a 3-D box gathers the G heads of every block
+//            position), then K/V tiles of 64 keys into a 3-stage ring.
+//   warp 1   tcgen05.mma (one thread): S_i = Q K_i^T into one of two TMEM
+//            buffers (M = 128 padded query rows, N = 64 keys), and
+//            O += P_i V_i into the TMEM accumulator (N = head_dim, V read as
+//            an MN-major operand straight from the TMA tile).
+//   warps 2-5  softmax, one query row per thread: reads S_i from TMEM, keeps a
+//            base-2 running maximum with an integer base B, writes
+//            P_i = bf16(2^(t - B)) into shared memory for the P.V MMA, and
+//            rescales O in TMEM by an exact power of two when B grows.
+//
+// Each CTA leaves its partial (B, l, O) in its own shared memory; after a
 // cluster barrier every CTA merges a slice of the rows by reading all partials
-// through distributed shared memory, and writes the bf16 output.  No partial
-// goes through global memory and no second kernel is needed.
+// through distributed shared memory, and writes the bf16 output.
 #include <cooperative_groups.h>
 
 #include "attn.cuh"
@@ -21,42 +28,59 @@ namespace cg = cooperative_groups;
 
 namespace df {
 
-// Byte offset of element (r, c) in a [64 rows][D] bf16 tile stored as D/64
-// column blocks of [64 rows][128 B] with the 128-byte swizzle (16-byte chunk
-// index XOR row % 8), which is the layout TMA writes.
-DF_DEV uint32_t sw_off(int r, int c) {
-    return (uint32_t)((c >> 6) * (64 * 128) + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
-}
+template <int D>
+struct AttnCfg {
+    static constexpr int HALVES = D / 64;
+    static constexpr int Q_BYTES = HALVES * 128 * 128;       // 128 query rows x D
+    static constexpr int KV_BYTES = HALVES * 64 * 128;       // 64 keys x D
+    static constexpr int P_BYTES = 128 * 128;                // 128 rows x 64 keys
+    static constexpr int RING = Q_BYTES + 2 * kAttnStages * KV_BYTES + 2 * P_BYTES;
+    static constexpr int SMEM = 1024 + RING + 256;
+    static constexpr uint32_t TMEM_COLS = 256;               // S[2] (2 x 64) + O (D)
+};
 
 template <int D>
-__global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ AttnParams p) {
-    constexpr int TILE_BYTES = 64 * D * 2;
-    constexpr int NDT = D / 8;     // n-tiles of the output
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_constant__ AttnParams p) {
+    using C = AttnCfg<D>;
+    constexpr int S = kAttnStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sQ = smem;
-    uint8_t* sK = sQ + TILE_BYTES;                   // [stages]
-    uint8_t* sV = sK + kAttnStages * TILE_BYTES;     // [stages]
-    uint64_t* bars = (uint64_t*)(sV + kAttnStages * TILE_BYTES);
-    // After the key loop the ring is reused: per-warp results, then the CTA's partial.
-    float* mo = (float*)(smem + TILE_BYTES);         // [4 warps][16][D]
-    float2* mml = (float2*)(mo + 4 * 16 * D);        // [4 warps][16] (m, l)
-    float* po = (float*)(mml + 4 * 16);              // [64][D]  partial O of this CTA
-    float2* pml = (float2*)(po + 64 * D);            // [64]     (m, l) of this CTA
-    float* wts = (float*)(pml + 64);                 // [64][4]  in-CTA merge weights
-    float* cm = wts + 64 * 4;                        // [64][splits] peers' row max
-    float* cl = cm + 64 * kAttnMaxSplits;            // [64][splits] peers' row sum
-    float* cw = cl + 64 * kAttnMaxSplits;            // [64][splits] normalised merge weights
-    __shared__ int s_abort;
+    uint8_t* sK = sQ + C::Q_BYTES;                 // [S][KV_BYTES]
+    uint8_t* sV = sK + S * C::KV_BYTES;            // [S][KV_BYTES]
+    uint8_t* sP = sV + S * C::KV_BYTES;            // [2][P_BYTES]
+    uint64_t* bars = (uint64_t*)(smem + C::RING);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = q_full + 1;                // [S]
+    uint64_t* kv_empty = kv_full + S;              // [S]
+    uint64_t* s_full = kv_empty + S;               // [2]
+    uint64_t* p_full = s_full + 2;                 // [2]
+    uint64_t* o_done = p_full + 2;                 // [2]
+    uint64_t* drain = o_done + 2;
+    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    // After the key loop the front of shared memory holds this CTA's partial.
+    float* po = (float*)smem;                      // [64][D]
+    float2* pml = (float2*)(po + 64 * D);          // [64] (integer base, row sum)
+    float* cm = (float*)(pml + 64);                // [64][splits] peers' bases
+    float* cl = cm + 64 * kAttnMaxSplits;          // [64][splits] peers' sums
+    float* cw = cl + 64 * kAttnMaxSplits;          // [64][splits] merge weights
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int nsplit = p.splits;
     const int g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) tma_prefetch_desc(&p.tmap);
+    long long* trace = p.trace ? p.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 8
+                               : nullptr;
+    if (trace && tid == 0) trace[0] = (long long)globaltimer_ns();
+    if (tid == 0) {
+        tma_prefetch_desc(&p.tmap);
+        tma_prefetch_desc(&p.tq);
+    }
     griddep_wait();
     griddep_launch();
+    if (trace && tid == 0) trace[1] = (long long)globaltimer_ns();
 
     const int R = p.G * p.gamma;
     const int rows_per = (R + nsplit - 1) / nsplit;
@@ -65,7 +89,7 @@ __global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ At
         for (int r = r_lo; r < r_hi; ++r) {
             const int j = r / p.G, hh = r % p.G;
             __nv_bfloat16* dst = p.out + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D;
-            for (int c = tid; c < D; c += 128) dst[c] = f2bf(0.f);
+            for (int c = tid; c < D; c += kAttnThreads) dst[c] = f2bf(0.f);
         }
         return;
     }
@@ -73,218 +97,223 @@ __global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ At
     const int kv0 = rank * p.chunk;
     const int kv1 = min(n, kv0 + p.chunk);
     const int ntiles = kv1 > kv0 ? (kv1 - kv0 + 63) / 64 : 0;
-    int RT = (R + 15) / 16;
-    if (RT == 3) RT = 4;
-    const int NKS = 4 / RT;
-    const int rt = warp % RT, ks = warp / RT;
-    const int W = 64 / NKS;         // keys of each tile handled by this warp
     const long long rowK = (long long)b * p.rows_req + (long long)p.layer * p.rows_layer + (long long)g * p.rows_kv;
     const long long rowV = rowK + p.rows_kind;
 
     if (tid == 0) {
-        s_abort = 0;
-        for (int i = 0; i < kAttnStages; ++i) mbar_init(&bars[i], 1);
+        mbar_init(q_full, 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
+    // Query rows R..127 of the padded M = 128 tile are zero.
+    for (int idx = tid; idx < (128 - R) * C::HALVES * 8; idx += kAttnThreads) {
+        const int r = R + idx / (C::HALVES * 8), rem = idx % (C::HALVES * 8);
+        const int h = rem / 8, c16 = rem % 8;
+        *reinterpret_cast<uint4*>(sQ + h * 16384 + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async();
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-        for (int it = 0; it < min(ntiles, kAttnStages); ++it) {
-            mbar_arrive_expect_tx(&bars[it], 2 * TILE_BYTES);
-            for (int h = 0; h < D / 64; ++h) {
-                tma_load_2d(sK + it * TILE_BYTES + h * 8192, &p.tmap, &bars[it], h * 64, (int)(rowK + kv0 + it * 64));
-                tma_load_2d(sV + it * TILE_BYTES + h * 8192, &p.tmap, &bars[it], h * 64, (int)(rowV + kv0 + it * 64));
-            }
-        }
-    }
-    // Q tile: row r = j*G + h  <->  block position j, query head g*G + h.
-    for (int idx = tid; idx < 64 * (D / 8); idx += 128) {
-        const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < R) {
-            const int j = r / p.G, hh = r % p.G;
-            const __nv_bfloat16* src = p.q + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c;
-            v = *reinterpret_cast<const uint4*>(src);
-        }
-        *reinterpret_cast<uint4*>(sQ + sw_off(r, c)) = v;
-    }
-    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 128;
 
-    uint32_t qa[D / 16][4];
-    {
-        const int mi = lane >> 3;
-        const int r = rt * 16 + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const int c = kk * 16 + (mi >> 1) * 8;
-            ldmatrix_x4(smem_u32(sQ) + sw_off(r, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-        }
-    }
-
-    // Base-2 online softmax with an integer base: m_t = running max of the
-    // log2-scaled scores, m_r = floor(m_t).  Every rescale is 2^(integer), so
-    // bf16(2^(t - m_r)) rescaled later equals bf16(2^(t - final base)) exactly.
-    float m_t[2] = {-INFINITY, -INFINITY}, m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-    float o[NDT][4];
-#pragma unroll
-    for (int i = 0; i < NDT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
-    for (int it = 0; it < ntiles; ++it) {
-        const int st = it % kAttnStages;
-        const bool ok = mbar_wait(&bars[st], (uint32_t)((it / kAttnStages) & 1), (volatile int*)&s_abort, p.status);
-        if (__syncthreads_or(!ok)) break;   // leave together so the block barriers stay matched
-        const int valid = kv1 - (kv0 + it * 64);
-        if (valid < 64) {
-            // Rows past the last key may hold any bits (never-written cache
-            // slack); P is 0 there, but 0 * NaN would poison O, so zero them.
-            uint8_t* vs = sV + st * TILE_BYTES;
-            for (int idx = tid; idx < (64 - valid) * (D / 8); idx += 128) {
-                const int r = valid + idx / (D / 8), c = (idx % (D / 8)) * 8;
-                *reinterpret_cast<uint4*>(vs + sw_off(r, c)) = make_uint4(0, 0, 0, 0);
-            }
-            __syncthreads();
-        }
-        const uint32_t kb = smem_u32(sK + st * TILE_BYTES), vb = smem_u32(sV + st * TILE_BYTES);
-        const int kvbase = kv0 + it * 64 + ks * W;
-        // ---- S = Q K^T over this warp's W keys (up to 8 n-tiles of 8 keys)
-        float sc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            if (nt * 8 < W) {
-                const int r = ks * W + nt * 8 + (lane & 7);
-#pragma unroll
-                for (int kp = 0; kp < D / 32; ++kp) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(kb + sw_off(r, kp * 32 + (lane >> 3) * 8), b0, b1, b2, b3);
-                    mma_bf16_16816(sc[nt], qa[2 * kp], b0, b1);
-                    mma_bf16_16816(sc[nt], qa[2 * kp + 1], b2, b3);
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, (uint32_t)(R * D * 2));
+            for (int h = 0; h < C::HALVES; ++h)
+                tma_load_3d(sQ + h * 16384, &p.tq, q_full, h * 64, g * p.G, b * p.gamma);
+            for (int it = 0; it < ntiles; ++it) {
+                const int st = it % S;
+                if (!mbar_wait(&kv_empty[st], (uint32_t)(((it / S) & 1) ^ 1), abort_flag, p.status)) break;
+                mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
+                for (int h = 0; h < C::HALVES; ++h) {
+                    tma_load_2d(sK + st * C::KV_BYTES + h * 8192, &p.tmap, &kv_full[st], h * 64,
+                                (int)(rowK + kv0 + it * 64));
+                    tma_load_2d(sV + st * C::KV_BYTES + h * 8192, &p.tmap, &kv_full[st], h * 64,
+                                (int)(rowV + kv0 + it * 64));
                 }
             }
         }
-        // ---- online softmax (log2 domain), rows lane/4 and lane/4 + 8
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64);
+            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+            for (int it = 0; it <= ntiles && ok; ++it) {
+                if (it < ntiles) {
+                    // S_it = Q K_it^T into S buffer it & 1 (free once the softmax read S_{it-2})
+                    const int st = it % S, sb = it & 1;
+                    if (!mbar_wait(&kv_full[st], (uint32_t)((it / S) & 1), abort_flag, p.status)) { ok = false; break; }
+                    if (it >= 2 && !mbar_wait(&p_full[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + st * C::KV_BYTES);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            if (nt * 8 < W) {
-                const int kv = kvbase + nt * 8 + 2 * (lane & 3);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const bool valid_k = (kv + (c & 1)) < kv1;
-                    sc[nt][c] = valid_k ? sc[nt][c] * p.scale_log2 : -INFINITY;
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        tc_mma_bf16(tS + sb * 64, umma_desc_sw128(qa + (kk >> 2) * 16384) + 2 * (kk & 3),
+                                    umma_desc_sw128(ka + (kk >> 2) * 8192) + 2 * (kk & 3), IDESC_S, kk > 0 ? 1u : 0u);
+                    tc_commit(&s_full[sb]);
                 }
-                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
-            }
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        m_t[0] = fmaxf(m_t[0], mx0);
-        m_t[1] = fmaxf(m_t[1], mx1);
-        const float nb0 = floorf(m_t[0]), nb1 = floorf(m_t[1]);      // -inf stays -inf
-        const float base0 = (nb0 == -INFINITY) ? 0.f : nb0;
-        const float base1 = (nb1 == -INFINITY) ? 0.f : nb1;
-        const float corr0 = exp2f(m_r[0] - base0), corr1 = exp2f(m_r[1] - base1);   // 0 while m_r is -inf
-        m_r[0] = nb0;
-        m_r[1] = nb1;
-        float ls0 = 0.f, ls1 = 0.f;
+                if (it >= 1) {
+                    // O += P_j V_j for the previous tile, once its P is written
+                    const int j = it - 1, pb = j & 1;
+                    if (!mbar_wait(&p_full[pb], (uint32_t)((j >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t pa = smem_u32(sP + pb * C::P_BYTES);
+                    const uint32_t va = smem_u32(sV + (j % S) * C::KV_BYTES);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            if (nt * 8 < W) {
-                sc[nt][0] = exp2f(sc[nt][0] - base0);
-                sc[nt][1] = exp2f(sc[nt][1] - base0);
-                sc[nt][2] = exp2f(sc[nt][2] - base1);
-                sc[nt][3] = exp2f(sc[nt][3] - base1);
-                ls0 += sc[nt][0] + sc[nt][1];
-                ls1 += sc[nt][2] + sc[nt][3];
-            }
-        }
-        l_r[0] = l_r[0] * corr0 + ls0;
-        l_r[1] = l_r[1] * corr1 + ls1;
-#pragma unroll
-        for (int i = 0; i < NDT; ++i) {
-            o[i][0] *= corr0;
-            o[i][1] *= corr0;
-            o[i][2] *= corr1;
-            o[i][3] *= corr1;
-        }
-        // ---- O += P V (P rounded to bf16)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            if (kk * 16 < W) {
-                uint32_t pa[4];
-                pa[0] = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
-                pa[1] = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
-                pa[2] = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-                pa[3] = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-                const int r = ks * W + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-                for (int nd = 0; nd < D / 16; ++nd) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(vb + sw_off(r, nd * 16 + (lane >> 4) * 8), b0, b1, b2, b3);
-                    mma_bf16_16816(o[2 * nd], pa, b0, b1);
-                    mma_bf16_16816(o[2 * nd + 1], pa, b2, b3);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tO, umma_desc_sw128(pa) + 2 * kk, umma_desc_sw128_mn(va + kk * 2048, 8192, 1024),
+                                    IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&o_done[pb]);
+                    tc_commit(&kv_empty[j % S]);
                 }
             }
-        }
-        __syncthreads();
-        if (tid == 0 && it + kAttnStages < ntiles && !s_abort) {
-            const int nx = it + kAttnStages;
-            fence_proxy_async();   // order this stage's generic-proxy accesses before the TMA refill
-            mbar_arrive_expect_tx(&bars[st], 2 * TILE_BYTES);
-            for (int h = 0; h < D / 64; ++h) {
-                tma_load_2d(sK + st * TILE_BYTES + h * 8192, &p.tmap, &bars[st], h * 64, (int)(rowK + kv0 + nx * 64));
-                tma_load_2d(sV + st * TILE_BYTES + h * 8192, &p.tmap, &bars[st], h * 64, (int)(rowV + kv0 + nx * 64));
+            if (*abort_flag) {
+                tc_commit(drain);   // let the issued MMAs finish before TMEM is released
+                volatile int never = 0;
+                mbar_wait(drain, 0, &never, nullptr);
             }
         }
-    }
+    } else {
+        // ------------------------------------------------------------ softmax (one query row per thread)
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const int e = tid - 64;                        // 0..127
+        const uint32_t lanes = (uint32_t)(q4 * 32) << 16;
+        float base = -INFINITY, mt = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int it = 0; it < ntiles; ++it) {
+            const int sb = it & 1;
+            ok = mbar_wait(&s_full[sb], (uint32_t)((it >> 1) & 1), abort_flag, p.status);
+            if (named_bar_or(1, 128, !ok)) { ok = false; break; }
+            tc_fence_after();
+            if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
+            const int kvb = kv0 + it * 64;
+            const uint32_t ts = tS + lanes + sb * 64;
+            float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 1);
-        l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 2);
-    }
-    __syncthreads();   // the ring is free from here on
-
-    // ---- this CTA's partial: merge the key shares of the warps of each row tile
-    {
-        const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float v[16];
+                tmem_ld16(ts + c0, v);
 #pragma unroll
-        for (int nd = 0; nd < NDT; ++nd) {
-            *reinterpret_cast<float2*>(&mo[(warp * 16 + r0) * D + nd * 8 + c0]) = make_float2(o[nd][0], o[nd][1]);
-            *reinterpret_cast<float2*>(&mo[(warp * 16 + r0 + 8) * D + nd * 8 + c0]) = make_float2(o[nd][2], o[nd][3]);
+                for (int i = 0; i < 16; ++i)
+                    if (kvb + c0 + i < kv1) mx = fmaxf(mx, v[i] * p.scale_log2);
+            }
+            mt = fmaxf(mt, mx);
+            const float nb = floorf(mt);
+            if (it >= 2) {   // the P.V of tile it-2 read this P buffer: wait for it
+                ok = mbar_wait(&o_done[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status);
+                if (named_bar_or(1, 128, !ok)) { ok = false; break; }
+            }
+            // Rescale O and l by 2^(base - nb), an exact power of two, when any row's
+            // integer base grew (the decision is taken by all 128 threads together:
+            // the TMEM accesses are warp-collective; other rows scale by 1).
+            const bool grow = nb > base;
+            if (named_bar_or(1, 128, grow && it >= 1)) {
+                ok = mbar_wait(&o_done[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), abort_flag, p.status);
+                if (named_bar_or(1, 128, !ok)) { ok = false; break; }
+                tc_fence_after();
+                const float f = grow ? exp2f(base - nb) : 1.0f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tO + lanes + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] *= f;
+                    tmem_st16(tO + lanes + c0, v);
+                }
+                tmem_wait_st();
+                l *= f;
+            }
+            if (grow) base = nb;
+            // The last tile of a split may extend past the last key: zero those V
+            // rows (P is 0 there, but 0 * NaN from never-written cache slack is NaN).
+            const int valid = kv1 - kvb;
+            if (valid < 64) {
+                uint8_t* vs = sV + (it % S) * C::KV_BYTES;
+                for (int idx = e; idx < (64 - valid) * C::HALVES * 8; idx += 128) {
+                    const int r = valid + idx / (C::HALVES * 8), rem = idx % (C::HALVES * 8);
+                    *reinterpret_cast<uint4*>(vs + (rem / 8) * 8192 + r * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            // P = bf16(2^(t - base)) into the swizzled K-major P tile, row `row`.
+            uint8_t* prow = sP + sb * C::P_BYTES + row * 128;
+            const float bb = (base == -INFINITY) ? 0.f : base;
+            float ls = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float v[16];
+                tmem_ld16(ts + c0, v);
+                uint32_t pk[8];
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    const float t0 = (kvb + c0 + i < kv1) ? v[i] * p.scale_log2 : -INFINITY;
+                    const float t1 = (kvb + c0 + i + 1 < kv1) ? v[i + 1] * p.scale_log2 : -INFINITY;
+                    const float e0 = exp2f(t0 - bb), e1 = exp2f(t1 - bb);
+                    ls += e0 + e1;
+                    pk[i / 2] = pack_bf16(e0, e1);
+                }
+                const int ch = c0 >> 3;   // 16-byte chunk of keys c0..c0+7
+                *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+            l += ls;
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&p_full[sb]);
         }
-        if ((lane & 3) == 0) {
-            mml[warp * 16 + r0] = make_float2(m_r[0], l_r[0]);
-            mml[warp * 16 + r0 + 8] = make_float2(m_r[1], l_r[1]);
+        // O of the whole split, once its last P.V has landed.
+        if (ok && ntiles >= 1) {
+            ok = mbar_wait(&o_done[(ntiles - 1) & 1], (uint32_t)(((ntiles - 1) >> 1) & 1), abort_flag, p.status);
+            ok = !named_bar_or(1, 128, !ok);
+            tc_fence_after();
         }
+        if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
+        named_bar_sync(1, 128);   // every softmax thread is past its P writes before the front is reused
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+            if (ok && ntiles >= 1) {
+                tmem_ld16(tO + lanes + c0, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            }
+            if (row < 64) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) po[row * D + c0 + i] = v[i];
+            }
+        }
+        if (row < 64) pml[row] = make_float2(base, ok ? l : 0.f);
     }
+    tc_fence_before();
     __syncthreads();
-    for (int r = tid; r < R; r += 128) {
-        const int t = r >> 4, rr = r & 15;
-        float M = -INFINITY;
-        for (int k2 = 0; k2 < NKS; ++k2) M = fmaxf(M, mml[(t + k2 * RT) * 16 + rr].x);
-        const float base = (M == -INFINITY) ? 0.f : M;
-        float L = 0.f;
-        for (int k2 = 0; k2 < NKS; ++k2) {
-            const float2 ml = mml[(t + k2 * RT) * 16 + rr];
-            const float wk = exp2f(ml.x - base);
-            wts[r * 4 + k2] = wk;
-            L += wk * ml.y;
-        }
-        pml[r] = make_float2(M, L);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    __syncthreads();
-    for (int idx = tid; idx < R * D; idx += 128) {
-        const int r = idx / D, c = idx % D, t = r >> 4, rr = r & 15;
-        float acc = 0.f;
-        for (int k2 = 0; k2 < NKS; ++k2) acc += wts[r * 4 + k2] * mo[((t + k2 * RT) * 16 + rr) * D + c];
-        po[r * D + c] = acc;
-    }
+    if (trace && tid == 0) trace[5] = (long long)globaltimer_ns();
 
     // ---- merge the cluster's partials through distributed shared memory
     cluster.sync();
+    if (trace && tid == 0) trace[6] = (long long)globaltimer_ns();
     const float* rpo[kAttnMaxSplits];
     const float2* rpml[kAttnMaxSplits];
 #pragma unroll
@@ -293,29 +322,30 @@ __global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ At
         rpml[s2] = s2 < nsplit ? cluster.map_shared_rank(pml, s2) : pml;
     }
     const int nr = r_hi - r_lo;
-    for (int idx = tid; idx < nr * nsplit; idx += 128) {
+    for (int idx = tid; idx < nr * nsplit; idx += kAttnThreads) {
         const int r = r_lo + idx / nsplit, s2 = idx % nsplit;
         const float2 ml = rpml[s2][r];
         cm[idx] = ml.x;
         cl[idx] = ml.y;
     }
     __syncthreads();
-    for (int rr = tid; rr < nr; rr += 128) {
+    for (int rr = tid; rr < nr; rr += kAttnThreads) {
         float M = -INFINITY;
-        for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, cm[rr * nsplit + s2]);
-        const float base = (M == -INFINITY) ? 0.f : M;
+        for (int s2 = 0; s2 < nsplit; ++s2)
+            if (cl[rr * nsplit + s2] > 0.f) M = fmaxf(M, cm[rr * nsplit + s2]);
+        const float bm = (M == -INFINITY) ? 0.f : M;
         float L = 0.f;
         for (int s2 = 0; s2 < nsplit; ++s2) {
-            const float l = cl[rr * nsplit + s2];
-            const float wv = l > 0.f ? exp2f(cm[rr * nsplit + s2] - base) : 0.f;
+            const float lv = cl[rr * nsplit + s2];
+            const float wv = lv > 0.f ? exp2f(cm[rr * nsplit + s2] - bm) : 0.f;
             cw[rr * nsplit + s2] = wv;
-            L += wv * l;
+            L += wv * lv;
         }
         const float inv = L > 0.f ? 1.0f / L : 0.f;
         for (int s2 = 0; s2 < nsplit; ++s2) cw[rr * nsplit + s2] *= inv;
     }
     __syncthreads();
-    for (int idx = tid; idx < nr * D; idx += 128) {
+    for (int idx = tid; idx < nr * D; idx += kAttnThreads) {
         const int rr = idx / D, c = idx % D, r = r_lo + rr;
         float v[kAttnMaxSplits];
 #pragma unroll
@@ -327,17 +357,34 @@ __global__ void __launch_bounds__(128) k_attn_cluster(const __grid_constant__ At
         const int j = r / p.G, hh = r % p.G;
         p.out[((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c] = f2bf(acc);
     }
+    if (trace && tid == 0) trace[7] = (long long)globaltimer_ns();
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
 }
 
-int attn_smem_bytes(int d) {
-    return 1024 + (1 + 2 * kAttnStages) * 64 * d * 2 + 64;
+int attn_smem_bytes(int d) { return d == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
+
+int attn_max_cluster(int d) {
+    static int cached[2] = {0, 0};
+    int& c = cached[d == 128 ? 1 : 0];
+    if (c) return c;
+    void (*kern)(AttnParams) = (d == 128) ? k_attn_tc<128> : k_attn_tc<64>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(d));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kAttnMaxSplits, 1, 1);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = attn_smem_bytes(d);
+    int size = 0;
+    if (cudaOccupancyMaxPotentialClusterSize(&size, kern, &cfg) != cudaSuccess || size < 1) size = 1;
+    cudaGetLastError();
+    c = size < kAttnMaxSplits ? size : kAttnMaxSplits;
+    return c;
 }
 
-void attn_plan(int B, int nkv, int cap, int num_sms, int& splits, int& chunk) {
+// One wave: at most one CTA per SM over all clusters, clusters of <= max_cluster.
+void attn_plan(int B, int nkv, int cap, int num_sms, int max_cluster, int& splits, int& chunk) {
     const int tiles = (cap + 63) / 64;
-    int s = (num_sms + B * nkv - 1) / (B * nkv);
-    s = s < 1 ? 1 : (s > kAttnMaxSplits ? kAttnMaxSplits : s);
+    int s = num_sms / (B * nkv);
+    s = s < 1 ? 1 : (s > max_cluster ? max_cluster : s);
     if (s > tiles) s = tiles;
     chunk = ((tiles + s - 1) / s) * 64;
     splits = (cap + chunk - 1) / chunk;
@@ -345,7 +392,7 @@ void attn_plan(int B, int nkv, int cap, int num_sms, int& splits, int& chunk) {
 
 int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, long long* launches) {
     const int smem = attn_smem_bytes(d);
-    void (*kern)(AttnParams) = (d == 128) ? k_attn_cluster<128> : k_attn_cluster<64>;
+    void (*kern)(AttnParams) = (d == 128) ? k_attn_tc<128> : k_attn_tc<64>;
     static bool done128 = false, done64 = false;
     bool& done = (d == 128) ? done128 : done64;
     if (!done) {
@@ -356,7 +403,7 @@ int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, lon
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.splits, p.nkv, B);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(kAttnThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];

@@ -6,6 +6,7 @@ namespace df {
 
 struct AttnParams {
     CUtensorMap tmap;            // cache slab as 2-D [rows, d] bf16, box {64, 64}, 128-byte swizzle
+    CUtensorMap tq;              // q as 3-D [B*gamma][nq][d] bf16, box {64, G, gamma}, 128-byte swizzle
     const __nv_bfloat16* q;      // [B*gamma, nq*d]
     __nv_bfloat16* out;          // [B*gamma, nq*d]
     const int* len;
@@ -14,14 +15,21 @@ struct AttnParams {
     long long rows_req, rows_layer, rows_kind, rows_kv;
     float scale_log2;            // log2(e) / sqrt(d)
     int* status;
+    // Diagnostic trace (null in normal use): per CTA 8 globaltimer stamps (ns):
+    // entry, past the dependency wait, Q staged, first tile landed, key loop done,
+    // partial ready, past the first cluster barrier, merge done.
+    long long* trace;
 };
 
 constexpr int kAttnStages = 3;
+constexpr int kAttnThreads = 192;   // TMA warp, MMA warp, 4 softmax warps
 constexpr int kAttnMaxSplits = 8;   // CTAs per cluster (portable cluster size)
 
 int attn_smem_bytes(int d);
+// Largest cluster the device schedules for the attention kernel (<= kAttnMaxSplits).
+int attn_max_cluster(int d);
 // Splits (= cluster size) and key rows per split for B requests of `cap` positions.
-void attn_plan(int B, int nkv, int cap, int num_sms, int& splits, int& chunk);
+void attn_plan(int B, int nkv, int cap, int num_sms, int max_cluster, int& splits, int& chunk);
 // Launch the cluster kernel: grid (splits, nkv, B), cluster (splits, 1, 1).
 int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, long long* launches);
 

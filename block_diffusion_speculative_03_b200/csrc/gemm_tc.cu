@@ -10,19 +10,24 @@
 
 namespace df {
 
+// Tile configuration per token width NT: one CTA per SM with the deepest ring
+// that fits (two CTAs per SM with half the ring measured slower at batch 1).
 template <int NT>
 struct GemmCfg {
+    static constexpr bool TWO_PER_SM = false;
     static constexpr int A_BYTES = 128 * 128;            // 128 rows x 64 bf16
     static constexpr int B_BYTES = NT * 128;             // NT rows x 64 bf16
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int CH = NT < 32 ? NT : 32;         // epilogue column chunk
-    static constexpr int XCH_FLOATS = 128 * 33;
+    static constexpr int XCH_FLOATS = 128 * (CH + 1);
     static constexpr int MISC_BYTES = 4096;
-    static constexpr int BUDGET = 232448 - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
+    static constexpr int SMEM_CAP = TWO_PER_SM ? (233472 / 2 - 2048) : 232448;
+    static constexpr int BUDGET = SMEM_CAP - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
     static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCH_FLOATS * 4 + MISC_BYTES;
     static constexpr uint32_t TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
+    static constexpr int MIN_BLOCKS = TWO_PER_SM ? 2 : 1;
 };
 
 DF_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
@@ -39,7 +44,7 @@ DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2
 }
 
 template <int NT>
-__global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const __grid_constant__ GemmParams p) {
     using C = GemmCfg<NT>;
     constexpr int S = C::STAGES;
     constexpr int CH = C::CH;
@@ -61,6 +66,9 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
     float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 8 : nullptr;
+    const long long clk0 = clock64();
+    if (trace && threadIdx.x == 0) trace[0] = (long long)globaltimer_ns();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -117,6 +125,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                 u += kb1 - kb0;
             }
             griddep_wait();
+            if (trace) trace[1] = (long long)globaltimer_ns();
             int stage = 0;
             uint32_t round = 0;
             long long issued = 0;
@@ -177,6 +186,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                 const uint32_t d = tmem + (uint32_t)(buf * NT);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&full[stage], round & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (trace && seg == 0 && kb == kb0) trace[2] = (long long)globaltimer_ns();
                     tc_fence_after();
                     const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
                     const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
@@ -191,6 +201,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                 ++seg;
                 u += kb1 - kb0;
             }
+            if (trace) trace[3] = (long long)globaltimer_ns();
             if (*abort_flag) {
                 // Drain the MMAs already issued before TMEM is released.
                 tc_commit(drain);
@@ -214,6 +225,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
             const uint32_t use = (uint32_t)(seg >> 1);
             const bool ok = mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
             if (named_bar_or(1, 128, !ok)) break;   // leave together: later named barriers stay matched
+            if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
             tc_fence_after();
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
             const bool whole = (kb0 == 0 && kb1 == KB);
@@ -337,7 +349,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                     }
                     case EPI_SWIGLU: {
 #pragma unroll
-                        for (int i = 0; i < CH; ++i) xch[row * 33 + i] = v[i];
+                        for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
                         named_bar_sync(1, 128);
                         if (row < 64) {
                             __nv_bfloat16* o = (__nv_bfloat16*)p.out;
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
 #pragma unroll
                             for (int i = 0; i < CH; ++i)
                                 if (mbase + i < p.M) {
-                                    const float up = xch[(row + 64) * 33 + i];
+                                    const float up = xch[(row + 64) * (CH + 1) + i];
                                     o[(size_t)(mbase + i) * p.ldo + f] = f2bf(silu(v[i]) * up);
                                 }
                         }
@@ -363,7 +375,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                         const int d = p.d, half = d >> 1;
                         const int i_in = lr % d;
 #pragma unroll
-                        for (int i = 0; i < CH; ++i) xch[row * 33 + i] = v[i];
+                        for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
                         named_bar_sync(1, 128);
                         const int prow = (i_in < half) ? row + half : row - half;
                         if (row_ok) {
@@ -382,7 +394,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
                                 const int pos = tok_pos[c0 + i];
                                 float x = v[i];
                                 if (rotate) {
-                                    const float pr = xch[prow * 33 + i];
+                                    const float pr = xch[prow * (CH + 1) + i];
                                     x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
                                 }
                                 if (is_q) {
@@ -441,6 +453,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
             ++seg;
             u += kb1 - kb0;
         }
+        if (trace && e == 0) trace[5] = (long long)globaltimer_ns();
     }
 
     tc_fence_before();
@@ -448,6 +461,10 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ Gemm
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (trace && threadIdx.x == 0) {
+        trace[6] = (long long)globaltimer_ns();
+        trace[7] = clock64() - clk0;
     }
 }
 

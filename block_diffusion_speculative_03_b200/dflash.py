@@ -94,6 +94,8 @@ def lib():
         "dflash_diag_set_launch_mode": (i32, [i32]),
         "dflash_diag_wait_selftest": (i32, [vp, vp, vp]),
         "dflash_diag_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
+        "dflash_diag_gemm_bf16_traced": (i32, [vp, vp, vp, i32, i32, i32, vp, sz, i32, vp, vp]),
+        "dflash_diag_attention_traced": (i32, [vp, vp, vp, vp, i32, i32, vp, C.POINTER(i32), vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -111,7 +113,8 @@ def exported_symbols() -> list:
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_wait_selftest",
-            "dflash_diag_attention"]
+            "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
+            "dflash_diag_attention_traced"]
 
 
 def _chk(st: int, where: str, check: bool = True) -> int:
@@ -262,3 +265,18 @@ def dflash_diag_wait_selftest(h: int, out: int, stream: int = 0) -> int:
 
 def dflash_diag_attention(h: int, c: int, q: int, out: int, layer: int, gamma: int, stream: int = 0) -> int:
     return _chk(lib().dflash_diag_attention(h, c, q, out, layer, gamma, stream), "dflash_diag_attention")
+
+
+def dflash_diag_gemm_bf16_traced(X: int, W: int, Y: int, M: int, N: int, K: int, scratch: int, scratch_bytes: int,
+                                 grid: int, trace: int, stream: int = 0) -> int:
+    return _chk(lib().dflash_diag_gemm_bf16_traced(X, W, Y, M, N, K, scratch, scratch_bytes, grid, trace, stream),
+                "dflash_diag_gemm_bf16_traced")
+
+
+def dflash_diag_attention_traced(h: int, c: int, q: int, out: int, layer: int, gamma: int, trace: int,
+                                 stream: int = 0) -> int:
+    """Returns the split count the kernel used."""
+    sp = C.c_int(0)
+    _chk(lib().dflash_diag_attention_traced(h, c, q, out, layer, gamma, trace, C.byref(sp), stream),
+         "dflash_diag_attention_traced")
+    return sp.value

@@ -28,6 +28,13 @@ int dflash_diag_gemm_scratch_bytes(int M, int N, int K, size_t* bytes);
 int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, int K,
                           void* scratch, size_t scratch_bytes, int grid, dflash_stream stream);
 
+/* Same, recording a per-CTA timeline into trace (device int64[grid * 8]):
+ * globaltimer stamps (ns) at entry, producer past the dependency wait, first
+ * stage landed, last MMA issued, accumulators drained, epilogue done, exit;
+ * then the CTA's clock64 span. */
+int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
+                                 size_t scratch_bytes, int grid, int64_t* trace, dflash_stream stream);
+
 /* Work partition of the persistent split-K GEMM (host only, no CUDA call).
  * `units` k-blocks in total, `kb` k-blocks per output tile, `ctas` CTAs.  For
  * output tile `tile`: first_cta = first CTA contributing to it, n_contrib = the
@@ -62,6 +69,13 @@ const char* dflash_diag_timed_name(int kind);
  * out: device bf16, same layout as q.  Synchronises the stream. */
 int dflash_diag_attention(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
                           dflash_stream stream);
+
+/* Same, recording per-CTA timestamps into trace (device int64[batch * n_kv_heads
+ * * splits * 8]: entry, past the dependency wait, Q staged, first tile landed,
+ * key loop done, partial ready, past the cluster barrier, merge done) and the
+ * split count used into *splits_out (host int, may be NULL). */
+int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
+                                 int64_t* trace, int* splits_out, dflash_stream stream);
 
 /* Self-test of the device-side bounded wait used by the pipelined kernels: a
  * one-warp kernel waits on a shared-memory barrier that nothing arrives at.  The
