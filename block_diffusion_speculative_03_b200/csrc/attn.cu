@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
             bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+            if (trace) trace[2] = (long long)globaltimer_ns();
             for (int it = 0; it <= ntiles && ok; ++it) {
                 if (it < ntiles) {
                     // S_it = Q K_it^T into S buffer it & 1 (free once the softmax read S_{it-2})
@@ -207,14 +208,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
             const int kvb = kv0 + it * 64;
             const uint32_t ts = tS + lanes + sb * 64;
+            // the row's 64 scores, in log2 units, masked past the last key
+            float t[64];
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) tmem_ld16(ts + c0, t + c0);
+            const int nvalid = kv1 - kvb;
             float mx = -INFINITY;
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float v[16];
-                tmem_ld16(ts + c0, v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (kvb + c0 + i < kv1) mx = fmaxf(mx, v[i] * p.scale_log2);
+            for (int i = 0; i < 64; ++i) {
+                t[i] = (i < nvalid) ? t[i] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, t[i]);
             }
             mt = fmaxf(mt, mx);
             const float nb = floorf(mt);
@@ -259,14 +262,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             float ls = 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < 64; c0 += 16) {
-                float v[16];
-                tmem_ld16(ts + c0, v);
                 uint32_t pk[8];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
-                    const float t0 = (kvb + c0 + i < kv1) ? v[i] * p.scale_log2 : -INFINITY;
-                    const float t1 = (kvb + c0 + i + 1 < kv1) ? v[i + 1] * p.scale_log2 : -INFINITY;
-                    const float e0 = exp2f(t0 - bb), e1 = exp2f(t1 - bb);
+                    const float e0 = ex2_fast(t[c0 + i] - bb), e1 = ex2_fast(t[c0 + i + 1] - bb);
                     ls += e0 + e1;
                     pk[i / 2] = pack_bf16(e0, e1);
                 }
@@ -345,17 +344,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         for (int s2 = 0; s2 < nsplit; ++s2) cw[rr * nsplit + s2] *= inv;
     }
     __syncthreads();
-    for (int idx = tid; idx < nr * D; idx += kAttnThreads) {
-        const int rr = idx / D, c = idx % D, r = r_lo + rr;
-        float v[kAttnMaxSplits];
-#pragma unroll
-        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) v[s2] = s2 < nsplit ? rpo[s2][r * D + c] : 0.f;
-        float acc = 0.f;
+    for (int idx = tid; idx < nr * (D / 4); idx += kAttnThreads) {
+        const int rr = idx / (D / 4), c = (idx % (D / 4)) * 4, r = r_lo + rr;
+        float4 v[kAttnMaxSplits];
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
-            if (s2 < nsplit) acc += cw[rr * nsplit + s2] * v[s2];
+            v[s2] = s2 < nsplit ? *reinterpret_cast<const float4*>(rpo[s2] + r * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+            if (s2 < nsplit) {
+                const float wv = cw[rr * nsplit + s2];
+                acc.x += wv * v[s2].x;
+                acc.y += wv * v[s2].y;
+                acc.z += wv * v[s2].z;
+                acc.w += wv * v[s2].w;
+            }
+        }
         const int j = r / p.G, hh = r % p.G;
-        p.out[((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c] = f2bf(acc);
+        __nv_bfloat16* dst = p.out + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c;
+        *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc.x, acc.y);
+        *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc.z, acc.w);
     }
     if (trace && tid == 0) trace[7] = (long long)globaltimer_ns();
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it

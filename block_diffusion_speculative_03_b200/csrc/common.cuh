@@ -287,6 +287,13 @@ DF_DEV void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 2^x with the MUFU.EX2 hardware instruction (ex2.approx.ftz: relative error
+// about 2^-22, -inf -> +0).
+DF_DEV float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 DF_DEV uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
