@@ -74,6 +74,27 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------------------
+# Replicas across ranks: every rank runs its own requests (no collective in the
+# step); a timed region's length is the max over ranks and the rate counts the
+# units of all ranks.
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, device) -> float:
+    """Max of this rank's time over all ranks (the value itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, ms: float) -> float:
+    """Units per second of the whole job: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # Algorithmic bytes per launch group (each weight byte once, activations in and
 # out once, each KV byte once per request and layer).
 # ---------------------------------------------------------------------------
@@ -374,13 +395,11 @@ def run_gpu(args):
     clocks = stop_sampler(sampler, max_sm, t_wall0, t_wall1)
     if world > 1:
         dist.barrier()
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dev)
     status = cache.status()
     assert status == 0, "device status %d" % status
     ms_step = ms / K
-    blocks_per_s = world * B * K / (ms / 1e3)
+    blocks_per_s = whole_job_rate(world, B, K, ms)
 
     hbm_peak, tc_peak, peak_src = measured_peaks()
     ab = algorithmic_bytes(w, B, g, T)
@@ -439,14 +458,10 @@ def run_gpu(args):
             i += 1
         e1.record(st)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         h2d = sum(x.numel() * x.element_size() for x in pin_hid[0])
         d2h = (out_dr.numel() + out_acc.numel() + out_nxt.numel()) * 4
-        e2e = {"value": world * B * K / (ems / 1e3), "unit": "blocks/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(world, B, K, ems), "unit": "blocks/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems / K}
     assert cache.status() == 0
 
