@@ -26,15 +26,12 @@ void ensure_carveout(const void* fn) {
     cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     done.push_back(fn);
 }
-}  // namespace df
-
-namespace {
 
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                       CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-PFN_encodeTiled_t get_encode() {
+static PFN_encodeTiled_t get_encode() {
     static PFN_encodeTiled_t fn = nullptr;
     if (!fn) {
         void* p = nullptr;
@@ -62,6 +59,9 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t r
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+}  // namespace df
+
+namespace {
 
 inline size_t al(size_t v, size_t a = 1024) { return (v + a - 1) / a * a; }
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }

@@ -112,6 +112,12 @@ inline int pick_nt(int M) {
 // ctas) and launches on `stream`.  Returns a cudaError_t.
 int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream);
 
+// 2-D bf16 tensor map (abi.cu): `inner` contiguous elements per row, `rows`
+// rows of `stride` elements, box {64, box_rows}, 128-byte swizzle, zero fill
+// out of bounds.  False when the driver's encoder rejects it.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                    uint32_t box_rows);
+
 // Bytes of split-tile partial scratch for ctas CTAs at tile width nt.
 inline size_t gemm_partial_bytes(int ctas, int nt) { return (size_t)2 * ctas * nt * 128 * sizeof(float); }
 

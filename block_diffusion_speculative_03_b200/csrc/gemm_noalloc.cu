@@ -1,0 +1,104 @@
+// The split-K tensor-core GEMM with its scratch in a static device array, for
+// callers that must not allocate device memory.
+//
+// dflash_diag_gemm_bf16 takes its split-tile partials and tile counters from
+// a buffer the caller allocates.  Some callers cannot provide one: a host that
+// owns all device memory through its own pool and hands a library no
+// allocator, a serving loop that forbids allocator calls between requests
+// (an allocation can synchronise the device or fragment the pool), or code
+// that must not grow its footprint after start-up.  For them this variant
+// keeps the scratch in a fixed array of this file's module, reserved when the
+// library's module loads, and never calls cudaMalloc, cudaFree or any library
+// that allocates.
+//
+// The kernel is the same persistent split-K kernel (gemm_tc.cu); only where
+// its scratch lives differs.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dflash.h"
+#include "../../include/dflash_diag.h"
+#include "common.cuh"
+#include "gemm.cuh"
+
+using namespace df;
+
+namespace {
+
+// Split-tile partials ([2 * ctas][nt][128] fp32) after the tile counters
+// (one int per output tile, 256-byte aligned).  One array per device: a
+// __device__ variable is instantiated in every context that loads the module.
+static __device__ __align__(256) unsigned char g_gemm_scratch[DFLASH_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxCtas = 160;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of this device's array, looked up once per device with that
+// device current.  The first lookup may load the module into the context.
+int scratch_ptr(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return DFLASH_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_gemm_scratch) != cudaSuccess || !p) return DFLASH_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return DFLASH_OK;
+}
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+}  // namespace
+
+int dflash_diag_gemm_bf16_noalloc(const void* X, const void* W, float* Y, int M, int N, int K, int grid,
+                                  dflash_stream stream) {
+    if (!X || !W || !Y || M < 1 || M > 4096 || N < 1 || K < 8 || K % 8 || grid < 0) return DFLASH_INVALID_ARG;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFLASH_CUDA;
+    const int nt = pick_nt(M);
+    const long long tiles = (long long)ceil_div(N, 128) * ceil_div(M, nt);
+    const long long units = tiles * ceil_div(K, 64);
+    // the CTA count the launcher will use (it never exceeds the unit count)
+    int ctas = std::min(sms, kMaxCtas);
+    if (grid > 0) ctas = std::min(grid, ctas);
+    if ((long long)ctas > units) ctas = (int)units;
+    const size_t counter_bytes = round_up((size_t)tiles * sizeof(int), 256);
+    const size_t need = counter_bytes + gemm_partial_bytes(ctas, nt);
+    if (need > (size_t)DFLASH_NOALLOC_SCRATCH_BYTES) return DFLASH_WORKSPACE;
+
+    void* scratch = nullptr;
+    int st = scratch_ptr(dev, &scratch);
+    if (st != DFLASH_OK) return st;
+
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!encode_bf16_2d(&p.ta[0], W, K, N, K, 128) || !encode_bf16_2d(&p.tb[0], X, K, M, K, nt))
+        return DFLASH_INVALID_ARG;
+    p.amat[0].rows = N;
+    p.n_amat = 1;
+    p.kb_per_b = ceil_div(K, 64);
+    p.M = M;
+    p.K = K;
+    p.epi = EPI_F32;
+    p.out = Y;
+    p.ldo = N;
+    p.counters = (int*)scratch;
+    p.partial = (float*)((unsigned char*)scratch + counter_bytes);
+    p.status = nullptr;
+    p.trace = nullptr;
+    p.ctas = ctas;   // the scratch above is sized for exactly this many CTAs
+    cudaStream_t s = (cudaStream_t)stream;
+    // The array keeps whatever the previous call left.  The kernel returns
+    // the counters to zero, but a call that stopped early (a timed-out wait)
+    // would leave them set, so they are cleared here; the partials are always
+    // written before they are read and need no clearing.
+    if (cudaMemsetAsync(p.counters, 0, counter_bytes, s) != cudaSuccess) return DFLASH_CUDA;
+    return launch_gemm_tc(p, nt, std::min(sms, kMaxCtas), s) == 0 ? DFLASH_OK : DFLASH_CUDA;
+}

@@ -96,6 +96,7 @@ def lib():
         "dflash_diag_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
         "dflash_diag_gemm_bf16_traced": (i32, [vp, vp, vp, i32, i32, i32, vp, sz, i32, vp, vp]),
         "dflash_diag_attention_traced": (i32, [vp, vp, vp, vp, i32, i32, vp, C.POINTER(i32), vp]),
+        "dflash_diag_gemm_bf16_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -114,7 +115,7 @@ def exported_symbols() -> list:
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_wait_selftest",
             "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
-            "dflash_diag_attention_traced"]
+            "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc"]
 
 
 def _chk(st: int, where: str, check: bool = True) -> int:
@@ -214,6 +215,16 @@ def dflash_diag_gemm_bf16(X: int, W: int, Y: int, M: int, N: int, K: int, scratc
                           grid: int = 0, stream: int = 0, check: bool = True) -> int:
     return _chk(lib().dflash_diag_gemm_bf16(X, W, Y, M, N, K, scratch, scratch_bytes, grid, stream),
                 "dflash_diag_gemm_bf16", check)
+
+
+DFLASH_NOALLOC_SCRATCH_BYTES = 6 << 20
+
+
+def dflash_diag_gemm_bf16_noalloc(X: int, W: int, Y: int, M: int, N: int, K: int, grid: int = 0, stream: int = 0,
+                                  check: bool = True) -> int:
+    """The same GEMM with its scratch in the library's static device array (no allocation)."""
+    return _chk(lib().dflash_diag_gemm_bf16_noalloc(X, W, Y, M, N, K, grid, stream),
+                "dflash_diag_gemm_bf16_noalloc", check)
 
 
 def dflash_diag_partition(units: int, kb: int, ctas: int, tile: int):

@@ -35,6 +35,39 @@ int dflash_diag_gemm_bf16(const void* X, const void* W, float* Y, int M, int N, 
 int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, int N, int K, void* scratch,
                                  size_t scratch_bytes, int grid, int64_t* trace, dflash_stream stream);
 
+/* Size of the static device array that dflash_diag_gemm_bf16_noalloc keeps its
+ * scratch in (6 MiB per device, reserved when the library's module loads). */
+#define DFLASH_NOALLOC_SCRATCH_BYTES (6u << 20)
+
+/* dflash_diag_gemm_bf16 without caller scratch and without any device
+ * allocation.  This is a library utility with no counterpart in the DFlash
+ * method; it serves callers that cannot allocate device memory (a host that
+ * owns all memory through its own pool, a serving loop that forbids allocator
+ * calls).  The split-tile partials and tile counters live in a static device
+ * array of DFLASH_NOALLOC_SCRATCH_BYTES; nothing is allocated, by this call or
+ * any library it uses.
+ *
+ * Same operands, layout and result as dflash_diag_gemm_bf16: X device bf16
+ * [M, K], W device bf16 [N, K], Y device fp32 [M, N] (all owned by the caller),
+ * K % 8 == 0, 1 <= M <= 4096; grid = persistent CTAs (0 = one per SM).
+ *
+ * Size limit: the scratch needed is the tile counters (4 bytes per 128 x nt
+ * output tile, nt = 16/32/64/128/256 from M) plus 2 * CTAs * nt * 512 bytes of
+ * partials.  M <= 32 always fits; a larger M fits only with a smaller grid.  A
+ * call whose need exceeds the array returns DFLASH_WORKSPACE and launches
+ * nothing.  Other returns: DFLASH_INVALID_ARG (bad sizes, pointers or
+ * alignment), DFLASH_CUDA (the symbol lookup, the counter clear or the launch
+ * failed).
+ *
+ * The first call on each device looks up the array's address with that device
+ * current (this may load the module); make that first call before any stream
+ * capture begins.  Each call clears the counters on `stream` before the launch.
+ * One array serves every caller on a device: calls that may overlap on the same
+ * device (other streams, other host threads) race on it and must be serialised
+ * by the caller. */
+int dflash_diag_gemm_bf16_noalloc(const void* X, const void* W, float* Y, int M, int N, int K, int grid,
+                                  dflash_stream stream);
+
 /* Work partition of the persistent split-K GEMM (host only, no CUDA call).
  * `units` k-blocks in total, `kb` k-blocks per output tile, `ctas` CTAs.  For
  * output tile `tile`: first_cta = first CTA contributing to it, n_contrib = the
