@@ -66,7 +66,7 @@ struct GemmParams {
     // EPI_LMHEAD
     int vocab;
     float* logits;               // [M, vocab] or null
-    float4* records;             // [n_tiles][M]: (top1, id bits, top2, 0)
+    float4* records;             // [M][n_tiles]: (top1, id bits, top2, 0)
     // Diagnostic trace (null in normal use): per CTA 8 globaltimer stamps (ns):
     // entry, producer past the dependency wait, first stage landed, last MMA
     // issued, accumulators drained, epilogue done, exit, clock64 span of the CTA.

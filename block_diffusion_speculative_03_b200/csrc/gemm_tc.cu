@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                             for (int qq = 1; qq < 4; ++qq)
                                 top2_merge(a1, ai, a2, lmred[(qq * CH + e) * 3 + 0],
                                            __float_as_int(lmred[(qq * CH + e) * 3 + 1]), lmred[(qq * CH + e) * 3 + 2]);
-                            p.records[(size_t)n_tile * p.M + mbase + e] = make_float4(a1, __int_as_float(ai), a2, 0.0f);
+                            p.records[(size_t)(mbase + e) * p.n_tiles + n_tile] = make_float4(a1, __int_as_float(ai), a2, 0.0f);
                         }
                         named_bar_sync(1, 128);
                         break;

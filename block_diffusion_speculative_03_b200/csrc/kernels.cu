@@ -102,18 +102,24 @@ DF_DEV void top2m(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
 
 // ---------------------------------------------------------------------------
 // LM-head reduction (bf16 path): merge the per-vocab-tile top-2 records of
-// every draft row.  One warp per row m = b*(gamma-1) + j.
+// every draft row.  One CTA per row m = b*(gamma-1) + j; the row's records are
+// contiguous ([M][n_vt]), so the CTA reads them coalesced in one or two rounds.
 // ---------------------------------------------------------------------------
-__global__ void k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M, int gm1, const int* __restrict__ req_ok,
-                            int* __restrict__ drafts, float* __restrict__ margin) {
+constexpr int kLmReduceThreads = 512;
+
+__global__ void __launch_bounds__(kLmReduceThreads) k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M,
+                                                                 int gm1, const int* __restrict__ req_ok,
+                                                                 int* __restrict__ drafts, float* __restrict__ margin) {
     griddep_wait();
     griddep_launch();
-    const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (m >= M) return;
+    __shared__ float s1[kLmReduceThreads / 32], s2[kLmReduceThreads / 32];
+    __shared__ int si[kLmReduceThreads / 32];
+    const int m = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const float4* row = rec + (size_t)m * n_vt;
     float a1 = -INFINITY, a2 = -INFINITY;
     int ai = 0x7fffffff;
-    for (int t = lane; t < n_vt; t += 32) {
-        const float4 r = rec[(size_t)t * M + m];
+    for (int t = threadIdx.x; t < n_vt; t += kLmReduceThreads) {
+        const float4 r = row[t];
         top2m(a1, ai, a2, r.x, __float_as_int(r.y), r.z);
     }
     for (int off = 16; off > 0; off >>= 1) {
@@ -122,7 +128,10 @@ __global__ void k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M, int
         const float b2 = __shfl_xor_sync(0xffffffffu, a2, off);
         top2m(a1, ai, a2, b1, bi, b2);
     }
-    if (lane == 0) {
+    if (lane == 0) { s1[w] = a1; si[w] = ai; s2[w] = a2; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int k = 1; k < kLmReduceThreads / 32; ++k) top2m(a1, ai, a2, s1[k], si[k], s2[k]);
         const bool ok = req_ok[m / gm1] != 0;
         drafts[m] = ok ? ai : -1;
         if (margin) margin[m] = ok ? a1 - a2 : 0.f;
@@ -450,7 +459,7 @@ template void launch_rmsnorm<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfl
 
 void launch_lm_reduce(const float4* rec, int n_vt, int M, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st) {
-    launch_k(k_lm_reduce, dim3((M * 32 + 255) / 256), dim3(256), 0, st, rec, n_vt, M, gm1, req_ok, drafts, margin);
+    launch_k(k_lm_reduce, dim3(M), dim3(kLmReduceThreads), 0, st, rec, n_vt, M, gm1, req_ok, drafts, margin);
 }
 void launch_top2_rows(const float* logits, int M, int V, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st) {
