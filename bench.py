@@ -64,6 +64,33 @@ def env_int(name, default):
         return default
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of k_gemm_tc per
+# launch, averaged over the 23 GEMM launches of one step of this workload, from
+# one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
+# kernel sources it was taken on; once they change the figure is void.
+GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.5e6,
+                "sources_sha256": "8fea179b970481306e782c9228b9955316bdab6e6edf37b9ecde5021894c2ea9"}
+
+
+def gemm_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "gemm.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_diffusion_speculative_03_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """Per-launch DRAM bytes of the GEMM kernel, or None when not measured for these sources."""
+    try:
+        if workload == GEMM_TRAFFIC["workload"] and gemm_sources_sha256() == GEMM_TRAFFIC["sources_sha256"]:
+            return GEMM_TRAFFIC["bytes_per_launch"]
+    except OSError:
+        pass
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -428,7 +455,7 @@ def run_gpu(args):
         gbytes = sum(kern[n][0] * ab[n] for n in gemm_names if n in kern)
         achieved = gbytes / (gms / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                    "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                    "frac": round(achieved / hbm_peak, 4), "traffic": measured_traffic(args.workload),
                     "kernel": "k_gemm_tc (all %d launches of %d steps)" % (gl, K),
                     "algorithmic_bytes_per_launch": round(gbytes / max(gl, 1)),
                     "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src}
