@@ -301,15 +301,25 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                         float acc[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) acc[i] = 0.0f;
-                        for (int ci = 0; ci < nc; ++ci) {
-                            const int pc = first + ci;
-                            if (pc == cta) {
+                        constexpr int MAXB = CH <= 16 ? 4 : 2;
+                        for (int b0 = 0; b0 < nc; b0 += MAXB) {
+                            float pv[MAXB][CH];
 #pragma unroll
-                                for (int i = 0; i < CH; ++i) acc[i] += v[i];
-                            } else {
-                                const float* src = p.partial + (size_t)sk_slot(pc, t, KB, U, P) * NT * 128;
+                            for (int bi = 0; bi < MAXB; ++bi) {
+                                const int pc = first + b0 + bi;
+                                if (b0 + bi < nc && pc != cta) {
+                                    const float* src = p.partial + (size_t)sk_slot(pc, t, KB, U, P) * NT * 128;
 #pragma unroll
-                                for (int i = 0; i < CH; ++i) acc[i] += __ldcg(src + (c0 + i) * 128 + row);
+                                    for (int i = 0; i < CH; ++i) pv[bi][i] = __ldcg(src + (c0 + i) * 128 + row);
+                                }
+                            }
+#pragma unroll
+                            for (int bi = 0; bi < MAXB; ++bi) {
+                                if (b0 + bi < nc) {
+                                    const bool own = first + b0 + bi == cta;
+#pragma unroll
+                                    for (int i = 0; i < CH; ++i) acc[i] += own ? v[i] : pv[bi][i];
+                                }
                             }
                         }
 #pragma unroll
