@@ -109,7 +109,8 @@ inline int pick_nt(int M) {
 }
 
 // Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
-// ctas) and launches on `stream`.  Returns a cudaError_t.
+// ctas) and launches on `stream`.  Returns a cudaError_t; cudaErrorInvalidValue
+// when units * 160 reaches 2^32 (the kernel's split-tile bookkeeping is 32-bit).
 int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream);
 
 // 2-D bf16 tensor map (abi.cu): `inner` contiguous elements per row, `rows`

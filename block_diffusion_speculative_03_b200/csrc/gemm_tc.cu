@@ -10,6 +10,9 @@
 
 namespace df {
 
+// Largest grid the launcher is given (the C ABI caps it at 160 CTAs).
+constexpr long long kGemmMaxGrid = 160;
+
 // Tile configuration per token width NT: one CTA per SM with the deepest ring
 // that fits (two CTAs per SM with half the ring measured slower at batch 1).
 template <int NT>
@@ -31,6 +34,15 @@ struct GemmCfg {
 };
 
 DF_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// The work partition of gemm.cuh in 32-bit arithmetic, for U * P < 2^32 (the
+// launcher checks): the split-tile bookkeeping sits on the critical path of a
+// GEMM's last tiles, where 64-bit divisions cost.
+DF_DEV uint32_t sk32_begin(uint32_t p, uint32_t U, uint32_t P) { return p * U / P; }
+DF_DEV uint32_t sk32_owner(uint32_t u, uint32_t U, uint32_t P) { return ((u + 1) * P - 1) / U; }
+DF_DEV int sk32_slot(uint32_t p, uint32_t tile, uint32_t KB, uint32_t U, uint32_t P) {
+    return (int)(2 * p + (tile == sk32_begin(p, U, P) / KB ? 0 : 1));
+}
 
 // Top-2 merge: a <- top2(a ∪ b); ties of the top value go to the lower id.
 DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
@@ -232,9 +244,12 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
             bool finish = true;
             int first = cta, nc = 1;
             if (!whole) {
-                first = sk_first_cta(t, KB, U, P);
-                nc = sk_n_contrib(t, KB, U, P);
-                float* dst = p.partial + (size_t)sk_slot(cta, t, KB, U, P) * NT * 128;
+                {
+                    const uint32_t t32 = (uint32_t)t, K32 = (uint32_t)KB, U32 = (uint32_t)U, P32 = (uint32_t)P;
+                    first = (int)sk32_owner(t32 * K32, U32, P32);
+                    nc = (int)sk32_owner((t32 + 1) * K32 - 1, U32, P32) - first + 1;
+                }
+                float* dst = p.partial + (size_t)sk32_slot(cta, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += 16) {
                     float v[16];
@@ -308,7 +323,8 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                             for (int bi = 0; bi < MAXB; ++bi) {
                                 const int pc = first + b0 + bi;
                                 if (b0 + bi < nc && pc != cta) {
-                                    const float* src = p.partial + (size_t)sk_slot(pc, t, KB, U, P) * NT * 128;
+                                    const float* src =
+                                        p.partial + (size_t)sk32_slot(pc, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
 #pragma unroll
                                     for (int i = 0; i < CH; ++i) pv[bi][i] = __ldcg(src + (c0 + i) * 128 + row);
                                 }
@@ -507,6 +523,7 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
         p.n_tiles = nt_total;
     }
     p.units = (long long)p.n_tiles * p.m_tiles * p.KB;
+    if (p.units * (long long)kGemmMaxGrid >= (1LL << 32)) return (int)cudaErrorInvalidValue;   // 32-bit partition arithmetic
     if (p.ctas <= 0 || p.ctas > num_sms) p.ctas = num_sms;
     if ((long long)p.ctas > p.units) p.ctas = (int)p.units;
     if (p.units == 0) return 0;
