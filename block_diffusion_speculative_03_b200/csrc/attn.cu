@@ -28,6 +28,9 @@ namespace cg = cooperative_groups;
 
 namespace df {
 
+// Largest lag (in powers of two) of a row's running integer base behind its maximum.
+constexpr float kAttnBaseLag = 8.0f;
+
 template <int D>
 struct AttnCfg {
     static constexpr int HALVES = D / 64;
@@ -203,33 +206,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         for (int it = 0; it < ntiles; ++it) {
             const int sb = it & 1;
             ok = mbar_wait(&s_full[sb], (uint32_t)((it >> 1) & 1), abort_flag, p.status);
-            if (named_bar_or(1, 128, !ok)) { ok = false; break; }
             tc_fence_after();
             if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
             const int kvb = kv0 + it * 64;
             const uint32_t ts = tS + lanes + sb * 64;
-            // the row's 64 scores, in log2 units, masked past the last key
+            // the row's 64 scores, in log2 units, masked past the last key; the row
+            // maximum over 8 independent partial maxima (exact in any order)
             float t[64];
-#pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) tmem_ld16(ts + c0, t + c0);
+            tmem_ld64(ts, t);
             const int nvalid = kv1 - kvb;
-            float mx = -INFINITY;
+            float m8[8];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                t[i] = (i < nvalid) ? t[i] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, t[i]);
+            for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+            if (nvalid >= 64) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    t[i] *= p.scale_log2;
+                    m8[i & 7] = fmaxf(m8[i & 7], t[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    t[i] = (i < nvalid) ? t[i] * p.scale_log2 : -INFINITY;
+                    m8[i & 7] = fmaxf(m8[i & 7], t[i]);
+                }
             }
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             mt = fmaxf(mt, mx);
             const float nb = floorf(mt);
-            if (it >= 2) {   // the P.V of tile it-2 read this P buffer: wait for it
+            if (ok && it >= 2)   // the P.V of tile it-2 read this P buffer: wait for it
                 ok = mbar_wait(&o_done[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status);
+            // The integer base may lag the running maximum by up to kAttnBaseLag: P is
+            // then at most 2^(kAttnBaseLag + 1), and every P and the row sum are the
+            // oracle's times one exact power of two, so nothing rounds differently; the
+            // O rescale (a wait for the previous P.V plus a TMEM round trip) becomes rare.
+            // One barrier per tile in the common case: it ORs "a wait failed" and "a
+            // row's base moves"; only then a second one tells the two apart.
+            const bool grow = nb > base + kAttnBaseLag;
+            if (named_bar_or(1, 128, !ok || (grow && it >= 1))) {
                 if (named_bar_or(1, 128, !ok)) { ok = false; break; }
-            }
-            // Rescale O and l by 2^(base - nb), an exact power of two, when any row's
-            // integer base grew (the decision is taken by all 128 threads together:
-            // the TMEM accesses are warp-collective; other rows scale by 1).
-            const bool grow = nb > base;
-            if (named_bar_or(1, 128, grow && it >= 1)) {
+                // Rescale O and l by 2^(base - nb), an exact power of two (the TMEM
+                // accesses are warp-collective, so all 128 threads take part; rows
+                // whose base did not grow scale by 1).
                 ok = mbar_wait(&o_done[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), abort_flag, p.status);
                 if (named_bar_or(1, 128, !ok)) { ok = false; break; }
                 tc_fence_after();
@@ -259,21 +278,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             // P = bf16(2^(t - base)) into the swizzled K-major P tile, row `row`.
             uint8_t* prow = sP + sb * C::P_BYTES + row * 128;
             const float bb = (base == -INFINITY) ? 0.f : base;
-            float ls = 0.f;
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums, one per 16 keys
 #pragma unroll
             for (int c0 = 0; c0 < 64; c0 += 16) {
                 uint32_t pk[8];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     const float e0 = ex2_fast(t[c0 + i] - bb), e1 = ex2_fast(t[c0 + i + 1] - bb);
-                    ls += e0 + e1;
+                    ls4[c0 >> 4] += e0 + e1;
                     pk[i / 2] = pack_bf16(e0, e1);
                 }
                 const int ch = c0 >> 3;   // 16-byte chunk of keys c0..c0+7
                 *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
-            l += ls;
+            l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&p_full[sb]);

@@ -21,7 +21,7 @@ struct AttnParams {
     long long* trace;
 };
 
-constexpr int kAttnStages = 3;
+constexpr int kAttnStages = 5;   // K/V ring depth: each stage is held until its tile's P.V is done
 constexpr int kAttnThreads = 192;   // TMA warp, MMA warp, 4 softmax warps
 constexpr int kAttnMaxSplits = 8;   // CTAs per cluster (portable cluster size)
 
