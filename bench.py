@@ -91,6 +91,14 @@ def measured_traffic(workload):
     return None
 
 
+def workload_description(w, B, T, g):
+    family = "LLaMA-3.1-8B-shaped" if w.name.startswith("llama") else "Qwen3-8B-shaped"
+    return ("%s drafter (hidden %d, %d layers, %d/%d heads, d %d, intermediate %d, vocab %d, %s LM head), "
+            "batch %d per GPU, context %d, gamma %d"
+            % (family, w.hidden, w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.intermediate, w.vocab,
+               "tied" if w.tied_lm_head else "separate", B, T, g))
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -515,9 +523,7 @@ def run_gpu(args):
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) target hiddens; benchmark datasets not used)",
-            "config": {"workload": "Qwen3-8B-shaped drafter (hidden 4096, 5 layers, 32/8 heads, d 128, "
-                                   "intermediate 12288, vocab 151936, tied LM head), batch %d per GPU, context %d, "
-                                   "gamma %d" % (B, T, g),
+            "config": {"workload": workload_description(w, B, T, g),
                        "global_batch": world * B, "seq_len": T, "gamma": g, "parallelism": "replicas x%d" % world,
                        "l2": "inputs larger than L2 (%.2f GB of weights streamed per step)" % (step_bytes / 1e9)},
             "drafted_tok_per_s": round(blocks_per_s * (g - 1), 1),
