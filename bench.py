@@ -92,7 +92,8 @@ def measured_traffic(workload):
 
 
 def workload_description(w, B, T, g):
-    family = "LLaMA-3.1-8B-shaped" if w.name.startswith("llama") else "Qwen3-8B-shaped"
+    family = ("LLaMA-3.1-8B-shaped" if w.name.startswith("llama")
+              else "Qwen3-4B-shaped" if w.name.startswith("qwen3_4b") else "Qwen3-8B-shaped")
     return ("%s drafter (hidden %d, %d layers, %d/%d heads, d %d, intermediate %d, vocab %d, %s LM head), "
             "batch %d per GPU, context %d, gamma %d"
             % (family, w.hidden, w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.intermediate, w.vocab,

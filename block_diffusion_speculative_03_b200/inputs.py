@@ -182,6 +182,15 @@ def preset(name: str) -> Workload:
         return Workload("llama31_8b", 4096, 5, 32, 8, 128, 14336, 128256, 5, 4096, 5e5, 1e-5, "bf16",
                         batch=16, gamma=16, context=[8192] * 16, tied_lm_head=False,
                         seed=0xDF1A5 + 4)
+    # The same draft step on a deeper drafter, and on a Qwen3-4B-shaped one
+    # (hidden 2560 with 32 query heads of 128: the attention width exceeds the
+    # hidden size).
+    if name == "qwen3_8b_depth8":
+        return Workload("qwen3_8b_depth8", 4096, 8, 32, 8, 128, 12288, 151936, 5, 4096, 1e6, 1e-6, "bf16",
+                        batch=1, gamma=16, context=[2048], seed=0xDF1A5 + 5)
+    if name == "qwen3_4b":
+        return Workload("qwen3_4b", 2560, 5, 32, 8, 128, 9728, 151936, 5, 2560, 1e6, 1e-6, "bf16",
+                        batch=1, gamma=16, context=[2048], seed=0xDF1A5 + 6)
     # Reduced bf16 shapes that span several GEMM tiles and ragged tails but
     # that the oracle finishes in seconds.
     if name == "small_bf16":
@@ -194,7 +203,8 @@ def preset(name: str) -> Workload:
     raise KeyError(name)
 
 
-PRESETS = ["tiny", "qwen3_8b", "qwen3_8b_b32", "long_ctx", "llama31_8b", "small_bf16", "small_bf16_untied"]
+PRESETS = ["tiny", "qwen3_8b", "qwen3_8b_b32", "long_ctx", "llama31_8b", "qwen3_8b_depth8", "qwen3_4b",
+           "small_bf16", "small_bf16_untied"]
 
 
 # Tensor ids of the generator streams.

@@ -160,3 +160,13 @@ def test_long_context_gamma_sweep():
 
 def test_llama31_8b_batch16():
     assert _run("llama31_8b", sample=[5], cycles=1) > 0
+
+
+def test_depth8_drafter():
+    # the same kernels on an 8-layer drafter (a deeper drafter than the 5-layer default)
+    assert _run("qwen3_8b_depth8", sample=[0], cycles=2) > 0
+
+
+def test_qwen3_4b_shaped_drafter():
+    # hidden 2560 with 32 x 128 query width: the O-proj reduces over 4096 into 2560
+    assert _run("qwen3_4b", sample=[0], cycles=2) > 0
