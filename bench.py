@@ -34,6 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 HBM_FALLBACK_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
 BF16_FALLBACK_TFLOPS = 1590.0
 
 # NVML clock-event reason bits
@@ -93,11 +94,22 @@ def measured_traffic(workload):
 
 def workload_description(w, B, T, g):
     family = ("LLaMA-3.1-8B-shaped" if w.name.startswith("llama")
-              else "Qwen3-4B-shaped" if w.name.startswith("qwen3_4b") else "Qwen3-8B-shaped")
+              else "Qwen3-4B-shaped" if w.name.startswith("qwen3_4b")
+              else "Qwen3-8B-shaped" if w.name.startswith(("qwen3_8b", "long_ctx"))
+              else "%s (%s, parity-size)" % (w.name, w.dtype))
     return ("%s drafter (hidden %d, %d layers, %d/%d heads, d %d, intermediate %d, vocab %d, %s LM head), "
             "batch %d per GPU, context %d, gamma %d"
             % (family, w.hidden, w.n_layers, w.n_q_heads, w.n_kv_heads, w.head_dim, w.intermediate, w.vocab,
                "tied" if w.tied_lm_head else "separate", B, T, g))
+
+
+def config_of(w, world, B, T, g, step_bytes):
+    """The config object of a bench line (the GPU arm and the reference arm report the same)."""
+    return {"workload": workload_description(w, B, T, g), "global_batch": world * B, "seq_len": T, "gamma": g,
+            "parallelism": "replicas x%d" % world,
+            "l2": ("inputs larger than L2 (%.2f GB of weights streamed per step)" % (step_bytes / 1e9)
+                   if step_bytes > L2_BYTES else "inputs fit in L2 (%.1f MB per step; a parity-size workload, "
+                   "not flushed)" % (step_bytes / 1e6))}
 
 
 def measured_peaks():
@@ -242,6 +254,7 @@ def run_reference(args):
     import torch
     from block_diffusion_speculative_03_b200 import inputs as I
     from oracle import oracle as O
+    w_full = I.preset(args.workload)
     w = I.preset(args.workload)
     w.batch = 1
     w.context = w.context[:1]
@@ -266,8 +279,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": n, "warmup": min(args.warmup, 1), "ms_per_step": 1e3 * dt / n,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "drafted_tok_per_s": bps * (w.gamma - 1),
-        "config": {"workload": "%s: batch 1, context %d, gamma %d (per request; the oracle runs one request)"
-                   % (w.name, w.context[0], w.gamma)},
+        "config": config_of(w_full, args.gpus, w_full.batch, w_full.context[0], w_full.gamma,
+                            step_algorithmic_bytes(w_full, w_full.batch, w_full.gamma, w_full.context[0])),
         "cpu_baseline": {"value": bps, "unit": "blocks/s", "cores": O.num_threads(), "kind": "oracle",
                          "sample": "%d full oracle cycles (draft block + fuse/inject of %d rows + accept) of one "
                                    "request (of %d requested steps; capped at ~90 s)" % (n, w.gamma, args.steps)},
@@ -524,9 +537,7 @@ def run_gpu(args):
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) target hiddens; benchmark datasets not used)",
-            "config": {"workload": workload_description(w, B, T, g),
-                       "global_batch": world * B, "seq_len": T, "gamma": g, "parallelism": "replicas x%d" % world,
-                       "l2": "inputs larger than L2 (%.2f GB of weights streamed per step)" % (step_bytes / 1e9)},
+            "config": config_of(w, world, B, T, g, step_bytes),
             "drafted_tok_per_s": round(blocks_per_s * (g - 1), 1),
             "roofline": roofline,
             "step_roofline": {"algorithmic_bytes": step_bytes, "flops": step_flops(w, B, g, T),

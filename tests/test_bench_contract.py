@@ -1,0 +1,34 @@
+"""The benchmark's output contract, checked on CPU through its reference arm
+(the CPU oracle) on the tiny workload: one JSON line with the fields a driver
+reads, and the same config description the GPU arm prints for that workload."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == "draft_blocks_per_s" and d["unit"] == "blocks/s"
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["steps"] >= 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_diffusion_speculative_03_b200 import inputs as I
+    w = I.preset("tiny")
+    assert d["config"] == bench.config_of(w, 1, w.batch, w.context[0], w.gamma,
+                                          bench.step_algorithmic_bytes(w, w.batch, w.gamma, w.context[0]))
