@@ -112,6 +112,17 @@ def config_of(w, world, B, T, g, step_bytes):
                    "not flushed)" % (step_bytes / 1e6))}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -198,13 +209,14 @@ class OracleCycle:
     shapes: draft_block over a context of the workload's length + fuse/inject of
     gamma verified rows + accept, then the same length reset as the GPU step."""
 
-    def __init__(self, w, weights_np):
+    def __init__(self, w, weights_np, acc32=0):
         from oracle import oracle as O
         from block_diffusion_speculative_03_b200 import inputs as I
         shape = dict(hidden=w.hidden, n_layers=w.n_layers, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                      head_dim=w.head_dim, intermediate=w.intermediate, vocab=w.vocab, n_sel=w.n_sel,
                      target_hidden=w.target_hidden, mask_id=w.mask_token,
-                     storage="f32" if w.dtype == "f32" else "bf16", rope_theta=w.rope_theta, rms_eps=w.rms_eps)
+                     storage="f32" if w.dtype == "f32" else "bf16", rope_theta=w.rope_theta, rms_eps=w.rms_eps,
+                     acc32=acc32)
         self.w = w
         self.od = O.OracleDrafter(shape, weights_np)
         T = w.context[0]
@@ -356,14 +368,32 @@ def run_gpu(args):
                       max_position=cap, max_gamma=g, device=dev)
     cache = drafter.new_cache(B, cap)
     st = torch.cuda.current_stream()
-    # prefill through the library: fuse + inject of B*T seeded target-hidden rows
+    # prefill through the library: fuse + inject of B*T seeded target-hidden rows,
+    # once to fill the cache and twice more timed (prefill ingestion, reported apart)
     hid = I.make_hiddens(w, B * T, stream=0, device=dev)
-    ctx = drafter.fuse_context(hid)
-    drafter.inject_kv(cache, ctx, torch.arange(0, B * T, T, dtype=torch.int32, device=dev),
-                      torch.full((B,), T, dtype=torch.int32, device=dev))
     lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    starts = torch.arange(0, B * T, T, dtype=torch.int32, device=dev)
+    pre_ms = []
+    for rep in range(3):
+        cache.set_len(zeros)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        ctx = drafter.fuse_context(hid)
+        drafter.inject_kv(cache, ctx, starts, lens)
+        p1.record()
+        torch.cuda.synchronize()
+        if rep:
+            pre_ms.append(p0.elapsed_time(p1))
+        del ctx
     cache.set_len(lens)
-    del hid, ctx
+    del hid
+    pre_t = statistics.median(pre_ms)
+    pre_flops = 2.0 * B * T * w.hidden * (w.n_sel * w.target_hidden + w.n_layers * 2 * w.n_kv_heads * w.head_dim)
+    prefill = {"rows": B * T, "ms": round(pre_t, 3), "rows_per_s": round(B * T / (pre_t / 1e3), 1),
+               "tflops": round(pre_flops / (pre_t / 1e3) / 1e12, 1),
+               "what": "fuse_context + inject_kv of the whole context (all requests), median of 2, "
+                       "allocation of the context buffer included"}
     # per-step inputs resident in HBM (a pool of distinct verified-row sets)
     POOL = 32
     step_hid = [I.make_hiddens(w, B * g, stream=1000 + i, device=dev) for i in range(POOL)]
@@ -515,21 +545,33 @@ def run_gpu(args):
     assert cache.status() == 0
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
-    cpu = None
+    cpu = cpu32 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # The oracle runs its requests one after another, so its blocks/s is its
+        # cycle rate on one request, whatever the batch.
         from oracle import oracle as O
         wc = I.preset(args.workload)
         wc.batch, wc.context = 1, wc.context[:1]
-        oc = OracleCycle(wc, oracle_weights_from(weights))
-        oc.cycle()                          # warm (first-touch of the host arrays)
-        n, t0 = 0, time.perf_counter()
-        while n < 8 and (n < 2 or time.perf_counter() - t0 < 12.0):
-            oc.cycle()
-            n += 1
-        dt = time.perf_counter() - t0
-        cpu = {"value": n / dt * B, "unit": "blocks/s", "cores": O.num_threads(), "kind": "oracle",
-               "sample": "%d oracle cycles of one request (draft block + fuse/inject of %d rows + accept), "
-                         "scaled to batch %d" % (n, g, B)}
+        host_w = oracle_weights_from(weights)
+
+        def time_cycles(acc32, max_n, max_s):
+            oc = OracleCycle(wc, host_w, acc32=acc32)
+            oc.cycle()                          # warm (first-touch of the host arrays)
+            n, t0 = 0, time.perf_counter()
+            while n < max_n and (n < 2 or time.perf_counter() - t0 < max_s):
+                oc.cycle()
+                n += 1
+            return n, time.perf_counter() - t0
+
+        n, dt = time_cycles(0, 8, 12.0)
+        cpu = {"value": n / dt, "unit": "blocks/s", "cores": O.num_threads(), "kind": "oracle",
+               "cpu_model": cpu_model(),
+               "sample": "%d oracle cycles (fp64 accumulation, the parity mode) of one request: draft block + "
+                         "fuse/inject of %d rows + accept" % (n, g)}
+        n, dt = time_cycles(1, 8, 8.0)
+        cpu32 = {"value": n / dt, "unit": "blocks/s", "cores": O.num_threads(), "kind": "oracle",
+                 "sample": "%d oracle cycles with fp32 accumulation (the oracle's sensitivity mode), "
+                           "one request" % n}
 
     if rank == 0:
         line = {
@@ -545,6 +587,8 @@ def run_gpu(args):
                               "peak_gbs": hbm_peak, "peak_source": peak_src},
             "per_kernel": per_kernel,
             "cpu_baseline": cpu,
+            "cpu_baseline_fp32_accumulation": cpu32,
+            "prefill": prefill,
             "e2e": e2e,
             "gpu_launches": launches,
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
