@@ -37,7 +37,11 @@
  *            v = R(h Wv^T); o = R(softmax(q K^T / sqrt(d)) V) over all cached
  *            rows [0, len) and all gamma block rows (no mask; query head hq
  *            reads kv head hq / (n_q_heads / n_kv_heads); P is rounded to bf16
- *            before it weights V); x = R(x + o Wo^T); h2 = R(RMSNorm(x) g_post);
+ *            before it weights V: with t_i = q.k_i log2(e) / sqrt(d),
+ *            P_i = R(2^(t_i - b)) for an integer b, divided by the sum of the
+ *            unrounded 2^(t_i - b); every integer b below the row maximum gives
+ *            the same o, as the values differ by one exact power of two);
+ *            x = R(x + o Wo^T); h2 = R(RMSNorm(x) g_post);
  *            m = R(silu(h2 Wg^T) * (h2 Wu^T)); x = R(x + m Wd^T).
  *            Then hf_j = R(RMSNorm(x_j) g_final) for j = 1..gamma-1, logits =
  *            hf_j . lm_head^T (fp32), draft_j = argmax (ties to the lowest id).
