@@ -29,6 +29,16 @@
 // storage is bf16 and the identity when storage is fp32.  Every accumulation is
 // fp64.  No blocking, fusion or reordering is done beyond what the definitions
 // state: plain loops, parallelised over independent outputs only.
+//
+// Pins (the test suite's CPU tests): R() against torch's bf16 cast and brute
+// force; RMSNorm, RoPE and attention against library routines, closed forms
+// and invariants; accept exhaustively against a brute-force scan; the loss
+// weights against their closed form; fuse, inject and draft through invariants
+// (concat order, chunked = one-shot injection, one bidirectional pass, zero
+// layers = norm + shared head).  The composition of oracle_fuse_context,
+// oracle_inject_kv and oracle_draft_block as a DFlash drafter (norm placement,
+// positions, mask id) follows the reading above and cannot be checked against
+// a trained DFlash model here: parity unpinned against the paper's model.
 
 #include <cmath>
 #include <cstdint>
