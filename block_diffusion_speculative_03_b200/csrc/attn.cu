@@ -12,10 +12,17 @@
 //            buffers (M = 128 padded query rows, N = 64 keys), and
 //            O += P_i V_i into the TMEM accumulator (N = head_dim, V read as
 //            an MN-major operand straight from the TMA tile).
-//   warps 2-5  softmax, one query row per thread: reads S_i from TMEM, keeps a
-//            base-2 running maximum with an integer base B, writes
-//            P_i = bf16(2^(t - B)) into shared memory for the P.V MMA, and
-//            rescales O in TMEM by an exact power of two when B grows.
+//   warps 2-5  softmax: reads S_i from TMEM, keeps a base-2 running maximum
+//            with an integer base B per row, writes P_i = bf16(2^(t - B)) into
+//            shared memory for the P.V MMA, and rescales O in TMEM by an exact
+//            power of two when B grows.
+//
+// The R <= 64 query rows fill CS = 2 (R > 32) or 4 copies of a window of
+// 128/CS rows of the M = 128 tile, so S holds every row CS times; the CS
+// threads that own a row's copies take 64/CS of each tile's keys each (a
+// thread reads only its own TMEM lane).  They agree on the row's base through
+// shared memory whenever one of them would move it, and add their partial
+// row sums at the end.  O accumulates in the first window's lanes.
 //
 // Each CTA leaves its partial (B, l, O) in its own shared memory; after a
 // cluster barrier every CTA merges a slice of the rows by reading all partials
@@ -38,14 +45,16 @@ struct AttnCfg {
     static constexpr int KV_BYTES = HALVES * 64 * 128;       // 64 keys x D
     static constexpr int P_BYTES = 128 * 128;                // 128 rows x 64 keys
     static constexpr int RING = Q_BYTES + 2 * kAttnStages * KV_BYTES + 2 * P_BYTES;
-    static constexpr int SMEM = 1024 + RING + 256;
+    static constexpr int SMEM = 1024 + RING + 256 + 512;     // + barriers, + row exchange [128]
     static constexpr uint32_t TMEM_COLS = 256;               // S[2] (2 x 64) + O (D)
 };
 
-template <int D>
+template <int D, int CS>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_constant__ AttnParams p) {
     using C = AttnCfg<D>;
     constexpr int S = kAttnStages;
+    constexpr int RW = 128 / CS;   // rows per window of the M = 128 tile
+    constexpr int KC = 64 / CS;    // keys of a tile per softmax thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sQ = smem;
@@ -62,6 +71,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     uint64_t* drain = o_done + 2;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    float* xch = (float*)(smem + C::RING + 256);   // [128] per TMEM lane: running max, then row sum
     // After the key loop the front of shared memory holds this CTA's partial.
     float* po = (float*)smem;                      // [64][D]
     float2* pml = (float2*)(po + 64 * D);          // [64] (integer base, row sum)
@@ -118,11 +128,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // Query rows R..127 of the padded M = 128 tile are zero.
-    for (int idx = tid; idx < (128 - R) * C::HALVES * 8; idx += kAttnThreads) {
-        const int r = R + idx / (C::HALVES * 8), rem = idx % (C::HALVES * 8);
-        const int h = rem / 8, c16 = rem % 8;
-        *reinterpret_cast<uint4*>(sQ + h * 16384 + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+    // Rows R..RW-1 of every window of the Q tile, and P rows RW..127 (never
+    // written, so O's lanes RW..127 stay zero), are zero.
+    {
+        const int per = (RW - R) * C::HALVES * 8;
+        for (int idx = tid; idx < CS * per; idx += kAttnThreads) {
+            const int k = idx / per, rem0 = idx % per;
+            const int r = k * RW + R + rem0 / (C::HALVES * 8), rem = rem0 % (C::HALVES * 8);
+            const int h = rem / 8, c16 = rem % 8;
+            *reinterpret_cast<uint4*>(sQ + h * 16384 + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+        }
+        for (int idx = tid; idx < 2 * (128 - RW) * 8; idx += kAttnThreads) {
+            const int pb = idx / ((128 - RW) * 8), rem = idx % ((128 - RW) * 8);
+            *reinterpret_cast<uint4*>(sP + pb * C::P_BYTES + (RW + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
     }
     fence_proxy_async();
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -135,9 +155,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, (uint32_t)(R * D * 2));
-            for (int h = 0; h < C::HALVES; ++h)
-                tma_load_3d(sQ + h * 16384, &p.tq, q_full, h * 64, g * p.G, b * p.gamma);
+            mbar_arrive_expect_tx(q_full, (uint32_t)(CS * R * D * 2));
+            for (int k = 0; k < CS; ++k)   // one copy of the R rows per window
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sQ + h * 16384 + k * RW * 128, &p.tq, q_full, h * 64, g * p.G, b * p.gamma);
             for (int it = 0; it < ntiles; ++it) {
                 const int st = it % S;
                 if (!mbar_wait(&kv_empty[st], (uint32_t)(((it / S) & 1) ^ 1), abort_flag, p.status)) break;
@@ -196,9 +217,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax (one query row per thread)
+        // ------------------------------------------------------------ softmax (KC keys of a row per thread)
         const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;
+        const int rl = q4 * 32 + lane;                 // this thread's TMEM lane
+        const int row = rl % RW, cs = rl / RW;         // query row, key slice (warp-uniform)
         const int e = tid - 64;                        // 0..127
         const uint32_t lanes = (uint32_t)(q4 * 32) << 16;
         float base = -INFINITY, mt = -INFINITY, l = 0.f;
@@ -208,66 +230,75 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             ok = mbar_wait(&s_full[sb], (uint32_t)((it >> 1) & 1), abort_flag, p.status);
             tc_fence_after();
             if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
-            const int kvb = kv0 + it * 64;
-            const uint32_t ts = tS + lanes + sb * 64;
-            // the row's 64 scores, in log2 units, masked past the last key; the row
-            // maximum over 8 independent partial maxima (exact in any order)
-            float t[64];
-            tmem_ld64(ts, t);
+            const int kvb = kv0 + it * 64 + cs * KC;   // first key of this thread's slice
+            const uint32_t ts = tS + lanes + sb * 64 + cs * KC;
+            // the slice's scores, in log2 units, masked past the last key; its maximum
+            // over 8 independent partial maxima (exact in any order)
+            float t[KC];
+            if constexpr (KC == 32) tmem_ld32w(ts, t); else tmem_ld16w(ts, t);
             const int nvalid = kv1 - kvb;
             float m8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-            if (nvalid >= 64) {
+            if (nvalid >= KC) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
+                for (int i = 0; i < KC; ++i) {
                     t[i] *= p.scale_log2;
                     m8[i & 7] = fmaxf(m8[i & 7], t[i]);
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
+                for (int i = 0; i < KC; ++i) {
                     t[i] = (i < nvalid) ? t[i] * p.scale_log2 : -INFINITY;
                     m8[i & 7] = fmaxf(m8[i & 7], t[i]);
                 }
             }
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mt = fmaxf(mt, mx);
-            const float nb = floorf(mt);
+            mt = fmaxf(mt, mx);   // running maximum of this slice
             if (ok && it >= 2)   // the P.V of tile it-2 read this P buffer: wait for it
                 ok = mbar_wait(&o_done[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status);
             // The integer base may lag the running maximum by up to kAttnBaseLag: P is
             // then at most 2^(kAttnBaseLag + 1), and every P and the row sum are the
             // oracle's times one exact power of two, so nothing rounds differently; the
             // O rescale (a wait for the previous P.V plus a TMEM round trip) becomes rare.
-            // One barrier per tile in the common case: it ORs "a wait failed" and "a
-            // row's base moves"; only then a second one tells the two apart.
-            const bool grow = nb > base + kAttnBaseLag;
-            if (named_bar_or(1, 128, !ok || (grow && it >= 1))) {
+            // A row's base moves only if one of its slices' maxima passes base + lag, so
+            // one barrier per tile ORs "a wait failed" and "a slice would move its base";
+            // only then do the slices exchange maxima (and the first tile always does).
+            const bool growl = floorf(mt) > base + kAttnBaseLag;
+            if (named_bar_or(1, 128, !ok || growl)) {
                 if (named_bar_or(1, 128, !ok)) { ok = false; break; }
-                // Rescale O and l by 2^(base - nb), an exact power of two (the TMEM
-                // accesses are warp-collective, so all 128 threads take part; rows
-                // whose base did not grow scale by 1).
-                ok = mbar_wait(&o_done[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), abort_flag, p.status);
-                if (named_bar_or(1, 128, !ok)) { ok = false; break; }
-                tc_fence_after();
-                const float f = grow ? exp2f(base - nb) : 1.0f;
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tO + lanes + c0, v);
+                xch[rl] = mt;
+                named_bar_sync(1, 128);
+                float mrow = mt;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] *= f;
-                    tmem_st16(tO + lanes + c0, v);
+                for (int k = 1; k < CS; ++k) mrow = fmaxf(mrow, xch[(rl + k * RW) & 127]);
+                const float nb = floorf(mrow);
+                const bool grow = nb > base + kAttnBaseLag;
+                if (it >= 1) {
+                    // Rescale O and l by 2^(base - nb), an exact power of two (the TMEM
+                    // accesses are warp-collective, so all 128 threads take part; rows
+                    // whose base did not grow scale by 1).
+                    ok = mbar_wait(&o_done[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), abort_flag, p.status);
+                    if (named_bar_or(1, 128, !ok)) { ok = false; break; }
+                    tc_fence_after();
+                    const float f = grow ? exp2f(base - nb) : 1.0f;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tO + lanes + c0, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] *= f;
+                        tmem_st16(tO + lanes + c0, v);
+                    }
+                    tmem_wait_st();
+                    l *= f;
                 }
-                tmem_wait_st();
-                l *= f;
+                if (grow) base = nb;
             }
-            if (grow) base = nb;
             // The last tile of a split may extend past the last key: zero those V
             // rows (P is 0 there, but 0 * NaN from never-written cache slack is NaN).
-            const int valid = kv1 - kvb;
+            const int valid = kv1 - (kv0 + it * 64);
             if (valid < 64) {
                 uint8_t* vs = sV + (it % S) * C::KV_BYTES;
                 for (int idx = e; idx < (64 - valid) * C::HALVES * 8; idx += 128) {
@@ -275,24 +306,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                     *reinterpret_cast<uint4*>(vs + (rem / 8) * 8192 + r * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            // P = bf16(2^(t - base)) into the swizzled K-major P tile, row `row`.
+            // P = bf16(2^(t - base)) into the swizzled K-major P tile: row `row`,
+            // keys cs*KC .. cs*KC+KC-1.
             uint8_t* prow = sP + sb * C::P_BYTES + row * 128;
             const float bb = (base == -INFINITY) ? 0.f : base;
-            float ls4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums, one per 16 keys
+            float ls[KC / 16];   // independent partial sums, one per 16 keys
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
+            for (int c0 = 0; c0 < KC; c0 += 16) {
                 uint32_t pk[8];
+                float s2 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     const float e0 = ex2_fast(t[c0 + i] - bb), e1 = ex2_fast(t[c0 + i + 1] - bb);
-                    ls4[c0 >> 4] += e0 + e1;
+                    s2 += e0 + e1;
                     pk[i / 2] = pack_bf16(e0, e1);
                 }
-                const int ch = c0 >> 3;   // 16-byte chunk of keys c0..c0+7
+                ls[c0 >> 4] = s2;
+                const int ch = (cs * KC + c0) >> 3;   // 16-byte chunk of 8 keys
                 *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
-            l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+            if constexpr (KC == 32) l += ls[0] + ls[1]; else l += ls[0];
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&p_full[sb]);
@@ -304,7 +338,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             tc_fence_after();
         }
         if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
+        xch[rl] = l;              // the slices' partial row sums (same base)
         named_bar_sync(1, 128);   // every softmax thread is past its P writes before the front is reused
+        float lrow = l;
+#pragma unroll
+        for (int k = 1; k < CS; ++k) lrow += xch[(rl + k * RW) & 127];
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
             float v[16];
@@ -314,12 +352,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = 0.f;
             }
-            if (row < 64) {
+            if (cs == 0) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) po[row * D + c0 + i] = v[i];
             }
         }
-        if (row < 64) pml[row] = make_float2(base, ok ? l : 0.f);
+        if (cs == 0) pml[row] = make_float2(base, ok ? lrow : 0.f);
     }
     tc_fence_before();
     __syncthreads();
@@ -395,7 +433,8 @@ int attn_max_cluster(int d) {
     static int cached[2] = {0, 0};
     int& c = cached[d == 128 ? 1 : 0];
     if (c) return c;
-    void (*kern)(AttnParams) = (d == 128) ? k_attn_tc<128> : k_attn_tc<64>;
+    // both row-copy variants use the same resources
+    void (*kern)(AttnParams) = (d == 128) ? k_attn_tc<128, 2> : k_attn_tc<64, 2>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(d));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kAttnMaxSplits, 1, 1);
@@ -420,9 +459,12 @@ void attn_plan(int B, int nkv, int cap, int num_sms, int max_cluster, int& split
 
 int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, long long* launches) {
     const int smem = attn_smem_bytes(d);
-    void (*kern)(AttnParams) = (d == 128) ? k_attn_tc<128> : k_attn_tc<64>;
-    static bool done128 = false, done64 = false;
-    bool& done = (d == 128) ? done128 : done64;
+    // Row copies: 4 when the R = G * gamma query rows fit 32 lanes, else 2 (R <= 64).
+    const bool four = p.G * p.gamma <= 32;
+    void (*kern)(AttnParams) = (d == 128) ? (four ? k_attn_tc<128, 4> : k_attn_tc<128, 2>)
+                                          : (four ? k_attn_tc<64, 4> : k_attn_tc<64, 2>);
+    static bool done_v[2][2] = {{false, false}, {false, false}};
+    bool& done = done_v[d == 128 ? 1 : 0][four ? 1 : 0];
     if (!done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return (int)e;

@@ -1,7 +1,9 @@
 """The block-attention kernel alone against the oracle's attention, on seeded
-q / K / V, for context lengths that give one to many K/V tiles per split and
+q / K / V, for context lengths that give one to many K/V tiles per split,
 every split count the planner picks (cluster merge through distributed
-shared memory)."""
+shared memory), and query-row counts G * gamma on both sides of 32 (four or
+two copies of the rows in the tile, each row's keys split over as many
+threads), padded windows included."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +18,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("lens,gamma,nq,nkv,d", [([2048], 16, 32, 8, 128), ([100, 3000], 16, 8, 2, 128),
                                                  ([5000, 17, 700], 8, 6, 3, 64), ([64], 4, 8, 2, 128),
-                                                 ([32768], 16, 32, 8, 128)])
+                                                 ([32768], 16, 32, 8, 128), ([4000], 8, 32, 8, 128),
+                                                 ([1500, 250], 11, 12, 4, 128)])
 def test_attention_kernel_matches_oracle(lens, gamma, nq, nkv, d):
     B = len(lens)
     w = I.Workload("attn", 512, 1, nq, nkv, d, 1024, 1024, 1, 512, 1e6, 1e-6, "bf16", batch=B, gamma=gamma,
