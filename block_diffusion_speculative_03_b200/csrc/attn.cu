@@ -8,10 +8,11 @@
 //
 //   warp 0   TMA: the Q tile once (a 3-D box gathers the G heads of every block
 //            position), then K/V tiles of 64 keys into a 3-stage ring.
-//   warp 1   tcgen05.mma (one thread): S_i = Q K_i^T into one of two TMEM
-//            buffers (M = 128 padded query rows, N = 64 keys), and
-//            O += P_i V_i into the TMEM accumulator (N = head_dim, V read as
-//            an MN-major operand straight from the TMA tile).
+//   warp 1   tcgen05.mma (one thread): S_i = Q K_i^T into one of three TMEM
+//            buffers (M = 128 rows, N = 64 keys), issued up to three tiles
+//            ahead of the softmax, and O += P_i V_i into the TMEM accumulator
+//            (N = head_dim, V read as an MN-major operand straight from the
+//            TMA tile) once the softmax has written P_i.
 //   warps 2-5  softmax: reads S_i from TMEM, keeps a base-2 running maximum
 //            with an integer base B per row, writes P_i = bf16(2^(t - B)) into
 //            shared memory for the P.V MMA, and rescales O in TMEM by an exact
@@ -46,7 +47,8 @@ struct AttnCfg {
     static constexpr int P_BYTES = 128 * 128;                // 128 rows x 64 keys
     static constexpr int RING = Q_BYTES + 2 * kAttnStages * KV_BYTES + 2 * P_BYTES;
     static constexpr int SMEM = 1024 + RING + 256 + 512;     // + barriers, + row exchange [128]
-    static constexpr uint32_t TMEM_COLS = 256;               // S[2] (2 x 64) + O (D)
+    static constexpr int NS = 3;                             // S buffers in TMEM
+    static constexpr uint32_t TMEM_COLS = 512;               // S[NS] (NS x 64) at 0, O (D) at 256
 };
 
 template <int D, int CS>
@@ -65,8 +67,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     uint64_t* q_full = bars;
     uint64_t* kv_full = q_full + 1;                // [S]
     uint64_t* kv_empty = kv_full + S;              // [S]
-    uint64_t* s_full = kv_empty + S;               // [2]
-    uint64_t* p_full = s_full + 2;                 // [2]
+    uint64_t* s_full = kv_empty + S;               // [NS]
+    uint64_t* p_full = s_full + C::NS;             // [2]
     uint64_t* o_done = p_full + 2;                 // [2]
     uint64_t* drain = o_done + 2;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
@@ -119,8 +121,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
         }
+        for (int i = 0; i < C::NS; ++i) mbar_init(&s_full[i], 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
             mbar_init(&o_done[i], 1);
         }
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
+    const uint32_t tS = tmem, tO = tmem + 256;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -178,37 +180,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
             bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
             if (trace) trace[2] = (long long)globaltimer_ns();
-            for (int it = 0; it <= ntiles && ok; ++it) {
-                if (it < ntiles) {
-                    // S_it = Q K_it^T into S buffer it & 1 (free once the softmax read S_{it-2})
-                    const int st = it % S, sb = it & 1;
-                    if (!mbar_wait(&kv_full[st], (uint32_t)((it / S) & 1), abort_flag, p.status)) { ok = false; break; }
-                    if (it >= 2 && !mbar_wait(&p_full[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + st * C::KV_BYTES);
+            const uint32_t qa = smem_u32(sQ);
+            // S_j = Q K_j^T into S buffer j % NS (free: the softmax has read S_{j-NS}).
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % S;
+                if (!mbar_wait(&kv_full[st], (uint32_t)((j / S) & 1), abort_flag, p.status)) return false;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(sK + st * C::KV_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        tc_mma_bf16(tS + sb * 64, umma_desc_sw128(qa + (kk >> 2) * 16384) + 2 * (kk & 3),
-                                    umma_desc_sw128(ka + (kk >> 2) * 8192) + 2 * (kk & 3), IDESC_S, kk > 0 ? 1u : 0u);
-                    tc_commit(&s_full[sb]);
-                }
-                if (it >= 1) {
-                    // O += P_j V_j for the previous tile, once its P is written
-                    const int j = it - 1, pb = j & 1;
-                    if (!mbar_wait(&p_full[pb], (uint32_t)((j >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t pa = smem_u32(sP + pb * C::P_BYTES);
-                    const uint32_t va = smem_u32(sV + (j % S) * C::KV_BYTES);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc_mma_bf16(tS + (j % C::NS) * 64, umma_desc_sw128(qa + (kk >> 2) * 16384) + 2 * (kk & 3),
+                                umma_desc_sw128(ka + (kk >> 2) * 8192) + 2 * (kk & 3), IDESC_S, kk > 0 ? 1u : 0u);
+                tc_commit(&s_full[j % C::NS]);
+                return true;
+            };
+            for (int j = 0; j < C::NS && j < ntiles && ok; ++j) ok = issue_s(j);
+            for (int it = 0; it < ntiles && ok; ++it) {
+                // O += P_it V_it once the softmax has written P_it (and so read S_it)
+                const int pb = it & 1;
+                if (!mbar_wait(&p_full[pb], (uint32_t)((it >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sP + pb * C::P_BYTES);
+                const uint32_t va = smem_u32(sV + (it % S) * C::KV_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_bf16(tO, umma_desc_sw128(pa) + 2 * kk, umma_desc_sw128_mn(va + kk * 2048, 8192, 1024),
-                                    IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&o_done[pb]);
-                    tc_commit(&kv_empty[j % S]);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_bf16(tO, umma_desc_sw128(pa) + 2 * kk, umma_desc_sw128_mn(va + kk * 2048, 8192, 1024),
+                                IDESC_PV, (it > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&o_done[pb]);
+                tc_commit(&kv_empty[it % S]);
+                if (it + C::NS < ntiles) ok = issue_s(it + C::NS);
             }
             if (*abort_flag) {
                 tc_commit(drain);   // let the issued MMAs finish before TMEM is released
@@ -226,12 +226,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         float base = -INFINITY, mt = -INFINITY, l = 0.f;
         bool ok = true;
         for (int it = 0; it < ntiles; ++it) {
-            const int sb = it & 1;
-            ok = mbar_wait(&s_full[sb], (uint32_t)((it >> 1) & 1), abort_flag, p.status);
+            const int sb = it & 1;           // P buffer
+            const int sbuf = it % C::NS;     // S buffer
+            ok = mbar_wait(&s_full[sbuf], (uint32_t)((it / C::NS) & 1), abort_flag, p.status);
             tc_fence_after();
             if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
             const int kvb = kv0 + it * 64 + cs * KC;   // first key of this thread's slice
-            const uint32_t ts = tS + lanes + sb * 64 + cs * KC;
+            const uint32_t ts = tS + lanes + sbuf * 64 + cs * KC;
             // the slice's scores, in log2 units, masked past the last key; its maximum
             // over 8 independent partial maxima (exact in any order)
             float t[KC];
