@@ -69,8 +69,8 @@ def env_int(name, default):
 # launch, averaged over the 23 GEMM launches of one step of this workload, from
 # one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
 # kernel sources it was taken on; once they change the figure is void.
-GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.5e6,
-                "sources_sha256": "41c73d5a622281ad35a86e6852745de6f13dfe5ce7dd4f4f9d07d70cb61dbbb5"}
+GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.6e6,
+                "sources_sha256": "5c4b7b9aa3ddbb6dcf12f1b4e71973eea6395cbf3e52ec4be4086c7718434762"}
 
 
 def gemm_sources_sha256():

@@ -240,20 +240,6 @@ int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st) {
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
 }
 
-// q of the block as a 3-D bf16 map [positions][heads][d] with box {64, G, gamma}:
-// one box gathers the G query heads of kv head g for every block position.
-bool encode_q_map(CUtensorMap* m, const void* q, int positions, int nq, int d, int G, int gamma) {
-    PFN_encodeTiled_t enc = get_encode();
-    if (!enc || ((uintptr_t)q & 15)) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nq, (cuuint64_t)positions};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)nq * d * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)gamma};
-    cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Activation operand map: rows x K bf16 with row stride `stride`, box rows nt.
 bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride, int nt) {
     return encode_bf16_2d(m, base, (uint64_t)K, (uint64_t)rows, (uint64_t)stride, (uint32_t)nt);
@@ -617,7 +603,6 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
     AttnParams ap;
     std::memset(&ap, 0, sizeof(ap));
     ap.tmap = cc->tm_slab;
-    if (!encode_q_map(&ap.tq, h->q, M, c.n_q_heads, d, c.n_q_heads / c.n_kv_heads, gamma)) return DFLASH_CUDA;
     ap.q = (const bf*)h->q;
     ap.out = (bf*)h->o;
     ap.len = cc->len;
@@ -984,8 +969,7 @@ int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* cc, const void*
     int splits, chunk;
     attn_plan(cc->batch, c.n_kv_heads, cc->capacity, h->num_sms, attn_max_cluster(d), splits, chunk);
     ap.tmap = cc->tm_slab;
-    if (!encode_q_map(&ap.tq, q, cc->batch * gamma, c.n_q_heads, d, c.n_q_heads / c.n_kv_heads, gamma))
-        return DFLASH_INVALID_ARG;
+    if ((uintptr_t)q & 15) return DFLASH_INVALID_ARG;   // q rows are read as 16-byte vectors
     ap.q = (const __nv_bfloat16*)q;
     ap.out = (__nv_bfloat16*)out;
     ap.len = cc->len;

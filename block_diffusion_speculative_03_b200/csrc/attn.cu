@@ -6,28 +6,30 @@
 // QKV epilogue wrote at [len, len+gamma): no mask.  CTA `rank` of the cluster
 // (b, g) takes keys [rank*chunk, (rank+1)*chunk).
 //
-//   warp 0   TMA: the Q tile once (a 3-D box gathers the G heads of every block
-//            position), then K/V tiles of 64 keys into a 3-stage ring.
-//   warp 1   tcgen05.mma (one thread): S_i = Q K_i^T into one of three TMEM
-//            buffers (M = 128 rows, N = 64 keys), issued up to three tiles
-//            ahead of the softmax, and O += P_i V_i into the TMEM accumulator
-//            (N = head_dim, V read as an MN-major operand straight from the
-//            TMA tile) once the softmax has written P_i.
-//   warps 2-5  softmax: reads S_i from TMEM, keeps a base-2 running maximum
-//            with an integer base B per row, writes P_i = bf16(2^(t - B)) into
-//            shared memory for the P.V MMA, and rescales O in TMEM by an exact
-//            power of two when B grows.
-//
 // The R <= 64 query rows fill CS = 2 (R > 32) or 4 copies of a window of
-// 128/CS rows of the M = 128 tile, so S holds every row CS times; the CS
-// threads that own a row's copies take 64/CS of each tile's keys each (a
-// thread reads only its own TMEM lane).  They agree on the row's base through
-// shared memory whenever one of them would move it, and add their partial
-// row sums at the end.  O accumulates in the first window's lanes.
+// RW = 128/CS lanes of an M = 128 tile: TMEM lane l holds query row l % RW and
+// takes key slice l / RW (64/CS keys) of every 64-key tile.  Q and P are MMA
+// operands in tensor memory, so the tensor cores read only K and V from
+// shared memory.
 //
-// Each CTA leaves its partial (B, l, O) in its own shared memory; after a
-// cluster barrier every CTA merges a slice of the rows by reading all partials
-// through distributed shared memory, and writes the bf16 output.
+//   warps 2-5  softmax, one TMEM lane per thread: first write the lane's Q row
+//            into TMEM; per tile read the lane's S slice, keep a base-2 running
+//            maximum with an integer base B per row, write P = bf16(2^(t - B))
+//            for the slice into a P buffer in TMEM (the lane's other columns
+//            stay zero), and rescale the lane's O by an exact power of two when
+//            B grows.  The lanes of a row agree on B through shared memory
+//            whenever one of them would move it.
+//   warp 0   TMA: K/V tiles of 64 keys into a kAttnStages-deep ring.
+//   warp 1   tcgen05.mma (one thread): S_i = Q K_i^T into one of three TMEM
+//            buffers (N = 64 keys), issued up to three tiles ahead of the
+//            softmax, and O += P_i V_i (N = head_dim, V an MN-major operand
+//            straight from the TMA tile) once P_i is written.
+//
+// Lane l of O so holds the P.V sum over key slice l / RW only; the CS lanes of
+// a row are added when the split's partial (B, l, O) is written to shared
+// memory.  After a cluster barrier every CTA merges a slice of the rows by
+// reading all partials through distributed shared memory, and writes the bf16
+// output.
 #include <cooperative_groups.h>
 
 #include "attn.cuh"
@@ -42,13 +44,18 @@ constexpr float kAttnBaseLag = 8.0f;
 template <int D>
 struct AttnCfg {
     static constexpr int HALVES = D / 64;
-    static constexpr int Q_BYTES = HALVES * 128 * 128;       // 128 query rows x D
     static constexpr int KV_BYTES = HALVES * 64 * 128;       // 64 keys x D
-    static constexpr int P_BYTES = 128 * 128;                // 128 rows x 64 keys
-    static constexpr int RING = Q_BYTES + 2 * kAttnStages * KV_BYTES + 2 * P_BYTES;
-    static constexpr int SMEM = 1024 + RING + 256 + 512;     // + barriers, + row exchange [128]
+    static constexpr int RING = 2 * kAttnStages * KV_BYTES;  // K ring, V ring
+    // + barriers, + row exchange [128]; at least half an SM's shared memory, so two of
+    // these CTAs (each allocating all 512 TMEM columns) never share an SM
+    static constexpr int SMEM = (1024 + RING + 768) > 117 * 1024 ? (1024 + RING + 768) : 117 * 1024;
     static constexpr int NS = 3;                             // S buffers in TMEM
-    static constexpr uint32_t TMEM_COLS = 512;               // S[NS] (NS x 64) at 0, O (D) at 256
+    static constexpr int PO_LD = D + 4;   // partial row stride (floats): 16-byte skew per row
+    // TMEM columns: S[NS] (NS x 64), Q (D/2 bf16 pairs), O (D), P[2] (2 x 32 bf16 pairs)
+    static constexpr uint32_t T_S = 0, T_Q = 192, T_O = 256, T_P = 384, TMEM_COLS = 512;
+    static_assert(T_S + NS * 64 <= T_Q && T_Q + D / 2 <= T_O && T_O + D <= T_P && T_P + 64 <= TMEM_COLS, "TMEM");
+    // the split's partial, written over the ring once the key loop is done
+    static_assert(128 * PO_LD * 4 + 64 * 8 + 3 * 64 * kAttnMaxSplits * 4 <= RING, "partial");
 };
 
 template <int D, int CS>
@@ -57,12 +64,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     constexpr int S = kAttnStages;
     constexpr int RW = 128 / CS;   // rows per window of the M = 128 tile
     constexpr int KC = 64 / CS;    // keys of a tile per softmax thread
+    constexpr int PO_LD = C::PO_LD;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* sQ = smem;
-    uint8_t* sK = sQ + C::Q_BYTES;                 // [S][KV_BYTES]
+    uint8_t* sK = smem;                            // [S][KV_BYTES]
     uint8_t* sV = sK + S * C::KV_BYTES;            // [S][KV_BYTES]
-    uint8_t* sP = sV + S * C::KV_BYTES;            // [2][P_BYTES]
     uint64_t* bars = (uint64_t*)(smem + C::RING);
     uint64_t* q_full = bars;
     uint64_t* kv_full = q_full + 1;                // [S]
@@ -74,9 +80,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     float* xch = (float*)(smem + C::RING + 256);   // [128] per TMEM lane: running max, then row sum
-    // After the key loop the front of shared memory holds this CTA's partial.
-    float* po = (float*)smem;                      // [64][D]
-    float2* pml = (float2*)(po + 64 * D);          // [64] (integer base, row sum)
+    // After the key loop the ring holds this CTA's partial.
+    float* po = (float*)smem;                      // [128][PO_LD] lanes' O, then rows 0..RW-1 summed
+    float2* pml = (float2*)(po + 128 * PO_LD);     // [64] (integer base, row sum)
     float* cm = (float*)(pml + 64);                // [64][splits] peers' bases
     float* cl = cm + 64 * kAttnMaxSplits;          // [64][splits] peers' sums
     float* cw = cl + 64 * kAttnMaxSplits;          // [64][splits] merge weights
@@ -89,12 +95,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     long long* trace = p.trace ? p.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 8
                                : nullptr;
     if (trace && tid == 0) trace[0] = (long long)globaltimer_ns();
-    if (tid == 0) {
-        tma_prefetch_desc(&p.tmap);
-        tma_prefetch_desc(&p.tq);
-    }
+    if (tid == 0) tma_prefetch_desc(&p.tmap);
     griddep_wait();
-    griddep_launch();
     if (trace && tid == 0) trace[1] = (long long)globaltimer_ns();
 
     const int R = p.G * p.gamma;
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     const long long rowV = rowK + p.rows_kind;
 
     if (tid == 0) {
-        mbar_init(q_full, 1);
+        mbar_init(q_full, 128);
         for (int i = 0; i < S; ++i) {
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
@@ -130,37 +132,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // Rows R..RW-1 of every window of the Q tile, and P rows RW..127 (never
-    // written, so O's lanes RW..127 stay zero), are zero.
-    {
-        const int per = (RW - R) * C::HALVES * 8;
-        for (int idx = tid; idx < CS * per; idx += kAttnThreads) {
-            const int k = idx / per, rem0 = idx % per;
-            const int r = k * RW + R + rem0 / (C::HALVES * 8), rem = rem0 % (C::HALVES * 8);
-            const int h = rem / 8, c16 = rem % 8;
-            *reinterpret_cast<uint4*>(sQ + h * 16384 + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
-        }
-        for (int idx = tid; idx < 2 * (128 - RW) * 8; idx += kAttnThreads) {
-            const int pb = idx / ((128 - RW) * 8), rem = idx % ((128 - RW) * 8);
-            *reinterpret_cast<uint4*>(sP + pb * C::P_BYTES + (RW + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-        }
-    }
-    fence_proxy_async();
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The next kernel may start only once this CTA holds its TMEM: a dependent CTA
+    // on this SM that allocated first and then waited for this grid would never
+    // let the allocation above succeed.
+    griddep_launch();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 256;
+    const uint32_t tS = tmem + C::T_S, tQ = tmem + C::T_Q, tO = tmem + C::T_O, tP = tmem + C::T_P;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, (uint32_t)(CS * R * D * 2));
-            for (int k = 0; k < CS; ++k)   // one copy of the R rows per window
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sQ + h * 16384 + k * RW * 128, &p.tq, q_full, h * 64, g * p.G, b * p.gamma);
             for (int it = 0; it < ntiles; ++it) {
                 const int st = it % S;
                 if (!mbar_wait(&kv_empty[st], (uint32_t)(((it / S) & 1) ^ 1), abort_flag, p.status)) break;
@@ -178,9 +163,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);   // Q (and zeroed P) in TMEM
+            tc_fence_after();
             if (trace) trace[2] = (long long)globaltimer_ns();
-            const uint32_t qa = smem_u32(sQ);
             // S_j = Q K_j^T into S buffer j % NS (free: the softmax has read S_{j-NS}).
             auto issue_s = [&](int j) -> bool {
                 const int st = j % S;
@@ -189,8 +174,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                 const uint32_t ka = smem_u32(sK + st * C::KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc_mma_bf16(tS + (j % C::NS) * 64, umma_desc_sw128(qa + (kk >> 2) * 16384) + 2 * (kk & 3),
-                                umma_desc_sw128(ka + (kk >> 2) * 8192) + 2 * (kk & 3), IDESC_S, kk > 0 ? 1u : 0u);
+                    tc_mma_bf16_ts(tS + (j % C::NS) * 64, tQ + kk * 8,
+                                   umma_desc_sw128(ka + (kk >> 2) * 8192) + 2 * (kk & 3), IDESC_S, kk > 0 ? 1u : 0u);
                 tc_commit(&s_full[j % C::NS]);
                 return true;
             };
@@ -200,12 +185,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                 const int pb = it & 1;
                 if (!mbar_wait(&p_full[pb], (uint32_t)((it >> 1) & 1), abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sP + pb * C::P_BYTES);
                 const uint32_t va = smem_u32(sV + (it % S) * C::KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc_mma_bf16(tO, umma_desc_sw128(pa) + 2 * kk, umma_desc_sw128_mn(va + kk * 2048, 8192, 1024),
-                                IDESC_PV, (it > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_bf16_ts(tO, tP + pb * 32 + kk * 8, umma_desc_sw128_mn(va + kk * 2048, 8192, 1024),
+                                   IDESC_PV, (it > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&o_done[pb]);
                 tc_commit(&kv_empty[it % S]);
                 if (it + C::NS < ntiles) ok = issue_s(it + C::NS);
@@ -223,6 +207,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         const int row = rl % RW, cs = rl / RW;         // query row, key slice (warp-uniform)
         const int e = tid - 64;                        // 0..127
         const uint32_t lanes = (uint32_t)(q4 * 32) << 16;
+        {
+            // The lane's Q row (zero past R) into the Q operand, and zeros into the
+            // lane's columns of both P buffers (other slices' keys stay zero).
+            const __nv_bfloat16* qsrc =
+                row < R ? p.q + ((size_t)(b * p.gamma + row / p.G) * p.nq + (size_t)(g * p.G + row % p.G)) * D
+                        : nullptr;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D / 2; c0 += 16) {   // columns c0..c0+15 = elements 2*c0..2*c0+31
+                float v[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 u = qsrc ? *reinterpret_cast<const uint4*>(qsrc + 2 * c0 + 8 * k) : make_uint4(0, 0, 0, 0);
+                    v[4 * k + 0] = __uint_as_float(u.x);
+                    v[4 * k + 1] = __uint_as_float(u.y);
+                    v[4 * k + 2] = __uint_as_float(u.z);
+                    v[4 * k + 3] = __uint_as_float(u.w);
+                }
+                tmem_st16(tQ + lanes + c0, v);
+            }
+            float z[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) tmem_st16(tP + lanes + c0, z);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(q_full);
+        }
         float base = -INFINITY, mt = -INFINITY, l = 0.f;
         bool ok = true;
         for (int it = 0; it < ntiles; ++it) {
@@ -233,30 +245,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             if (trace && it == 0 && e == 0) trace[3] = (long long)globaltimer_ns();
             const int kvb = kv0 + it * 64 + cs * KC;   // first key of this thread's slice
             const uint32_t ts = tS + lanes + sbuf * 64 + cs * KC;
-            // the slice's scores, in log2 units, masked past the last key; its maximum
-            // over 8 independent partial maxima (exact in any order)
+            // the slice's raw scores, masked past the last key, and their maximum over 8
+            // independent partial maxima (exact in any order).  The scale to log2 units
+            // is applied to the maximum (rounding is monotonic, so this equals the
+            // maximum of the scaled scores) and inside the exponent's FMA.
             float t[KC];
             if constexpr (KC == 32) tmem_ld32w(ts, t); else tmem_ld16w(ts, t);
             const int nvalid = kv1 - kvb;
+            if (nvalid < KC) {
+#pragma unroll
+                for (int i = 0; i < KC; ++i) t[i] = (i < nvalid) ? t[i] : -INFINITY;
+            }
             float m8[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
-            if (nvalid >= KC) {
+            for (int k = 0; k < 8; ++k) m8[k] = t[k];
 #pragma unroll
-                for (int i = 0; i < KC; ++i) {
-                    t[i] *= p.scale_log2;
-                    m8[i & 7] = fmaxf(m8[i & 7], t[i]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < KC; ++i) {
-                    t[i] = (i < nvalid) ? t[i] * p.scale_log2 : -INFINITY;
-                    m8[i & 7] = fmaxf(m8[i & 7], t[i]);
-                }
-            }
+            for (int i = 8; i < KC; ++i) m8[i & 7] = fmaxf(m8[i & 7], t[i]);
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mt = fmaxf(mt, mx);   // running maximum of this slice
+            mt = fmaxf(mt, mx * p.scale_log2);   // running maximum of this slice, log2 units
             if (ok && it >= 2)   // the P.V of tile it-2 read this P buffer: wait for it
                 ok = mbar_wait(&o_done[sb], (uint32_t)(((it - 2) >> 1) & 1), abort_flag, p.status);
             // The integer base may lag the running maximum by up to kAttnBaseLag: P is
@@ -277,9 +284,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                 const float nb = floorf(mrow);
                 const bool grow = nb > base + kAttnBaseLag;
                 if (it >= 1) {
-                    // Rescale O and l by 2^(base - nb), an exact power of two (the TMEM
-                    // accesses are warp-collective, so all 128 threads take part; rows
-                    // whose base did not grow scale by 1).
+                    // Rescale the lane's O and l by 2^(base - nb), an exact power of two
+                    // (the TMEM accesses are warp-collective, so all 128 threads take
+                    // part; rows whose base did not grow scale by 1).
                     ok = mbar_wait(&o_done[(it - 1) & 1], (uint32_t)(((it - 1) >> 1) & 1), abort_flag, p.status);
                     if (named_bar_or(1, 128, !ok)) { ok = false; break; }
                     tc_fence_after();
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
 #pragma unroll 1
                     for (int c0 = 0; c0 < D; c0 += 16) {
                         float v[16];
-                        tmem_ld16(tO + lanes + c0, v);
+                        tmem_ld16w(tO + lanes + c0, v);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) v[i] *= f;
                         tmem_st16(tO + lanes + c0, v);
@@ -306,29 +313,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                     const int r = valid + idx / (C::HALVES * 8), rem = idx % (C::HALVES * 8);
                     *reinterpret_cast<uint4*>(vs + (rem / 8) * 8192 + r * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
                 }
+                fence_proxy_async();   // the P.V MMA reads these rows through the async proxy
             }
-            // P = bf16(2^(t - base)) into the swizzled K-major P tile: row `row`,
-            // keys cs*KC .. cs*KC+KC-1.
-            uint8_t* prow = sP + sb * C::P_BYTES + row * 128;
+            // P = bf16(2^(t - base)) of the slice's keys, two per TMEM column, into
+            // this lane's columns cs*KC/2 .. of P buffer sb.
             const float bb = (base == -INFINITY) ? 0.f : base;
+            uint32_t pk[KC / 2];
             float ls[KC / 16];   // independent partial sums, one per 16 keys
 #pragma unroll
             for (int c0 = 0; c0 < KC; c0 += 16) {
-                uint32_t pk[8];
                 float s2 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
-                    const float e0 = ex2_fast(t[c0 + i] - bb), e1 = ex2_fast(t[c0 + i + 1] - bb);
+                    const float e0 = ex2_fast(fmaf(t[c0 + i], p.scale_log2, -bb));
+                    const float e1 = ex2_fast(fmaf(t[c0 + i + 1], p.scale_log2, -bb));
                     s2 += e0 + e1;
-                    pk[i / 2] = pack_bf16(e0, e1);
+                    pk[(c0 + i) / 2] = pack_bf16(e0, e1);
                 }
                 ls[c0 >> 4] = s2;
-                const int ch = (cs * KC + c0) >> 3;   // 16-byte chunk of 8 keys
-                *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(prow + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
-            if constexpr (KC == 32) l += ls[0] + ls[1]; else l += ls[0];
-            fence_proxy_async();
+            const uint32_t tp = tP + lanes + sb * 32 + cs * (KC / 2);
+            if constexpr (KC == 32) {
+                float pv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pv[i] = __uint_as_float(pk[i]);
+                tmem_st16(tp, pv);
+                l += ls[0] + ls[1];
+            } else {
+                tmem_st8u(tp, pk);
+                l += ls[0];
+            }
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[sb]);
         }
@@ -340,23 +355,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         }
         if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
         xch[rl] = l;              // the slices' partial row sums (same base)
-        named_bar_sync(1, 128);   // every softmax thread is past its P writes before the front is reused
+        named_bar_sync(1, 128);   // every softmax thread is past the key loop before the ring is reused
         float lrow = l;
 #pragma unroll
         for (int k = 1; k < CS; ++k) lrow += xch[(rl + k * RW) & 127];
+        // the lane's O (its key slice's share of the row) into po[rl]
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
             float v[16];
             if (ok && ntiles >= 1) {
-                tmem_ld16(tO + lanes + c0, v);
+                tmem_ld16w(tO + lanes + c0, v);
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = 0.f;
             }
-            if (cs == 0) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) po[row * D + c0 + i] = v[i];
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(po + rl * PO_LD + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        named_bar_sync(1, 128);
+        // add the CS slices of each row into its first-window lane; the row's CS
+        // threads take D/CS columns each
+#pragma unroll 1
+        for (int c = cs * (D / CS); c < (cs + 1) * (D / CS); c += 4) {
+            float4 a = *reinterpret_cast<const float4*>(po + row * PO_LD + c);
+#pragma unroll
+            for (int k = 1; k < CS; ++k) {
+                const float4 o2 = *reinterpret_cast<const float4*>(po + (row + k * RW) * PO_LD + c);
+                a.x += o2.x;
+                a.y += o2.y;
+                a.z += o2.z;
+                a.w += o2.w;
             }
+            *reinterpret_cast<float4*>(po + row * PO_LD + c) = a;
         }
         if (cs == 0) pml[row] = make_float2(base, ok ? lrow : 0.f);
     }
@@ -407,7 +438,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         float4 v[kAttnMaxSplits];
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
-            v[s2] = s2 < nsplit ? *reinterpret_cast<const float4*>(rpo[s2] + r * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[s2] = s2 < nsplit ? *reinterpret_cast<const float4*>(rpo[s2] + r * PO_LD + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {

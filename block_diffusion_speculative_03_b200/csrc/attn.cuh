@@ -6,8 +6,7 @@ namespace df {
 
 struct AttnParams {
     CUtensorMap tmap;            // cache slab as 2-D [rows, d] bf16, box {64, 64}, 128-byte swizzle
-    CUtensorMap tq;              // q as 3-D [B*gamma][nq][d] bf16, box {64, G, gamma}, 128-byte swizzle
-    const __nv_bfloat16* q;      // [B*gamma, nq*d]
+    const __nv_bfloat16* q;      // [B*gamma, nq*d], 16-byte aligned
     __nv_bfloat16* out;          // [B*gamma, nq*d]
     const int* len;
     const int* req_ok;
@@ -16,12 +15,12 @@ struct AttnParams {
     float scale_log2;            // log2(e) / sqrt(d)
     int* status;
     // Diagnostic trace (null in normal use): per CTA 8 globaltimer stamps (ns):
-    // entry, past the dependency wait, Q staged, first tile landed, key loop done,
+    // entry, past the dependency wait, Q in tensor memory, first tile landed, key loop done,
     // partial ready, past the first cluster barrier, merge done.
     long long* trace;
 };
 
-constexpr int kAttnStages = 5;   // K/V ring depth: each stage is held until its tile's P.V is done
+constexpr int kAttnStages = 7;   // K/V ring depth: each stage is held until its tile's P.V is done
 constexpr int kAttnThreads = 192;   // TMA warp, MMA warp, 4 softmax warps
 constexpr int kAttnMaxSplits = 8;   // CTAs per cluster (portable cluster size)
 

@@ -99,12 +99,13 @@ const char* dflash_diag_timed_name(int kind);
  * layer `layer`, q (device bf16 [batch*gamma, n_q_heads*head_dim], rows b*gamma+j)
  * attends over cache rows [0, len[b] + gamma) of that layer (the caller writes
  * the block's own K/V rows at [len, len+gamma) and keeps len + gamma <= capacity);
- * out: device bf16, same layout as q.  Synchronises the stream. */
+ * out: device bf16, same layout as q.  q must be 16-byte aligned (DFLASH_INVALID_ARG
+ * otherwise).  Synchronises the stream. */
 int dflash_diag_attention(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
                           dflash_stream stream);
 
 /* Same, recording per-CTA timestamps into trace (device int64[batch * n_kv_heads
- * * splits * 8]: entry, past the dependency wait, Q staged, first tile landed,
+ * * splits * 8]: entry, past the dependency wait, Q in tensor memory, first tile landed,
  * key loop done, partial ready, past the cluster barrier, merge done) and the
  * split count used into *splits_out (host int, may be NULL). */
 int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
