@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 OUT = os.path.join(PKG, "libdflash.so")
-SOURCES = ["abi.cu", "gemm_tc.cu", "attn.cu", "kernels.cu", "gemm_noalloc.cu"]
+SOURCES = ["abi.cu", "gemm_tc.cu", "attn.cu", "kernels.cu", "gemm_noalloc.cu", "policy.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + os.path.join(ROOT, "include")]

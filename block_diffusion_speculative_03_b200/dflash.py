@@ -1,4 +1,5 @@
-"""ctypes binding of libdflash (include/dflash.h, include/dflash_diag.h).
+"""ctypes binding of libdflash (include/dflash.h, include/dflash_diag.h,
+include/dflash_policy.h).
 
 Functions carry the C names and only marshal arguments: every step of the
 draft step runs in the library's CUDA kernels.  Pointers are passed as ints
@@ -53,6 +54,16 @@ class dflash_cache_info(C.Structure):
                 ("stride_kind", C.c_int64), ("stride_layer", C.c_int64), ("stride_request", C.c_int64)]
 
 
+DFLASH_POLICY_MAX_CANDIDATES = 8
+
+
+class dflash_gamma_policy(C.Structure):
+    _fields_ = [("n_candidates", C.c_int), ("candidates", C.c_int * DFLASH_POLICY_MAX_CANDIDATES),
+                ("decay", C.c_double), ("cost_fixed", C.c_double), ("cost_per_token", C.c_double),
+                ("prior_accepts", C.c_double), ("prior_rejects", C.c_double), ("accepts", C.c_double),
+                ("rejects", C.c_double)]
+
+
 _lib = None
 
 
@@ -97,6 +108,12 @@ def lib():
         "dflash_diag_gemm_bf16_traced": (i32, [vp, vp, vp, i32, i32, i32, vp, sz, i32, vp, vp]),
         "dflash_diag_attention_traced": (i32, [vp, vp, vp, vp, i32, i32, vp, C.POINTER(i32), vp]),
         "dflash_diag_gemm_bf16_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
+        "dflash_gamma_policy_init": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(i32), i32, C.c_double,
+                                           C.c_double, C.c_double, C.c_double, C.c_double]),
+        "dflash_gamma_policy_observe": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(C.c_int32), i32, i32]),
+        "dflash_gamma_policy_alpha": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(C.c_double)]),
+        "dflash_gamma_policy_expected_tokens": (i32, [C.c_double, i32, C.POINTER(C.c_double)]),
+        "dflash_gamma_policy_choose": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(i32)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -115,7 +132,9 @@ def exported_symbols() -> list:
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_wait_selftest",
             "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
-            "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc"]
+            "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc",
+            "dflash_gamma_policy_init", "dflash_gamma_policy_observe", "dflash_gamma_policy_alpha",
+            "dflash_gamma_policy_expected_tokens", "dflash_gamma_policy_choose"]
 
 
 def _chk(st: int, where: str, check: bool = True) -> int:
@@ -291,3 +310,41 @@ def dflash_diag_attention_traced(h: int, c: int, q: int, out: int, layer: int, g
     _chk(lib().dflash_diag_attention_traced(h, c, q, out, layer, gamma, trace, C.byref(sp), stream),
          "dflash_diag_attention_traced")
     return sp.value
+
+
+# -- block-size policy (include/dflash_policy.h; host arithmetic, no device) -------
+def dflash_gamma_policy_init(candidates: Sequence[int], decay: float, cost_fixed: float, cost_per_token: float,
+                             prior_accepts: float, prior_rejects: float, check: bool = True):
+    """Returns a new dflash_gamma_policy (or the status when check=False and it fails)."""
+    p = dflash_gamma_policy()
+    arr = (C.c_int * max(len(candidates), 1))(*candidates)
+    st = lib().dflash_gamma_policy_init(C.byref(p), arr, len(candidates), decay, cost_fixed, cost_per_token,
+                                        prior_accepts, prior_rejects)
+    _chk(st, "dflash_gamma_policy_init", check)
+    return p if st == 0 else st
+
+
+def dflash_gamma_policy_observe(p: dflash_gamma_policy, accept_len: Sequence[int], gamma: int,
+                                check: bool = True) -> int:
+    arr = (C.c_int32 * max(len(accept_len), 1))(*[int(a) for a in accept_len])
+    return _chk(lib().dflash_gamma_policy_observe(C.byref(p), arr, len(accept_len), gamma),
+                "dflash_gamma_policy_observe", check)
+
+
+def dflash_gamma_policy_alpha(p: dflash_gamma_policy) -> float:
+    out = C.c_double()
+    _chk(lib().dflash_gamma_policy_alpha(C.byref(p), C.byref(out)), "dflash_gamma_policy_alpha")
+    return out.value
+
+
+def dflash_gamma_policy_expected_tokens(alpha: float, gamma: int, check: bool = True):
+    out = C.c_double()
+    st = lib().dflash_gamma_policy_expected_tokens(alpha, gamma, C.byref(out))
+    _chk(st, "dflash_gamma_policy_expected_tokens", check)
+    return out.value if st == 0 else st
+
+
+def dflash_gamma_policy_choose(p: dflash_gamma_policy) -> int:
+    out = C.c_int()
+    _chk(lib().dflash_gamma_policy_choose(C.byref(p), C.byref(out)), "dflash_gamma_policy_choose")
+    return out.value

@@ -1,7 +1,8 @@
 """Torch-memory convenience layer over the C ABI.
 
 :class:`Drafter` owns the device workspace and borrows the weight tensors;
-:class:`Cache` owns the cache memory of a batch of requests.  All arithmetic
+:class:`Cache` owns the cache memory of a batch of requests; :class:`GammaPolicy`
+holds the host-side block-size policy between cycles.  All arithmetic
 happens in libdflash; this module allocates device memory with torch, passes
 pointers and the current CUDA stream, and checks statuses.
 """
@@ -166,6 +167,31 @@ class Drafter:
                 self.handle = None
         except Exception:
             pass
+
+
+class GammaPolicy:
+    """Block size for the next cycle from the acceptance lengths seen so far
+    (include/dflash_policy.h): a geometric acceptance estimate with forgetting
+    factor `decay`, and the candidate with the most expected committed tokens per
+    unit of cycle cost (cost_fixed + cost_per_token * gamma).  Host only."""
+
+    def __init__(self, candidates: Sequence[int] = (4, 8, 16), decay: float = 0.5, cost_fixed: float = 1.0,
+                 cost_per_token: float = 0.02, prior_accepts: float = 1.0, prior_rejects: float = 1.0):
+        self.state = D.dflash_gamma_policy_init(list(candidates), decay, cost_fixed, cost_per_token,
+                                                prior_accepts, prior_rejects)
+
+    def choose(self) -> int:
+        return D.dflash_gamma_policy_choose(self.state)
+
+    def observe(self, accept_len, gamma: int) -> None:
+        """accept_len: the cycle's acceptance lengths (host sequence or tensor)."""
+        if torch.is_tensor(accept_len):
+            accept_len = accept_len.cpu().tolist()
+        D.dflash_gamma_policy_observe(self.state, list(accept_len), gamma)
+
+    @property
+    def alpha(self) -> float:
+        return D.dflash_gamma_policy_alpha(self.state)
 
 
 def shape_from_workload(w) -> Dict:

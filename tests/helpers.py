@@ -49,3 +49,21 @@ def synth_target(drafts: np.ndarray, a_star: int, rand_tokens: np.ndarray, vocab
     if a_star < gamma - 1 and t[a_star] == drafts[a_star]:
         t[a_star] = (t[a_star] + 1) % vocab
     return t
+
+
+def gamma_schedule(w: I.Workload, cycles: int, candidates, decay: float = 0.5, cost_fixed: float = 1.0,
+                   cost_per_token: float = 0.05, prior=(1.0, 1.0)):
+    """Block sizes the library's gamma policy picks over `cycles` cycles of
+    workload w, with each cycle's planned acceptance lengths (the workload's plan
+    for its largest block, clipped to the block picked: the same truncated
+    geometric law).  Host values only, fed alike to the GPU path and the oracle."""
+    from block_diffusion_speculative_03_b200 import dflash as D
+    plan = I.plan_accept(w, cycles, gamma=max(candidates)).numpy()
+    p = D.dflash_gamma_policy_init(list(candidates), decay, cost_fixed, cost_per_token, prior[0], prior[1])
+    out = []
+    for c in range(cycles):
+        g = D.dflash_gamma_policy_choose(p)
+        a = np.minimum(plan[c], g - 1).astype(np.int32)
+        D.dflash_gamma_policy_observe(p, a.tolist(), g)
+        out.append((g, a))
+    return out

@@ -24,7 +24,7 @@ def _declared(header):
 
 
 def test_exports_every_declared_symbol(lib):
-    names = _declared("dflash.h") + _declared("dflash_diag.h")
+    names = _declared("dflash.h") + _declared("dflash_diag.h") + _declared("dflash_policy.h")
     assert len(names) >= 20
     for n in names:
         assert hasattr(lib, n), n

@@ -8,6 +8,7 @@ import pytest
 import torch
 
 from block_diffusion_speculative_03_b200 import inputs as I
+from tests.helpers import gamma_schedule
 from tests.parity import Pair
 
 pytestmark = pytest.mark.gpu
@@ -51,6 +52,26 @@ def test_small_bf16_untied_ragged_heads_and_empty_context():
     # request with an empty context, separate LM head
     n = _chain("small_bf16_untied")
     assert n > 0
+
+
+def test_small_bf16_chain_dynamic_block_size():
+    # The block size follows the host-side gamma policy from cycle to cycle
+    # (4 -> 8 -> 16 -> 8 ...), through the same cache: every cycle's drafts,
+    # acceptance, next anchor and cache rows against the oracle.
+    w = I.preset("small_bf16")
+    w.cycles = 6
+    sched = gamma_schedule(w, w.cycles, (4, 8, 16), decay=0.5, cost_per_token=0.02)
+    assert len({g for g, _ in sched}) == 3
+    pr = Pair(w)
+    pr.prefill()
+    anchors = I.make_anchors(w).numpy()
+    compared = 0
+    for cyc, (g, a_star) in enumerate(sched):
+        o_dr, g_dr, n = pr.draft(anchors, g)
+        compared += n
+        anchors = pr.verify_and_accept(o_dr, g, a_star, cyc)
+        pr.check_cache()
+    assert compared > 0
 
 
 @pytest.mark.parametrize("gamma", [1, 2, 5, 8])
