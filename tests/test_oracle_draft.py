@@ -116,6 +116,28 @@ def test_draft_step_matches_torch_library_composition_bf16():
     assert np.array_equal(drafts[ok], rlog.argmax(1).numpy()[ok])
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_empty_context_is_a_bidirectional_encoder_over_the_block(dtype):
+    # T = 0: nothing injected, so the block attends only to itself, at positions
+    # 0..gamma-1, with no mask: a plain bidirectional encoder over the block.
+    w = micro(dtype, context=[0])
+    W = I.make_weights(w)
+    od = oracle_drafter(w, W)
+    cache = od.new_cache(8)
+    cache["committed"] = cache["len"]
+    assert cache["len"] == 0
+    drafts, margin, logits = od.draft_block(cache, 23, 6, want_logits=True)
+    empty = [h[:0] for h in I.make_hiddens(w, 1)]
+    _, _, _, rlog = torch_reference(w, W, empty, 6, 23)
+    if dtype == "f32":
+        assert np.allclose(logits, rlog.numpy(), rtol=1e-9, atol=1e-11)
+        assert np.array_equal(drafts, rlog.argmax(1).numpy())
+    else:
+        assert np.max(np.abs(logits - rlog.numpy())) < 2e-2
+        ok = margin > 0.05
+        assert np.array_equal(drafts[ok], rlog.argmax(1).numpy()[ok])
+
+
 def test_fuse_concat_order_and_projection():
     # W_fc = [0 | I | 0] picks exactly the second selected layer: ctx = RMSNorm(h_1) * g
     w = micro("f32", hidden=32, target_hidden=32)
