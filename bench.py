@@ -70,7 +70,7 @@ def env_int(name, default):
 # one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
 # kernel sources it was taken on; once they change the figure is void.
 GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.6e6,
-                "sources_sha256": "5c4b7b9aa3ddbb6dcf12f1b4e71973eea6395cbf3e52ec4be4086c7718434762"}
+                "sources_sha256": "75cc540e3725c847588f0130c9c199a236f956bcbadbbafa2e92e6119d82f48f"}
 
 
 def gemm_sources_sha256():

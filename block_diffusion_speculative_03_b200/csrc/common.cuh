@@ -267,13 +267,6 @@ DF_DEV void tmem_st8u(uint32_t taddr, const uint32_t* v) {
 }
 DF_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-DF_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // UMMA shared-memory descriptor of an MN-major operand tile stored with the
 // 128-byte swizzle: rows of 64 bf16 along M/N (128 B), 8-row groups along K
 // `sbo` bytes apart, groups of 64 M/N elements `lbo` bytes apart.
