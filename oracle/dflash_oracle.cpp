@@ -20,6 +20,8 @@
 //   * §5 (claims), lossless verification: drafts are kept only while they equal
 //     the target's own greedy tokens                      -> oracle_accept
 //   * §2.3 loss-weighting bullet: w_k = exp(-(k-1)/gamma)  -> oracle_loss_weights
+//   * §3 contribution 2 / §4 KV-injection ablation: the input-fusion drafter that
+//     KV injection is compared against                  -> oracle_ingest_fused_input
 //
 // The summaries give no layer equations.  The layer internals used here
 // (pre-norm RMSNorm, rotate-half RoPE, grouped-query attention without a mask,
@@ -35,7 +37,8 @@
 // and invariants; accept exhaustively against a brute-force scan; the loss
 // weights against their closed form; fuse, inject and draft through invariants
 // (concat order, chunked = one-shot injection, one bidirectional pass, zero
-// layers = norm + shared head).  The composition of oracle_fuse_context,
+// layers = norm + shared head); the input-fusion ingest against a torch causal
+// composition, chunked = one-shot, and one layer = injecting the normed feature.  The composition of oracle_fuse_context,
 // oracle_inject_kv and oracle_draft_block as a DFlash drafter (norm placement,
 // positions, mask id) follows the reading above and cannot be checked against
 // a trained DFlash model here: parity unpinned against the paper's model.
@@ -292,6 +295,89 @@ void oracle_inject_kv(const oracle_config* c, const oracle_weights* w, const dou
                 }
             }
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Input-fusion ablation (the conditioning DFlash is compared against: DFlash
+// technical summary, §3 contribution 2 and the KV-injection ablation bullet of
+// §4).  Instead of a2, context row r at absolute position p = pos0 + r enters
+// the drafter as its input hidden state x = ctx_r and passes through the draft
+// layers like a token; each layer caches the K/V of its own normed state:
+//   h = R(RMSNorm(x) * g_in,l);  K_l[p] = R(RoPE_p(h . W_k,l^T));  V_l[p] = R(h . W_v,l^T)
+//   q = R(RoPE_p(h . W_q,l^T));  o = R(attention over cached rows [0, p]) (causal)
+//   x = R(x + o . W_o,l^T);  h2 = R(RMSNorm(x) * g_post,l);
+//   m = R(silu(h2 . W_g,l^T) * (h2 . W_u,l^T));  x = R(x + m . W_d,l^T)
+// The last layer's attention and MLP change no cached value and are skipped.
+// Rows are appended in order and attend only to rows at or before their own
+// position, so appending in chunks gives the same cache as appending at once.
+// ---------------------------------------------------------------------------
+void oracle_ingest_fused_input(const oracle_config* c, const oracle_weights* w, const double* ctx,
+                               int rows, int pos0, double* k_cache, double* v_cache, int cap) {
+    g_acc32 = c->acc32;
+    int S = c->storage, H = c->hidden, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
+    int Nq = nq * d, Nkv = nkv * d, I = c->intermediate;
+    std::vector<double> x(ctx, ctx + (size_t)rows * H);
+    std::vector<double> g(H), tmp(H), h((size_t)rows * H), y((size_t)rows * H);
+    std::vector<double> q((size_t)rows * Nq), kk((size_t)rows * Nkv), vv((size_t)rows * Nkv), o((size_t)rows * Nq);
+    std::vector<double> gt((size_t)rows * I), up((size_t)rows * I), mm((size_t)rows * I);
+    for (int l = 0; l < c->n_layers; ++l) {
+        load_vec(w->g_in[l], H, S, g.data());
+        for (int r = 0; r < rows; ++r) {
+            oracle_rmsnorm(x.data() + (size_t)r * H, g.data(), H, c->rms_eps, tmp.data());
+            for (int t = 0; t < H; ++t) h[(size_t)r * H + t] = R(tmp[t], S);
+        }
+        linear(h.data(), rows, H, w->wk[l], Nkv, S, kk.data());
+        linear(h.data(), rows, H, w->wv[l], Nkv, S, vv.data());
+        for (int r = 0; r < rows; ++r) {
+            long p = (long)pos0 + r;
+            for (int g2 = 0; g2 < nkv; ++g2) {
+                double* kh = kk.data() + (size_t)r * Nkv + (size_t)g2 * d;
+                const double* vh = vv.data() + (size_t)r * Nkv + (size_t)g2 * d;
+                oracle_rope(kh, d, p, c->rope_theta);
+                size_t base = (((size_t)l * nkv + g2) * cap + p) * d;
+                for (int t = 0; t < d; ++t) {
+                    k_cache[base + t] = R(kh[t], S);
+                    v_cache[base + t] = R(vh[t], S);
+                }
+            }
+        }
+        if (l == c->n_layers - 1) break;
+        linear(h.data(), rows, H, w->wq[l], Nq, S, q.data());
+        for (int r = 0; r < rows; ++r)
+            for (int hq = 0; hq < nq; ++hq)
+                oracle_rope(q.data() + (size_t)r * Nq + (size_t)hq * d, d, (long)pos0 + r, c->rope_theta);
+        for (auto& e : q) e = R(e, S);
+        // causal: row r reads cached rows [0, pos0 + r]
+        for (int r = 0; r < rows; ++r) {
+            int n = pos0 + r + 1;
+            std::vector<double> K((size_t)nkv * n * d), Vv((size_t)nkv * n * d);
+            for (int g2 = 0; g2 < nkv; ++g2)
+                for (int i = 0; i < n; ++i)
+                    for (int t = 0; t < d; ++t) {
+                        size_t src = (((size_t)l * nkv + g2) * cap + i) * d + t;
+                        K[((size_t)g2 * n + i) * d + t] = k_cache[src];
+                        Vv[((size_t)g2 * n + i) * d + t] = v_cache[src];
+                    }
+            oracle_attention(q.data() + (size_t)r * Nq, 1, nq, K.data(), Vv.data(), n, nkv, d, S == 1,
+                             o.data() + (size_t)r * Nq);
+        }
+        for (auto& e : o) e = R(e, S);
+        linear(o.data(), rows, Nq, w->wo[l], H, S, y.data());
+        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
+        load_vec(w->g_post[l], H, S, g.data());
+        for (int r = 0; r < rows; ++r) {
+            oracle_rmsnorm(x.data() + (size_t)r * H, g.data(), H, c->rms_eps, tmp.data());
+            for (int t = 0; t < H; ++t) h[(size_t)r * H + t] = R(tmp[t], S);
+        }
+        linear(h.data(), rows, H, w->w_gate[l], I, S, gt.data());
+        linear(h.data(), rows, H, w->w_up[l], I, S, up.data());
+        for (size_t i = 0; i < mm.size(); ++i) {
+            double a = gt[i];
+            mm[i] = R(a / (1.0 + std::exp(-a)) * up[i], S);
+        }
+        linear(mm.data(), rows, I, w->w_down[l], H, S, y.data());
+        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
     }
 }
 

@@ -52,6 +52,8 @@ def lib():
         L.oracle_fuse_context.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.POINTER(C.c_void_p),
                                           C.c_long, C.c_int, dp]
         L.oracle_inject_kv.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, C.c_int, dp, dp, C.c_int]
+        L.oracle_ingest_fused_input.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, C.c_int, dp, dp,
+                                                C.c_int]
         L.oracle_draft_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, dp, C.c_int, C.c_int,
                                          C.c_int, C.c_int, ip, dp, dp]
         L.oracle_accept.restype = C.c_int
@@ -187,6 +189,18 @@ class OracleDrafter:
             raise ValueError("capacity")
         lib().oracle_inject_kv(C.byref(self.cfg), C.byref(self.w), _dp(ctx), rows, cache["len"],
                                _dp(cache["k"]), _dp(cache["v"]), cache["cap"])
+        cache["len"] += rows
+
+    def ingest_fused_input(self, cache: Dict, ctx: np.ndarray) -> None:
+        """Input-fusion ablation: the context rows pass through the draft layers as
+        input hidden states (causal over the context) and every layer caches the
+        K/V of its own normed state, in place of inject_kv."""
+        ctx = np.ascontiguousarray(ctx, dtype=np.float64)
+        rows = ctx.shape[0]
+        if cache["len"] + rows > cache["cap"]:
+            raise ValueError("capacity")
+        lib().oracle_ingest_fused_input(C.byref(self.cfg), C.byref(self.w), _dp(ctx), rows, cache["len"],
+                                        _dp(cache["k"]), _dp(cache["v"]), cache["cap"])
         cache["len"] += rows
 
     def draft_block(self, cache: Dict, anchor: int, gamma: int, want_logits: bool = False):
