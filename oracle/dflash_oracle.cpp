@@ -150,17 +150,19 @@ void oracle_rope(double* v, int d, long pos, double theta) {
     }
 }
 
-// Multi-head attention without a mask.  q: [nrow][nq][d]; k, v: [nkv][n][d];
-// o: [nrow][nq][d].  Query head hq reads key/value head hq / (nq/nkv).
-// Scores are scaled by 1/sqrt(d).  The softmax is written in base 2 with an
-// integer shift: t_i = s_i * log2(e) / sqrt(d), B = floor(max_i t_i),
-// e_i = 2^(t_i - B), o = sum_i e_i v_i / sum_i e_i, which is the softmax.  With
-// round_p != 0 the weights e_i are rounded to bf16 before they multiply V (the
-// denominator keeps the unrounded e_i); shifting by an integer B makes that
-// rounding independent of how the keys are split into blocks.  The output is
-// not rounded here.
-void oracle_attention(const double* q, int nrow, int nq, const double* k, const double* v,
-                      int n, int nkv, int d, int round_p, double* o) {
+// Multi-head attention without a mask, over one block of keys, unnormalised.
+// q: [nrow][nq][d]; k, v: [nkv][n][d].  Query head hq reads key/value head
+// hq / (nq/nkv).  Scores are scaled by 1/sqrt(d) and the softmax is written in
+// base 2 with an integer shift: t_i = (q . k_i) * log2(e) / sqrt(d),
+// B = floor(max_i t_i), e_i = 2^(t_i - B).  Outputs per (row, head):
+//   num[r][hq][u] = sum_i P_i v_i[u] with P_i = e_i, or R(e_i) (bf16) when round_p,
+//   z[r][hq]      = sum_i e_i        (the unrounded weights),
+//   base[r][hq]   = B                (-inf when n == 0).
+// Because B is an integer, the weights of a key are the same numbers times an
+// exact power of two whatever block of keys it is in, so blocks with their own
+// bases combine exactly: rescale each block's num and z by 2^(B_block - B_all).
+void oracle_attention_block(const double* q, int nrow, int nq, const double* k, const double* v,
+                            int n, int nkv, int d, int round_p, double* num, double* z, double* base) {
     int G = nq / nkv;
     const double scale = 1.4426950408889634 / std::sqrt((double)d);   // log2(e) / sqrt(d)
     #pragma omp parallel for collapse(2) schedule(static)
@@ -181,15 +183,28 @@ void oracle_attention(const double* q, int nrow, int nq, const double* k, const 
             const double B = std::floor(m);
             double Z = 0.0;
             for (int i = 0; i < n; ++i) { t[i] = std::exp2(t[i] - B); Z += t[i]; }
-            double* ov = o + ((long)r * nq + hq) * d;
+            double* ov = num + ((long)r * nq + hq) * d;
             for (int u = 0; u < d; ++u) ov[u] = 0.0;
             for (int i = 0; i < n; ++i) {
                 double e = round_p ? oracle_round_bf16(t[i]) : t[i];
                 for (int u = 0; u < d; ++u) ov[u] += e * vh[(long)i * d + u];
             }
-            for (int u = 0; u < d; ++u) ov[u] /= Z;
+            z[(long)r * nq + hq] = Z;
+            base[(long)r * nq + hq] = B;
         }
     }
+}
+
+// Attention output: o = num / z of oracle_attention_block over all n keys,
+// which is softmax(q K^T / sqrt(d)) V (with round_p: the bf16-rounded weights
+// R(2^(t_i - B)) in the numerator, the unrounded ones in the denominator).  The
+// output is not rounded here.
+void oracle_attention(const double* q, int nrow, int nq, const double* k, const double* v,
+                      int n, int nkv, int d, int round_p, double* o) {
+    std::vector<double> z((size_t)nrow * nq), base((size_t)nrow * nq);
+    oracle_attention_block(q, nrow, nq, k, v, n, nkv, d, round_p, o, z.data(), base.data());
+    for (long rh = 0; rh < (long)nrow * nq; ++rh)
+        for (int u = 0; u < d; ++u) o[rh * d + u] /= z[rh];
 }
 
 // y[m][n] = sum_k x[m][k] * W[n][k]; W in storage type, [N, K] row-major.
@@ -382,104 +397,97 @@ void oracle_ingest_fused_input(const oracle_config* c, const oracle_weights* w, 
 }
 
 // ---------------------------------------------------------------------------
-// a3..a7: draft one block of gamma positions in one forward pass.
-// Position 0 holds the clean anchor token, positions 1..gamma-1 the mask
-// token; block position j sits at absolute position len + j.  Every block
-// query sees the whole committed context [0, len) and every block position
-// (no mask).  The block's own K/V are used for this pass only and are not
-// written to the cache.  Mask position j predicts the token at len + j:
-// drafts[j-1] = argmax of its logits (ties to the lowest index), j = 1..gamma-1.
-// logits (optional): [(gamma-1), vocab], margin (optional): top1 - top2 per row.
+// a4..a6: one draft layer l on the block's hidden states x [gamma][H], in place.
+// Block position j sits at absolute position len + j.  Every block query sees
+// the whole committed context [0, len) of layer l (k_cache/v_cache, this
+// oracle's [L][nkv][cap][d] layout) and every block position (no mask).  The
+// block's own K/V are used for this pass only and are not written to the cache.
+//   h = R(RMSNorm(x) * g_in);  q = R(RoPE(h . Wq^T)), k = R(RoPE(h . Wk^T)), v = R(h . Wv^T)
+//   o = R(attention(q, [context K; k], [context V; v]))  (bf16 P when storage is bf16)
+//   x = R(x + o . Wo^T);  h2 = R(RMSNorm(x) * g_post)
+//   m = R(silu(h2 . Wg^T) * (h2 . Wu^T));  x = R(x + m . Wd^T)
 // ---------------------------------------------------------------------------
-void oracle_draft_block(const oracle_config* c, const oracle_weights* w,
+void oracle_draft_layer(const oracle_config* c, const oracle_weights* w, int l,
                         const double* k_cache, const double* v_cache, int cap, int len,
-                        int anchor, int gamma, int* drafts, double* logits, double* margin) {
+                        int gamma, double* x) {
     g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
-    int Nq = nq * d, Nkv = nkv * d, I = c->intermediate, V = c->vocab;
+    int Nq = nq * d, Nkv = nkv * d, I = c->intermediate;
     int n = len + gamma;
-
-    // a3: embedding of [anchor, mask, ..., mask] (exact copies of table rows).
-    std::vector<double> x((size_t)gamma * H);
-    for (int j = 0; j < gamma; ++j) {
-        int tok = (j == 0) ? anchor : c->mask_id;
-        for (int t = 0; t < H; ++t) x[(size_t)j * H + t] = load(w->embed, (long)tok * H + t, S);
-    }
-
     std::vector<double> g(H), h((size_t)gamma * H), tmp(H);
     std::vector<double> q((size_t)gamma * Nq), kb((size_t)gamma * Nkv), vb((size_t)gamma * Nkv);
     std::vector<double> K((size_t)nkv * n * d), Vv((size_t)nkv * n * d), o((size_t)gamma * Nq);
     std::vector<double> y((size_t)gamma * H);
     std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I);
+    size_t xs = (size_t)gamma * H;
 
-    for (int l = 0; l < c->n_layers; ++l) {
-        // a4: h = R(RMSNorm(x) * g_in); q, k with RoPE at len + j; v.
-        load_vec(w->g_in[l], H, S, g.data());
-        for (int j = 0; j < gamma; ++j) {
-            oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
-            for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
-        }
-        linear(h.data(), gamma, H, w->wq[l], Nq, S, q.data());
-        linear(h.data(), gamma, H, w->wk[l], Nkv, S, kb.data());
-        linear(h.data(), gamma, H, w->wv[l], Nkv, S, vb.data());
-        for (int j = 0; j < gamma; ++j) {
-            long p = (long)len + j;
-            for (int hq = 0; hq < nq; ++hq) oracle_rope(q.data() + (size_t)j * Nq + (size_t)hq * d, d, p, c->rope_theta);
-            for (int g2 = 0; g2 < nkv; ++g2) oracle_rope(kb.data() + (size_t)j * Nkv + (size_t)g2 * d, d, p, c->rope_theta);
-        }
-        for (auto& e : q) e = R(e, S);
-        for (auto& e : kb) e = R(e, S);
-        for (auto& e : vb) e = R(e, S);
-
-        // a5: keys/values = injected context rows [0, len) then the block rows.
-        for (int g2 = 0; g2 < nkv; ++g2) {
-            for (int i = 0; i < len; ++i)
-                for (int t = 0; t < d; ++t) {
-                    size_t src = (((size_t)l * nkv + g2) * cap + i) * d + t;
-                    K[((size_t)g2 * n + i) * d + t] = k_cache[src];
-                    Vv[((size_t)g2 * n + i) * d + t] = v_cache[src];
-                }
-            for (int j = 0; j < gamma; ++j)
-                for (int t = 0; t < d; ++t) {
-                    K[((size_t)g2 * n + len + j) * d + t] = kb[(size_t)j * Nkv + (size_t)g2 * d + t];
-                    Vv[((size_t)g2 * n + len + j) * d + t] = vb[(size_t)j * Nkv + (size_t)g2 * d + t];
-                }
-        }
-        oracle_attention(q.data(), gamma, nq, K.data(), Vv.data(), n, nkv, d, S == 1, o.data());
-        for (auto& e : o) e = R(e, S);
-
-        // a6: x = R(x + o.Wo^T); h2 = R(RMSNorm(x) * g_post);
-        //     m = R(silu(h2.Wg^T) * (h2.Wu^T)); x = R(x + m.Wd^T)
-        linear(o.data(), gamma, Nq, w->wo[l], H, S, y.data());
-        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
-        load_vec(w->g_post[l], H, S, g.data());
-        for (int j = 0; j < gamma; ++j) {
-            oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
-            for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
-        }
-        linear(h.data(), gamma, H, w->w_gate[l], I, S, gt.data());
-        linear(h.data(), gamma, H, w->w_up[l], I, S, up.data());
-        for (size_t i = 0; i < mm.size(); ++i) {
-            double a = gt[i];
-            double silu = a / (1.0 + std::exp(-a));
-            mm[i] = R(silu * up[i], S);
-        }
-        linear(mm.data(), gamma, I, w->w_down[l], H, S, y.data());
-        for (size_t i = 0; i < x.size(); ++i) x[i] = R(x[i] + y[i], S);
+    // a4: h = R(RMSNorm(x) * g_in); q, k with RoPE at len + j; v.
+    load_vec(w->g_in[l], H, S, g.data());
+    for (int j = 0; j < gamma; ++j) {
+        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
     }
-
-    // a7: final norm of the mask positions, shared LM head, argmax.
-    int nd = gamma - 1;
-    if (nd <= 0) return;
-    load_vec(w->g_final, H, S, g.data());
-    std::vector<double> hf((size_t)nd * H);
-    for (int j = 1; j < gamma; ++j) {
-        oracle_rmsnorm(x.data() + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
-        for (int t = 0; t < H; ++t) hf[(size_t)(j - 1) * H + t] = R(tmp[t], S);
+    linear(h.data(), gamma, H, w->wq[l], Nq, S, q.data());
+    linear(h.data(), gamma, H, w->wk[l], Nkv, S, kb.data());
+    linear(h.data(), gamma, H, w->wv[l], Nkv, S, vb.data());
+    for (int j = 0; j < gamma; ++j) {
+        long p = (long)len + j;
+        for (int hq = 0; hq < nq; ++hq) oracle_rope(q.data() + (size_t)j * Nq + (size_t)hq * d, d, p, c->rope_theta);
+        for (int g2 = 0; g2 < nkv; ++g2) oracle_rope(kb.data() + (size_t)j * Nkv + (size_t)g2 * d, d, p, c->rope_theta);
     }
-    std::vector<double> lg((size_t)nd * V);
-    linear(hf.data(), nd, H, w->lm_head, V, S, lg.data());
-    for (int r = 0; r < nd; ++r) {
+    for (auto& e : q) e = R(e, S);
+    for (auto& e : kb) e = R(e, S);
+    for (auto& e : vb) e = R(e, S);
+
+    // a5: keys/values = injected context rows [0, len) then the block rows.
+    for (int g2 = 0; g2 < nkv; ++g2) {
+        for (int i = 0; i < len; ++i)
+            for (int t = 0; t < d; ++t) {
+                size_t src = (((size_t)l * nkv + g2) * cap + i) * d + t;
+                K[((size_t)g2 * n + i) * d + t] = k_cache[src];
+                Vv[((size_t)g2 * n + i) * d + t] = v_cache[src];
+            }
+        for (int j = 0; j < gamma; ++j)
+            for (int t = 0; t < d; ++t) {
+                K[((size_t)g2 * n + len + j) * d + t] = kb[(size_t)j * Nkv + (size_t)g2 * d + t];
+                Vv[((size_t)g2 * n + len + j) * d + t] = vb[(size_t)j * Nkv + (size_t)g2 * d + t];
+            }
+    }
+    oracle_attention(q.data(), gamma, nq, K.data(), Vv.data(), n, nkv, d, S == 1, o.data());
+    for (auto& e : o) e = R(e, S);
+
+    // a6: x = R(x + o.Wo^T); h2 = R(RMSNorm(x) * g_post);
+    //     m = R(silu(h2.Wg^T) * (h2.Wu^T)); x = R(x + m.Wd^T)
+    linear(o.data(), gamma, Nq, w->wo[l], H, S, y.data());
+    for (size_t i = 0; i < xs; ++i) x[i] = R(x[i] + y[i], S);
+    load_vec(w->g_post[l], H, S, g.data());
+    for (int j = 0; j < gamma; ++j) {
+        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
+    }
+    linear(h.data(), gamma, H, w->w_gate[l], I, S, gt.data());
+    linear(h.data(), gamma, H, w->w_up[l], I, S, up.data());
+    for (size_t i = 0; i < mm.size(); ++i) {
+        double a = gt[i];
+        double silu = a / (1.0 + std::exp(-a));
+        mm[i] = R(silu * up[i], S);
+    }
+    linear(mm.data(), gamma, I, w->w_down[l], H, S, y.data());
+    for (size_t i = 0; i < xs; ++i) x[i] = R(x[i] + y[i], S);
+}
+
+// a7 (second half): the shared LM head and argmax on already-normalised rows
+// hf [rows][H]: logits = hf . lm_head^T (not rounded), drafts[r] = argmax
+// (ties to the lowest index), margin[r] = top-1 minus top-2 logit.
+// logits (optional): [rows][vocab]; margin (optional).
+void oracle_lm_head(const oracle_config* c, const oracle_weights* w, const double* hf, int rows,
+                    int* drafts, double* logits, double* margin) {
+    g_acc32 = c->acc32;
+    int S = c->storage, H = c->hidden, V = c->vocab;
+    if (rows <= 0) return;
+    std::vector<double> lg((size_t)rows * V);
+    linear(hf, rows, H, w->lm_head, V, S, lg.data());
+    for (int r = 0; r < rows; ++r) {
         const double* row = lg.data() + (size_t)r * V;
         int best = 0;
         for (int vv = 1; vv < V; ++vv) if (row[vv] > row[best]) best = vv;
@@ -489,6 +497,52 @@ void oracle_draft_block(const oracle_config* c, const oracle_weights* w,
         if (margin) margin[r] = (V > 1) ? row[best] - second : INFINITY;
     }
     if (logits) std::memcpy(logits, lg.data(), sizeof(double) * lg.size());
+}
+
+// a7 (first half): the final norm of the mask positions j = 1..gamma-1 of the
+// block's last hidden states x [gamma][H]: hf[j-1] = R(RMSNorm(x_j) * g_final).
+void oracle_final_norm(const oracle_config* c, const oracle_weights* w, const double* x, int gamma,
+                       double* hf) {
+    int S = c->storage, H = c->hidden;
+    std::vector<double> g(H), tmp(H);
+    load_vec(w->g_final, H, S, g.data());
+    for (int j = 1; j < gamma; ++j) {
+        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) hf[(size_t)(j - 1) * H + t] = R(tmp[t], S);
+    }
+}
+
+// a3: embedding of [anchor, mask, ..., mask] (exact copies of table rows) into x [gamma][H].
+void oracle_embed_block(const oracle_config* c, const oracle_weights* w, int anchor, int gamma, double* x) {
+    int S = c->storage, H = c->hidden;
+    for (int j = 0; j < gamma; ++j) {
+        int tok = (j == 0) ? anchor : c->mask_id;
+        for (int t = 0; t < H; ++t) x[(size_t)j * H + t] = load(w->embed, (long)tok * H + t, S);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3..a7: draft one block of gamma positions in one forward pass: the embedding
+// (position 0 holds the clean anchor token, positions 1..gamma-1 the mask
+// token), every draft layer once (oracle_draft_layer), then the final norm and
+// the shared LM head.  Mask position j predicts the token at len + j:
+// drafts[j-1] = argmax of its logits (ties to the lowest index), j = 1..gamma-1.
+// logits (optional): [(gamma-1), vocab], margin (optional): top1 - top2 per row.
+// ---------------------------------------------------------------------------
+void oracle_draft_block(const oracle_config* c, const oracle_weights* w,
+                        const double* k_cache, const double* v_cache, int cap, int len,
+                        int anchor, int gamma, int* drafts, double* logits, double* margin) {
+    g_acc32 = c->acc32;
+    int H = c->hidden;
+    std::vector<double> x((size_t)gamma * H);
+    oracle_embed_block(c, w, anchor, gamma, x.data());
+    for (int l = 0; l < c->n_layers; ++l)
+        oracle_draft_layer(c, w, l, k_cache, v_cache, cap, len, gamma, x.data());
+    int nd = gamma - 1;
+    if (nd <= 0) return;
+    std::vector<double> hf((size_t)nd * H);
+    oracle_final_norm(c, w, x.data(), gamma, hf.data());
+    oracle_lm_head(c, w, hf.data(), nd, drafts, logits, margin);
 }
 
 // ---------------------------------------------------------------------------

@@ -47,6 +47,8 @@ def lib():
         L.oracle_rmsnorm.argtypes = [dp, dp, C.c_int, C.c_double, dp]
         L.oracle_rope.argtypes = [dp, C.c_int, C.c_long, C.c_double]
         L.oracle_attention.argtypes = [dp, C.c_int, C.c_int, dp, dp, C.c_int, C.c_int, C.c_int, C.c_int, dp]
+        L.oracle_attention_block.argtypes = [dp, C.c_int, C.c_int, dp, dp, C.c_int, C.c_int, C.c_int, C.c_int,
+                                             dp, dp, dp]
         L.oracle_layer_ids.argtypes = [C.c_int, C.c_int, ip]
         L.oracle_loss_weights.argtypes = [C.c_int, dp]
         L.oracle_fuse_context.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.POINTER(C.c_void_p),
@@ -56,6 +58,11 @@ def lib():
                                                 C.c_int]
         L.oracle_draft_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, dp, C.c_int, C.c_int,
                                          C.c_int, C.c_int, ip, dp, dp]
+        L.oracle_draft_layer.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, C.c_int,
+                                         C.c_int, dp]
+        L.oracle_embed_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, C.c_int, dp]
+        L.oracle_final_norm.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, dp]
+        L.oracle_lm_head.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, ip, dp, dp]
         L.oracle_accept.restype = C.c_int
         L.oracle_accept.argtypes = [C.c_int, C.c_int, ip, ip, ip, ip, ip, ip]
         L.oracle_num_threads.restype = C.c_int
@@ -112,6 +119,23 @@ def attention(q, k, v, round_p: bool = False) -> np.ndarray:
     o = np.empty_like(q)
     lib().oracle_attention(_dp(q), nrow, nq, _dp(k), _dp(v), n, nkv, d, int(round_p), _dp(o))
     return o
+
+
+def attention_block(q, k, v, round_p: bool = False):
+    """Unnormalised attention over one block of keys: q [nrow, nq, d]; k, v
+    [nkv, n, d] -> (num [nrow, nq, d], z [nrow, nq], base [nrow, nq]) with
+    o = num / z and base the block's integer base-2 shift."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    nrow, nq, d = q.shape
+    nkv, n, _ = k.shape
+    num = np.empty_like(q)
+    z = np.empty((nrow, nq), dtype=np.float64)
+    base = np.empty((nrow, nq), dtype=np.float64)
+    lib().oracle_attention_block(_dp(q), nrow, nq, _dp(k), _dp(v), n, nkv, d, int(round_p), _dp(num), _dp(z),
+                                 _dp(base))
+    return num, z, base
 
 
 def layer_ids(n_target_layers: int, n_sel: int) -> List[int]:
@@ -215,6 +239,44 @@ class OracleDrafter:
                                  cache["cap"], cache["len"], int(anchor), int(gamma), _ip(drafts),
                                  _dp(logits) if logits is not None else None, _dp(margin))
         return drafts[:nd], margin[:nd], (logits[:nd] if logits is not None else None)
+
+    # -- the draft step one piece at a time (call-local parity: each piece can
+    #    be fed the GPU's own inputs) ----------------------------------------
+    def embed_block(self, anchor: int, gamma: int) -> np.ndarray:
+        x = np.empty((gamma, self.shape["hidden"]), dtype=np.float64)
+        lib().oracle_embed_block(C.byref(self.cfg), C.byref(self.w), int(anchor), int(gamma), _dp(x))
+        return x
+
+    def draft_layer(self, cache: Dict, layer: int, x: np.ndarray) -> np.ndarray:
+        """Layer `layer` on the block's hidden states x [gamma, hidden] over the
+        cache's committed context; returns the layer's output (x is not changed)."""
+        y = np.array(x, dtype=np.float64, copy=True, order="C")
+        gamma = y.shape[0]
+        if cache["len"] + gamma > cache["cap"]:
+            raise ValueError("capacity")
+        lib().oracle_draft_layer(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(cache["k"]), _dp(cache["v"]),
+                                 cache["cap"], cache["len"], gamma, _dp(y))
+        return y
+
+    def final_norm(self, x: np.ndarray) -> np.ndarray:
+        """hf rows of the mask positions 1..gamma-1 of x [gamma, hidden]."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        gamma = x.shape[0]
+        hf = np.empty((max(gamma - 1, 1), self.shape["hidden"]), dtype=np.float64)
+        lib().oracle_final_norm(C.byref(self.cfg), C.byref(self.w), _dp(x), gamma, _dp(hf))
+        return hf[:gamma - 1]
+
+    def lm_head(self, hf: np.ndarray):
+        """Shared LM head + argmax on normalised rows hf [rows, hidden] ->
+        (drafts [rows] int32, margin [rows], logits [rows, vocab])."""
+        hf = np.ascontiguousarray(hf, dtype=np.float64)
+        rows = hf.shape[0]
+        drafts = np.zeros(max(rows, 1), dtype=np.int32)
+        margin = np.zeros(max(rows, 1), dtype=np.float64)
+        logits = np.zeros((max(rows, 1), self.shape["vocab"]), dtype=np.float64)
+        lib().oracle_lm_head(C.byref(self.cfg), C.byref(self.w), _dp(hf), rows, _ip(drafts), _dp(logits),
+                             _dp(margin))
+        return drafts[:rows], margin[:rows], logits[:rows]
 
     def accept(self, cache: Dict, drafts, target) -> tuple:
         """Returns (status, accept_len, next_anchor) and updates cache lengths."""

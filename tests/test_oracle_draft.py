@@ -287,3 +287,20 @@ def test_argmax_ties_go_to_lowest_index():
     assert logits[0][5] == logits[0][11] == logits[0][15] > 0
     assert list(drafts) == [5, 5]
     assert np.all(margin == 0.0)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_piecewise_draft_equals_one_call(dtype):
+    # embed -> every layer -> final norm -> LM head, called one piece at a time
+    # (the form the call-local GPU parity tests feed the GPU's own inputs to),
+    # reproduces the one-call draft bit for bit
+    w = micro(dtype)
+    W = I.make_weights(w)
+    hid = I.make_hiddens(w, 20)
+    od, ctx, cache, drafts, margin, logits = _run_oracle(w, W, hid, 5, 11)
+    x = od.embed_block(11, 5)
+    for l in range(w.n_layers):
+        x = od.draft_layer(cache, l, x)
+    hf = od.final_norm(x)
+    d2, m2, l2 = od.lm_head(hf)
+    assert np.array_equal(d2, drafts) and np.array_equal(m2, margin) and np.array_equal(l2, logits)
