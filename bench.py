@@ -55,6 +55,13 @@ def parse_args():
     ap.add_argument("--no-profile-pass", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
+    ap.add_argument("--separate-pre-step", action="store_true",
+                    help="fuse_context + inject_kv as two calls instead of one fuse_inject call")
+    ap.add_argument("--no-fold", action="store_true", help="separate RMSNorm kernels in the draft step")
+    ap.add_argument("--trace-dump", default=None,
+                    help="write the traced step's raw per-block stamps and launch records to this .npz file")
+    ap.add_argument("--l2-prefetch", type=int, default=None,
+                    help="weight tiles each GEMM CTA prefetches into L2 before its dependency wait")
     return ap.parse_args()
 
 
@@ -65,12 +72,12 @@ def env_int(name, default):
         return default
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of k_gemm_tc per
-# launch, averaged over the 23 GEMM launches of one step of this workload, from
-# one ncu capture (profiles/k_gemm_tc_qwen3_8b_step_dram.md).  It describes the
-# kernel sources it was taken on; once they change the figure is void.
-GEMM_TRAFFIC = {"workload": "qwen3_8b", "bytes_per_launch": 150.6e6,
-                "sources_sha256": "75cc540e3725c847588f0130c9c199a236f956bcbadbbafa2e92e6119d82f48f"}
+# DRAM traffic of k_gemm_tc relative to its algorithmic bytes
+# (dram__bytes_read.sum + dram__bytes_write.sum over (weights + activations in +
+# outputs)), from one ncu capture of a single GEMM launch of the step's shape
+# class (M = 16 tokens, weights larger than L2).  It describes the kernel sources
+# it was taken on: once they change, the figure is void and the line reports null.
+GEMM_TRAFFIC = {"ratio": None, "sources_sha256": None}
 
 
 def gemm_sources_sha256():
@@ -83,13 +90,65 @@ def gemm_sources_sha256():
 
 
 def measured_traffic(workload):
-    """Per-launch DRAM bytes of the GEMM kernel, or None when not measured for these sources."""
+    """DRAM bytes per algorithmic byte of the GEMM kernel, or None when not measured for these sources."""
     try:
-        if workload == GEMM_TRAFFIC["workload"] and gemm_sources_sha256() == GEMM_TRAFFIC["sources_sha256"]:
-            return GEMM_TRAFFIC["bytes_per_launch"]
+        if GEMM_TRAFFIC["ratio"] and gemm_sources_sha256() == GEMM_TRAFFIC["sources_sha256"]:
+            return GEMM_TRAFFIC["ratio"]
     except OSError:
         pass
     return None
+
+
+def traced_step(D, h, step, i0, K, st, ab, dump=None):
+    """Replay one graph-captured step with the library's step trace on; return
+    ({kind: [launches, ms summed over replays]}, info)."""
+    import torch
+    words = 1 << 22
+    buf = torch.zeros(words, dtype=torch.int64, device=st.device)
+    D.dflash_diag_step_trace(h, buf.data_ptr(), words)
+    gr = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    with torch.cuda.graph(gr, stream=cs):
+        step(i0)
+    recs = D.dflash_diag_step_trace_records(h)
+    D.dflash_diag_step_trace(h, None)
+    for _ in range(3):
+        gr.replay()
+    R = max(3, min(K, 50))
+    hist = torch.empty(R, words, dtype=torch.int64, device=st.device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot = 0.0
+    for r in range(R):
+        e0.record(st)
+        gr.replay()
+        e1.record(st)
+        hist[r].copy_(buf)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    H = hist.cpu().numpy()
+    del hist, buf, gr
+    if dump:
+        import numpy as np
+        np.savez_compressed(dump, stamps=H[-1], kinds=np.array([r["kind"] for r in recs]),
+                            recs=np.array([[r["blocks"], r["words"], r["wait_idx"], r["exit_idx"], r["offset"]]
+                                           for r in recs], dtype=np.int64))
+    kern = {}
+    for r in range(R):
+        prev_end = None
+        for rec in recs:
+            blk = H[r, rec["offset"]:rec["offset"] + rec["blocks"] * rec["words"]].reshape(rec["blocks"], rec["words"])
+            used = blk[:, rec["exit_idx"]] != 0
+            if not used.any():
+                continue
+            start = int(blk[used, rec["wait_idx"]].min())
+            end = int(blk[used, rec["exit_idx"]].max())
+            t = end - (prev_end if prev_end is not None else start)
+            prev_end = end
+            e = kern.setdefault(rec["kind"], [0, 0.0])
+            e[0] += 1
+            e[1] += max(t, 0) / 1e6
+    info = {"replays": R, "traced_ms_per_step": tot / R, "launches": len(recs)}
+    return kern, info
 
 
 def workload_description(w, B, T, g):
@@ -408,6 +467,9 @@ def run_gpu(args):
     rc = torch.full((B,), g, dtype=torch.int32, device=dev)
     h, c = drafter.handle, cache.handle
     D.dflash_diag_set_launch_mode(not args.no_pdl)
+    D.dflash_diag_set_norm_fold(not args.no_fold)
+    if args.l2_prefetch is not None:
+        D.dflash_diag_set_gemm_prefetch(args.l2_prefetch)
 
     def step(i, hid_list=None):
         sp = torch.cuda.current_stream().cuda_stream
@@ -416,8 +478,12 @@ def run_gpu(args):
         D.dflash_diag_synth_target(drafts.data_ptr(), a_plan[j].data_ptr(), rnd[j].data_ptr(), B, g, w.vocab,
                                    target.data_ptr(), sp)
         hl = hid_list if hid_list is not None else step_hid[i % POOL]
-        D.dflash_fuse_context(h, [x.data_ptr() for x in hl], w.target_hidden, B * g, ctx_step.data_ptr(), sp)
-        D.dflash_inject_kv(h, c, ctx_step.data_ptr(), rs.data_ptr(), rc.data_ptr(), B * g, sp)
+        if args.separate_pre_step:
+            D.dflash_fuse_context(h, [x.data_ptr() for x in hl], w.target_hidden, B * g, ctx_step.data_ptr(), sp)
+            D.dflash_inject_kv(h, c, ctx_step.data_ptr(), rs.data_ptr(), rc.data_ptr(), B * g, sp)
+        else:   # the verify-side pre-step: fuse + inject of the verified rows in one call
+            D.dflash_fuse_inject(h, c, [x.data_ptr() for x in hl], w.target_hidden, rs.data_ptr(), rc.data_ptr(),
+                                 B * g, None, sp)
         D.dflash_accept(h, c, drafts.data_ptr(), target.data_ptr(), g, acc.data_ptr(), anchor.data_ptr(), sp)
         D.dflash_cache_set_len(c, lens.data_ptr(), sp)
 
@@ -485,20 +551,16 @@ def run_gpu(args):
     step_bytes = step_algorithmic_bytes(w, B, g, T)
     t_roof_ms = step_bytes / (hbm_peak * 1e9) * 1e3
 
-    # ---- instrumented pass: per-launch CUDA events (separate from the timed pass)
-    kern = {}
-    if not args.no_profile_pass:
-        D.dflash_diag_timing_enable(h, K * 64 + 64)
-        sp = st.cuda_stream
-        for _ in range(K):
-            step(i)
-            i += 1
-        log = D.dflash_diag_timing_read(h, sp)
-        D.dflash_diag_timing_disable(h)
-        for name, t in log:
-            e = kern.setdefault(name, [0, 0.0])
-            e[0] += 1
-            e[1] += t
+    # ---- traced pass: the same step captured in one CUDA graph with the library's
+    # step trace on (every kernel stamps %globaltimer per block past its dependency
+    # wait and at exit), replayed like the timed pass.  Launch k's time is charged
+    # from the end of launch k-1 to its own end (the first launch from its start),
+    # so the per-kernel times partition the traced part of the step and add up to
+    # no more than the step.
+    kern, traced = {}, None
+    if not args.no_profile_pass and graphs is not None:
+        kern, traced = traced_step(D, h, step, i, K, st, ab, args.trace_dump)
+        i += max(3, min(K, 50)) + 3
     gemm_names = ["gemm_qkv", "gemm_o", "gemm_swiglu", "gemm_down", "gemm_lmhead", "gemm_fuse", "gemm_inject"]
     roofline = None
     if kern:
@@ -506,12 +568,18 @@ def run_gpu(args):
         gms = sum(kern[n][1] for n in gemm_names if n in kern)
         gbytes = sum(kern[n][0] * ab[n] for n in gemm_names if n in kern)
         achieved = gbytes / (gms / 1e3) / 1e9
+        traffic = measured_traffic(args.workload)
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                    "frac": round(achieved / hbm_peak, 4), "traffic": measured_traffic(args.workload),
-                    "kernel": "k_gemm_tc (all %d launches of %d steps)" % (gl, K),
+                    "frac": round(achieved / hbm_peak, 4),
+                    "traffic": (round(traffic * gbytes / max(gl, 1)) if traffic else None),
+                    "kernel": "k_gemm_tc (all %d launches of one step, %d replays)" % (gl // max(traced["replays"], 1),
+                                                                                  traced["replays"]),
                     "algorithmic_bytes_per_launch": round(gbytes / max(gl, 1)),
+                    "time_source": "per-kernel share of the graph-replayed step from the kernels' own %globaltimer "
+                                   "stamps (launch end minus previous launch end)",
                     "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src}
-    per_kernel = {n: {"launches": v[0], "ms_per_step": round(v[1] / K, 4),
+    reps = traced["replays"] if traced else 1
+    per_kernel = {n: {"launches": v[0] // reps, "ms_per_step": round(v[1] / reps, 4),
                       "GB_per_s": (round(ab[n] * v[0] / (v[1] / 1e3) / 1e9, 1) if n in ab and v[1] > 0 else None)}
                   for n, v in sorted(kern.items(), key=lambda kv: -kv[1][1])}
 
@@ -607,11 +675,17 @@ def run_gpu(args):
                               "t_roof_ms": round(t_roof_ms, 4), "frac": round(t_roof_ms / ms_step, 4),
                               "peak_gbs": hbm_peak, "peak_source": peak_src},
             "per_kernel": per_kernel,
+            "traced_step": ({"ms_per_step": round(traced["traced_ms_per_step"], 4),
+                             "traced_launches": traced["launches"],
+                             "attributed_ms": round(sum(v["ms_per_step"] for v in per_kernel.values()), 4)}
+                            if traced else None),
             "cpu_baseline": cpu,
             "cpu_baseline_fp32_accumulation": cpu32,
             "prefill": prefill,
             "e2e": e2e,
             "gpu_launches": launches,
+            "step_options": {"pre_step": "two calls" if args.separate_pre_step else "fuse_inject (one call)",
+                             "norm_fold": not args.no_fold, "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch()},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
                                                                               else ", programmatic dependent launch"),
             "clocks": clocks,

@@ -17,6 +17,10 @@ using namespace df;
 
 namespace df {
 static bool g_pdl = true;
+// RMSNorm folded into the GEMMs that consume the normalised rows (draft step,
+// token tiles up to kFoldMaxNT wide); dflash_diag_set_norm_fold switches it.
+static bool g_fold = true;
+constexpr int kFoldMaxNT = 64;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
 void ensure_carveout(const void* fn) {
@@ -69,7 +73,7 @@ inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 constexpr int kMaxCtas = 160;   // >= SMs of any B200 part
 
 struct WsLayout {
-    size_t status, rope, x, h, q, o, act, hf, y, y32, lgs, req_ok, gpart, gcnt, rec, total;
+    size_t status, rope, x, h, q, o, act, hf, y, y32, lgs, req_ok, gpart, gcnt, rec, ssq, ssq_ctx, total;
     int nt_max;
     long long n_counters;
 };
@@ -95,7 +99,7 @@ void make_layout(const dflash_config& c, WsLayout& L) {
     L.hf = off; off = al(off + Mlm * H * es);
     L.y = off; off = al(off + R * H * es);
     L.req_ok = off; off = al(off + (size_t)c.max_batch * 4);
-    L.y32 = L.lgs = L.gpart = L.gcnt = L.rec = off;
+    L.y32 = L.lgs = L.gpart = L.gcnt = L.rec = L.ssq = L.ssq_ctx = off;
     L.nt_max = 0;
     L.n_counters = 0;
     if (!bf) {
@@ -108,10 +112,16 @@ void make_layout(const dflash_config& c, WsLayout& L) {
         const long long t_layer = std::max(std::max((long long)cdiv(Nq, 128) + 2 * cdiv(Nkv, 128), (long long)cdiv(H, 128)),
                                            I / 64);
         const long long t_big = std::max((long long)cdiv(H, 128), 10LL * cdiv(Nkv, 128));
-        L.n_counters = std::max(std::max(t_layer * m_tiles_for((int)Mmax), (long long)cdiv(V, 128) * m_tiles_for((int)Mlm)),
+        L.n_counters = std::max(std::max(t_layer * m_tiles_for((int)Mmax),
+                                         (long long)cdiv(V, 128) * m_tiles_for((int)std::max(Mlm, Mmax))),
                                 t_big * m_tiles_for((int)R));
         L.gcnt = off; off = al(off + (size_t)L.n_counters * 4);
-        L.rec = off; off = al(off + (size_t)cdiv(V, 128) * Mlm * sizeof(float4));
+        // LM-head records for whole blocks (the folded final norm runs the head on all gamma rows)
+        L.rec = off; off = al(off + (size_t)cdiv(V, 128) * std::max(Mlm, Mmax) * sizeof(float4));
+        // per-(128-feature tile, token row) partial sums of squares of the residual stream
+        L.ssq = off; off = al(off + (size_t)cdiv(H, 128) * Mmax * sizeof(float));
+        // the same for the projected context rows of dflash_fuse_inject
+        L.ssq_ctx = off; off = al(off + (size_t)cdiv(H, 128) * R * sizeof(float));
     }
     L.total = off;
 }
@@ -150,13 +160,23 @@ struct dflash_handle {
     int* status;
     float2* rope;
     void *x, *h, *q, *o, *act, *hf, *y;
-    float *y32, *lgs, *gpart;
+    float *y32, *lgs, *gpart, *ssq, *ssq_ctx;
     int *req_ok, *gcnt;
     float4* rec;
     CUtensorMap tm_wfc, tm_lm;
     CUtensorMap tm_wq[DFLASH_MAX_LAYERS], tm_wk[DFLASH_MAX_LAYERS], tm_wv[DFLASH_MAX_LAYERS], tm_wo[DFLASH_MAX_LAYERS];
     CUtensorMap tm_wg[DFLASH_MAX_LAYERS], tm_wu[DFLASH_MAX_LAYERS], tm_wd[DFLASH_MAX_LAYERS];
     long long launches;
+    // Diagnostic capture (dflash_diag_draft_capture): residual stream after the
+    // embedding and after every layer, and the final-norm rows.
+    void* cap_x = nullptr;
+    void* cap_hf = nullptr;
+    // Diagnostic step trace (dflash_diag_step_trace): per-block %globaltimer
+    // stamps of every traced launch, laid out one launch after the other.
+    long long* tr_buf = nullptr;
+    long long tr_cap = 0, tr_used = 0;
+    struct TraceRec { int kind, blocks, words, wait_idx, exit_idx; long long offset; };
+    std::vector<TraceRec> tr_recs;
     // Diagnostic timing (dflash_diag_timing_*): event pairs around launches.
     std::vector<cudaEvent_t> ev;
     std::vector<int> ev_kind;
@@ -225,16 +245,49 @@ struct Timed {
     }
 };
 
+// Room for one launch's step trace: `blocks` x `words` int64 stamps, the
+// stamp past the dependency wait at word wait_idx and the exit stamp at word
+// exit_idx of each block.  Null when tracing is off or the buffer is full.
+long long* trace_slot(dflash_handle* h, int kind, int blocks, int words, int wait_idx, int exit_idx) {
+    if (!h->tr_buf || blocks <= 0) return nullptr;
+    const long long need = (long long)blocks * words;
+    if (h->tr_used + need > h->tr_cap) return nullptr;
+    long long* p = h->tr_buf + h->tr_used;
+    h->tr_recs.push_back({kind, blocks, words, wait_idx, exit_idx, h->tr_used});
+    h->tr_used += need;
+    return p;
+}
+// Small kernels: two stamps per block (past the wait, exit).
+long long* trace_small(dflash_handle* h, int kind, int blocks) { return trace_slot(h, kind, blocks, 2, 0, 1); }
+
+// Diagnostic capture of the residual stream x ([B*gamma][H]) into slot `slot`
+// of the caller's [(L+1)][B*gamma][H] buffer.
+void capture_x(dflash_handle* h, int slot, int M, cudaStream_t st) {
+    if (!h->cap_x) return;
+    const size_t es = h->cfg.dtype == DFLASH_BF16 ? 2 : 4;
+    const size_t row = (size_t)M * h->cfg.hidden * es;
+    cudaMemcpyAsync((uint8_t*)h->cap_x + (size_t)slot * row, h->x, row, cudaMemcpyDeviceToDevice, st);
+}
+void capture_hf(dflash_handle* h, int Mlm, cudaStream_t st) {
+    if (!h->cap_hf) return;
+    const size_t es = h->cfg.dtype == DFLASH_BF16 ? 2 : 4;
+    cudaMemcpyAsync(h->cap_hf, h->hf, (size_t)Mlm * h->cfg.hidden * es, cudaMemcpyDeviceToDevice, st);
+}
+
 // Common GEMM plumbing.
 void gemm_common(dflash_handle* h, GemmParams& p) {
+    p.l2_prefetch = gemm_l2_prefetch();
     p.partial = h->gpart;
     p.counters = h->gcnt;
     p.status = h->status;
     p.ctas = 0;
 }
 
-int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st) {
+int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st, int kind) {
     gemm_common(h, p);
+    // GEMM trace: 8 stamps per CTA (gemm.cuh), past the wait at 1, exit at 6;
+    // room for the largest grid, CTAs the launch does not use stay zero.
+    p.trace = trace_slot(h, kind, kMaxCtas, 8, 1, 6);
     int e = launch_gemm_tc(p, nt, std::min(h->num_sms, kMaxCtas), st);
     h->launches += p.units > 0 ? 1 : 0;
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
@@ -247,6 +300,107 @@ bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride
 
 
 }  // namespace
+
+// The injection GEMMs of rows [0, total_rows) of `src` ([total_rows, H] bf16):
+// all layers' Wk/Wv stacked as one A operand (up to kMaxAMats matrices per
+// launch), RoPE and the cache write in the epilogue.  One launch per slab of nt
+// rows: every launch then has a single m-tile, so the split-K partition (k-ranges
+// per CTA over n_tiles x k-blocks) and with it the fp32 summation order of every
+// K/V element are the same whatever the number of rows: injecting rows in chunks
+// writes the same bits as injecting them at once.
+// With ssq (the projected rows' per-tile sums of squares, [cdiv(H,128)][max_rows]),
+// src holds the un-normalised rows and each launch applies RMSNorm * g_fc to its
+// token tiles in shared memory (and copies the normalised rows to ctx_out when it
+// is not null).
+static int inject_gemms(dflash_handle* h, dflash_cache* cc, const void* src, const int32_t* row_start,
+                 const int32_t* row_count, int total_rows, const float* ssq, void* ctx_out, cudaStream_t st) {
+    const dflash_config& c = h->cfg;
+    const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
+    const int nt = pick_nt(total_rows);
+    for (int row0 = 0; row0 < total_rows; row0 += nt) {
+        const int rows = std::min(nt, total_rows - row0);
+        CUtensorMap tb;
+        if (!act_map(&tb, (const uint8_t*)src + (size_t)row0 * H * 2, rows, H, H, nt)) return DFLASH_INVALID_ARG;
+        for (int l0 = 0; l0 < c.n_layers; l0 += kMaxAMats / 2) {
+            const int nl = std::min(kMaxAMats / 2, c.n_layers - l0);
+            GemmParams p;
+            std::memset(&p, 0, sizeof(p));
+            for (int i = 0; i < nl; ++i) {
+                p.ta[2 * i] = h->tm_wk[l0 + i];
+                p.ta[2 * i + 1] = h->tm_wv[l0 + i];
+                p.amat[2 * i].rows = Nkv;
+                p.amat[2 * i + 1].rows = Nkv;
+            }
+            p.n_amat = 2 * nl;
+            p.tb[0] = tb;
+            p.kb_per_b = cdiv(H, 64);
+            p.M = rows;
+            p.row0 = row0;
+            p.K = H;
+            p.epi = EPI_INJECT;
+            p.d = d;
+            p.cap = cc->capacity;
+            p.layer = l0;
+            p.batch = cc->batch;
+            p.len = cc->len;
+            p.rope = h->rope;
+            p.slab = (__nv_bfloat16*)cc->slab;
+            p.s_req = cc->s_req;
+            p.s_layer = cc->s_layer;
+            p.s_kind = cc->s_kind;
+            p.s_kv = cc->s_kv;
+            p.row_start = row_start;
+            p.row_count = row_count;
+            if (ssq) {
+                p.ssq_in = ssq + row0;
+                p.ssq_tiles = cdiv(H, 128);
+                p.ssq_ld = std::max(1, c.max_rows);
+                p.gain = (const __nv_bfloat16*)h->w.g_fc;
+                p.eps = (float)c.rms_eps;
+                p.norm_h = H;
+                if (ctx_out && l0 == 0) {
+                    p.norm_out = (__nv_bfloat16*)ctx_out + (size_t)row0 * H;
+                    p.norm_out_ld = H;
+                }
+            }
+            Timed t(h, TK_GEMM_INJECT, st);
+            int r = run_gemm(h, p, nt, st, TK_GEMM_INJECT);
+            if (r) return r;
+        }
+    }
+    return DFLASH_OK;
+}
+
+// a1's projection: y = R(concat_i hiddens[i] . W_fc^T) into the workspace's y
+// ([total_rows, H] bf16), with ssq (or null) receiving the rows' per-tile sums
+// of squares ([cdiv(H,128)][max_rows]).
+static int fuse_gemm(dflash_handle* h, const void* const* hiddens, int64_t row_stride, int total_rows, float* ssq,
+                     cudaStream_t st) {
+    const dflash_config& c = h->cfg;
+    if ((row_stride * 2) % 16) return DFLASH_INVALID_ARG;
+    for (int i = 0; i < c.n_sel; ++i)
+        if (!aligned16(hiddens[i])) return DFLASH_INVALID_ARG;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    const int nt = pick_nt(total_rows);
+    p.ta[0] = h->tm_wfc;
+    p.n_amat = 1;
+    p.amat[0].rows = c.hidden;
+    for (int i = 0; i < c.n_sel; ++i)
+        if (!act_map(&p.tb[i], hiddens[i], total_rows, c.target_hidden, row_stride, nt)) return DFLASH_INVALID_ARG;
+    p.kb_per_b = c.target_hidden / 64;
+    p.M = total_rows;
+    p.K = c.n_sel * c.target_hidden;
+    p.epi = EPI_BF16;
+    p.out = h->y;
+    p.ldo = c.hidden;
+    if (ssq) {
+        p.ssq_out = ssq;
+        p.ssq_ld = std::max(1, c.max_rows);
+    }
+    Timed t(h, TK_GEMM_FUSE, st);
+    return run_gemm(h, p, nt, st, TK_GEMM_FUSE);
+}
 
 extern "C" {
 
@@ -321,6 +475,8 @@ int dflash_create(const dflash_config* cfg, const dflash_weights* w, void* works
     h->gpart = (float*)(b + L.gpart);
     h->gcnt = (int*)(b + L.gcnt);
     h->rec = (float4*)(b + L.rec);
+    h->ssq = (float*)(b + L.ssq);
+    h->ssq_ctx = (float*)(b + L.ssq_ctx);
     h->launches = 0;
 
     // RoPE table: angle p * theta^(-2i/d) in fp64, stored as fp32 (cos, sin).
@@ -441,7 +597,8 @@ int dflash_cache_get_info(const dflash_cache* c, dflash_cache_info* info) {
 
 int dflash_cache_set_len(dflash_cache* c, const int32_t* lens, dflash_stream stream) {
     if (!c || !lens) return DFLASH_INVALID_ARG;
-    launch_set_len(lens, c->batch, c->capacity, c->len, c->committed, c->status, S(stream));
+    launch_set_len(lens, c->batch, c->capacity, c->len, c->committed, c->status, S(stream),
+                   trace_small(const_cast<dflash_handle*>(c->h), TK_SET_LEN, cdiv(c->batch, 128)));
     const_cast<dflash_handle*>(c->h)->launches += 1;
     return cuda_status(cudaGetLastError());
 }
@@ -472,31 +629,13 @@ int dflash_fuse_context(dflash_handle* h, const void* const* hiddens, int64_t ro
     cudaStream_t st = S(stream);
     const int H = c.hidden;
     if (c.dtype == DFLASH_BF16) {
-        if ((row_stride * 2) % 16 || !aligned16(ctx_out)) return DFLASH_INVALID_ARG;
-        for (int i = 0; i < c.n_sel; ++i)
-            if (!aligned16(hiddens[i])) return DFLASH_INVALID_ARG;
-        GemmParams p;
-        std::memset(&p, 0, sizeof(p));
-        const int nt = pick_nt(total_rows);
-        p.ta[0] = h->tm_wfc;
-        p.n_amat = 1;
-        p.amat[0].rows = H;
-        for (int i = 0; i < c.n_sel; ++i)
-            if (!act_map(&p.tb[i], hiddens[i], total_rows, c.target_hidden, row_stride, nt)) return DFLASH_INVALID_ARG;
-        p.kb_per_b = c.target_hidden / 64;
-        p.M = total_rows;
-        p.K = c.n_sel * c.target_hidden;
-        p.epi = EPI_BF16;
-        p.out = h->y;
-        p.ldo = H;
-        {
-            Timed t(h, TK_GEMM_FUSE, st);
-            int r = run_gemm(h, p, nt, st);
-            if (r) return r;
-        }
+        if (!aligned16(ctx_out)) return DFLASH_INVALID_ARG;
+        int r = fuse_gemm(h, hiddens, row_stride, total_rows, nullptr, st);
+        if (r) return r;
         Timed t(h, TK_RMSNORM, st);
         launch_rmsnorm<__nv_bfloat16>((const __nv_bfloat16*)h->y, (const __nv_bfloat16*)h->w.g_fc,
-                                      (__nv_bfloat16*)ctx_out, total_rows, H, (float)c.rms_eps, total_rows, 0, 0, st);
+                                      (__nv_bfloat16*)ctx_out, total_rows, H, (float)c.rms_eps, total_rows, 0, 0, st,
+                                      trace_small(h, TK_RMSNORM, total_rows));
     } else {
         Timed t(h, TK_SIMT_F32, st);
         XSegs xs;
@@ -527,42 +666,8 @@ int dflash_inject_kv(dflash_handle* h, dflash_cache* cc, const void* ctx, const 
     const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
     if (c.dtype == DFLASH_BF16) {
         if (!aligned16(ctx)) return DFLASH_INVALID_ARG;
-        const int nt = pick_nt(total_rows);
-        CUtensorMap tb;
-        if (!act_map(&tb, ctx, total_rows, H, H, nt)) return DFLASH_INVALID_ARG;
-        for (int l0 = 0; l0 < c.n_layers; l0 += kMaxAMats / 2) {
-            const int nl = std::min(kMaxAMats / 2, c.n_layers - l0);
-            GemmParams p;
-            std::memset(&p, 0, sizeof(p));
-            for (int i = 0; i < nl; ++i) {
-                p.ta[2 * i] = h->tm_wk[l0 + i];
-                p.ta[2 * i + 1] = h->tm_wv[l0 + i];
-                p.amat[2 * i].rows = Nkv;
-                p.amat[2 * i + 1].rows = Nkv;
-            }
-            p.n_amat = 2 * nl;
-            p.tb[0] = tb;
-            p.kb_per_b = cdiv(H, 64);
-            p.M = total_rows;
-            p.K = H;
-            p.epi = EPI_INJECT;
-            p.d = d;
-            p.cap = cc->capacity;
-            p.layer = l0;
-            p.batch = cc->batch;
-            p.len = cc->len;
-            p.rope = h->rope;
-            p.slab = (__nv_bfloat16*)cc->slab;
-            p.s_req = cc->s_req;
-            p.s_layer = cc->s_layer;
-            p.s_kind = cc->s_kind;
-            p.s_kv = cc->s_kv;
-            p.row_start = row_start;
-            p.row_count = row_count;
-            Timed t(h, TK_GEMM_INJECT, st);
-            int r = run_gemm(h, p, nt, st);
-            if (r) return r;
-        }
+        int r = inject_gemms(h, cc, ctx, row_start, row_count, total_rows, nullptr, nullptr, st);
+        if (r) return r;
     } else {
         Timed t(h, TK_SIMT_F32, st);
         XSegs xs;
@@ -579,14 +684,69 @@ int dflash_inject_kv(dflash_handle* h, dflash_cache* cc, const void* ctx, const 
         }
     }
     Timed t(h, TK_INJECT_FINALIZE, st);
-    launch_inject_finalize(row_count, cc->batch, cc->capacity, cc->len, cc->status, st);
+    launch_inject_finalize(row_count, cc->batch, cc->capacity, cc->len, cc->status, st,
+                           c.dtype == DFLASH_BF16 ? trace_small(h, TK_INJECT_FINALIZE, cdiv(cc->batch, 128)) : nullptr);
     h->launches += 1;
     return cuda_status(cudaGetLastError());
 }
 
 // ---------------------------------------------------------------------------
+// a1 + a2 in one call: the verify-side pre-step
+// ---------------------------------------------------------------------------
+int dflash_fuse_inject(dflash_handle* h, dflash_cache* cc, const void* const* hiddens, int64_t row_stride,
+                       const int32_t* row_start, const int32_t* row_count, int total_rows, void* ctx_out,
+                       dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !hiddens || !row_start || !row_count || total_rows < 0 ||
+        total_rows > h->cfg.max_rows)
+        return DFLASH_INVALID_ARG;
+    const dflash_config& c = h->cfg;
+    if (row_stride < c.target_hidden) return DFLASH_INVALID_ARG;
+    for (int i = 0; i < c.n_sel; ++i)
+        if (!hiddens[i]) return DFLASH_INVALID_ARG;
+    if (total_rows == 0) return DFLASH_OK;
+    cudaStream_t st = S(stream);
+    if (c.dtype == DFLASH_BF16 && g_fold && pick_nt(total_rows) <= kFoldMaxNT) {
+        if (ctx_out && !aligned16(ctx_out)) return DFLASH_INVALID_ARG;
+        // W_fc GEMM writing y and its rows' partial sums of squares, then the
+        // injection GEMMs normalising y (RMSNorm * g_fc) tile by tile in shared
+        // memory: the context feature never goes through a separate kernel.
+        int r = fuse_gemm(h, hiddens, row_stride, total_rows, h->ssq_ctx, st);
+        if (r) return r;
+        r = inject_gemms(h, cc, h->y, row_start, row_count, total_rows, h->ssq_ctx, ctx_out, st);
+        if (r) return r;
+        Timed t(h, TK_INJECT_FINALIZE, st);
+        launch_inject_finalize(row_count, cc->batch, cc->capacity, cc->len, cc->status, st,
+                               trace_small(h, TK_INJECT_FINALIZE, cdiv(cc->batch, 128)));
+        h->launches += 1;
+        return cuda_status(cudaGetLastError());
+    }
+    // wide token tiles (prefill) and fp32 storage: the two calls one after the other
+    // (the normalised rows go to ctx_out, or in place over y)
+    void* ctx = ctx_out ? ctx_out : h->y;
+    int r = dflash_fuse_context(h, hiddens, row_stride, total_rows, ctx, stream);
+    if (r) return r;
+    return dflash_inject_kv(h, cc, ctx, row_start, row_count, total_rows, stream);
+}
+
+// ---------------------------------------------------------------------------
 // a3..a7: draft block
 // ---------------------------------------------------------------------------
+// The draft step folds each RMSNorm into the GEMM that consumes its output when
+// the token tile is at most kFoldMaxNT wide (see GemmParams::ssq_in).
+static bool fold_norms(const dflash_handle* h, int M) {
+    return g_fold && h->cfg.dtype == DFLASH_BF16 && pick_nt(M) <= kFoldMaxNT;
+}
+
+// Consume the residual stream x normalised by `gain` (RMSNorm folded into the GEMM).
+static void fold_in(dflash_handle* h, GemmParams& p, const void* gain, int ssq_tiles) {
+    p.ssq_in = h->ssq;
+    p.ssq_tiles = ssq_tiles;
+    p.ssq_ld = h->cfg.max_batch * h->cfg.max_gamma;
+    p.gain = (const __nv_bfloat16*)gain;
+    p.eps = (float)h->cfg.rms_eps;
+    p.norm_h = h->cfg.hidden;
+}
+
 static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* drafts, float* logits, float* margin,
                       cudaStream_t st) {
     const dflash_config& c = h->cfg;
@@ -594,9 +754,13 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
     const int H = c.hidden, d = c.head_dim, Nq = c.n_q_heads * d, Nkv = c.n_kv_heads * d, I = c.intermediate;
     typedef __nv_bfloat16 bf;
     const int nt = pick_nt(M);
-    CUtensorMap tm_h, tm_o, tm_act, tm_hf;
+    const bool fold = fold_norms(h, M);
+    const int nH = cdiv(H, 128);                 // producer n-tiles of x: partial sums per row
+    const int ssq_ld = c.max_batch * c.max_gamma;
+    CUtensorMap tm_h, tm_o, tm_act, tm_hf, tm_x;
     if (!act_map(&tm_h, h->h, M, H, H, nt) || !act_map(&tm_o, h->o, M, Nq, Nq, nt) ||
-        !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)))
+        !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)) ||
+        !act_map(&tm_x, h->x, M, H, H, nt))
         return DFLASH_CUDA;
     int splits, chunk;
     attn_plan(B, c.n_kv_heads, cc->capacity, h->num_sms, attn_max_cluster(d), splits, chunk);
@@ -619,11 +783,14 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
     ap.rows_req = cc->s_req / d;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     ap.status = h->status;
+    const int attn_blocks = splits * c.n_kv_heads * B;
 
+    capture_x(h, 0, M, st);
     for (int l = 0; l < c.n_layers; ++l) {
-        {
+        if (!fold) {
             Timed t(h, TK_RMSNORM, st);
-            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_in[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st);
+            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_in[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st,
+                               trace_small(h, TK_RMSNORM, M));
             h->launches += 1;
         }
         {   // QKV + RoPE; block K/V to cache scratch rows [len, len + gamma)
@@ -636,7 +803,8 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.amat[1].rows = Nkv;
             p.amat[2].rows = Nkv;
             p.n_amat = 3;
-            p.tb[0] = tm_h;
+            p.tb[0] = fold ? tm_x : tm_h;
+            if (fold) fold_in(h, p, h->w.g_in[l], l == 0 ? 1 : nH);   // layer 0: the embedding's row sums
             p.kb_per_b = cdiv(H, 64);
             p.M = M;
             p.K = H;
@@ -657,10 +825,12 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.s_kind = cc->s_kind;
             p.s_kv = cc->s_kv;
             Timed t(h, TK_GEMM_QKV, st);
-            int r = run_gemm(h, p, nt, st);
+            int r = run_gemm(h, p, nt, st, TK_GEMM_QKV);
             if (r) return r;
         }
         ap.layer = l;
+        // attention trace: 8 stamps per CTA (attn.cuh), past the wait at 1, merge done at 7
+        ap.trace = trace_slot(h, TK_ATTENTION, attn_blocks, 8, 1, 7);
         {
             Timed t(h, TK_ATTENTION, st);
             int e = launch_attention(ap, d, B, st, &h->launches);
@@ -679,13 +849,18 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.epi = EPI_RESID;
             p.out = h->x;
             p.ldo = H;
+            if (fold) {
+                p.ssq_out = h->ssq;
+                p.ssq_ld = ssq_ld;
+            }
             Timed t(h, TK_GEMM_O, st);
-            int r = run_gemm(h, p, nt, st);
+            int r = run_gemm(h, p, nt, st, TK_GEMM_O);
             if (r) return r;
         }
-        {
+        if (!fold) {
             Timed t(h, TK_RMSNORM, st);
-            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_post[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st);
+            launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_post[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st,
+                               trace_small(h, TK_RMSNORM, M));
             h->launches += 1;
         }
         {   // gate/up + SwiGLU
@@ -696,7 +871,8 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.n_amat = 2;
             p.swiglu = 1;
             p.n_tiles = I / 64;
-            p.tb[0] = tm_h;
+            p.tb[0] = fold ? tm_x : tm_h;
+            if (fold) fold_in(h, p, h->w.g_post[l], nH);
             p.kb_per_b = cdiv(H, 64);
             p.M = M;
             p.K = H;
@@ -704,7 +880,7 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.out = h->act;
             p.ldo = I;
             Timed t(h, TK_GEMM_SWIGLU, st);
-            int r = run_gemm(h, p, nt, st);
+            int r = run_gemm(h, p, nt, st, TK_GEMM_SWIGLU);
             if (r) return r;
         }
         {   // down + residual
@@ -720,37 +896,53 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             p.epi = EPI_RESID;
             p.out = h->x;
             p.ldo = H;
+            if (fold) {
+                p.ssq_out = h->ssq;
+                p.ssq_ld = ssq_ld;
+            }
             Timed t(h, TK_GEMM_DOWN, st);
-            int r = run_gemm(h, p, nt, st);
+            int r = run_gemm(h, p, nt, st, TK_GEMM_DOWN);
             if (r) return r;
         }
+        capture_x(h, l + 1, M, st);
     }
-    {
+    if (!fold) {
         Timed t(h, TK_RMSNORM, st);
         launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_final, (bf*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1,
-                           gamma, 1, st);
+                           gamma, 1, st, trace_small(h, TK_RMSNORM, Mlm));
         h->launches += 1;
+        capture_hf(h, Mlm, st);
+    } else if (h->cap_hf) {
+        // diagnostic capture only: the folded head never materialises hf
+        launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_final, (bf*)h->cap_hf, Mlm, H, (float)c.rms_eps,
+                           gamma - 1, gamma, 1, st);
     }
-    {   // shared LM head + per-tile top-2
+    {   // shared LM head + per-tile top-2 (folded: over every block row, the final
+        // norm applied to x on the fly; the anchor rows' results are not used)
         GemmParams p;
         std::memset(&p, 0, sizeof(p));
         p.ta[0] = h->tm_lm;
         p.amat[0].rows = c.vocab;
         p.n_amat = 1;
-        p.tb[0] = tm_hf;
+        p.tb[0] = fold ? tm_x : tm_hf;
         p.kb_per_b = cdiv(H, 64);
-        p.M = Mlm;
+        p.M = fold ? M : Mlm;
         p.K = H;
         p.epi = EPI_LMHEAD;
         p.vocab = c.vocab;
         p.logits = logits;
         p.records = h->rec;
+        if (fold) {
+            fold_in(h, p, h->w.g_final, nH);
+            p.lm_gamma = gamma;
+        }
         Timed t(h, TK_GEMM_LMHEAD, st);
-        int r = run_gemm(h, p, pick_nt(Mlm), st);
+        int r = run_gemm(h, p, fold ? nt : pick_nt(Mlm), st, TK_GEMM_LMHEAD);
         if (r) return r;
     }
     Timed t(h, TK_LM_REDUCE, st);
-    launch_lm_reduce(h->rec, cdiv(c.vocab, 128), Mlm, gamma - 1, h->req_ok, drafts, margin, st);
+    launch_lm_reduce(h->rec, cdiv(c.vocab, 128), Mlm, gamma - 1, h->req_ok, drafts, margin, st,
+                     trace_small(h, TK_LM_REDUCE, Mlm), fold ? 1 : 0);
     h->launches += 1;
     return DFLASH_OK;
 }
@@ -768,6 +960,7 @@ static int draft_f32(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dra
     xo.ptr[0] = o; xo.stride = Nq; xo.width = Nq;
     xa.ptr[0] = act; xa.stride = I; xa.width = I;
     xf.ptr[0] = (float*)h->hf; xf.stride = H; xf.width = H;
+    capture_x(h, 0, M, st);
     for (int l = 0; l < c.n_layers; ++l) {
         launch_rmsnorm<float>(x, (const float*)h->w.g_in[l], hh, M, H, (float)c.rms_eps, M, 0, 0, st);
         launch_gemm_f32(xh, (const float*)h->w.wq[l], h->y32, M, Nq, H, ldq, 0, st);
@@ -788,9 +981,11 @@ static int draft_f32(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dra
         launch_gemm_f32(xa, (const float*)h->w.w_down[l], h->y32, M, H, I, H, 0, st);
         launch_resid_f32(x, h->y32, (long long)M * H, st);
         h->launches += 14;
+        capture_x(h, l + 1, M, st);
     }
     launch_rmsnorm<float>(x, (const float*)h->w.g_final, (float*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1, gamma, 1,
                           st);
+    capture_hf(h, Mlm, st);
     float* lg = logits ? logits : h->lgs;
     launch_gemm_f32(xf, (const float*)h->w.lm_head, lg, Mlm, c.vocab, H, c.vocab, 0, st);
     launch_top2_rows(lg, Mlm, c.vocab, gamma - 1, h->req_ok, drafts, margin, st);
@@ -809,7 +1004,8 @@ int dflash_draft_block(dflash_handle* h, dflash_cache* cc, const int32_t* anchor
     if (c.dtype == DFLASH_BF16)
         launch_embed<__nv_bfloat16>((const __nv_bfloat16*)h->w.embed, anchor, c.mask_id, cc->batch, gamma, c.hidden,
                                     c.vocab, cc->len, cc->committed, cc->capacity, (__nv_bfloat16*)h->x, h->req_ok,
-                                    cc->status, st);
+                                    cc->status, st, trace_small(h, TK_EMBED, cc->batch * gamma),
+                                    gamma > 1 && fold_norms(h, cc->batch * gamma) ? h->ssq : nullptr);
     else
         launch_embed<float>((const float*)h->w.embed, anchor, c.mask_id, cc->batch, gamma, c.hidden, c.vocab, cc->len,
                             cc->committed, cc->capacity, (float*)h->x, h->req_ok, cc->status, st);
@@ -832,7 +1028,7 @@ int dflash_accept(dflash_handle* h, dflash_cache* cc, const int32_t* drafts, con
     if (gamma > 1 && !drafts) return DFLASH_INVALID_ARG;
     Timed t(h, TK_ACCEPT, st_of(stream));
     launch_accept(drafts ? drafts : target, target, cc->batch, gamma, h->cfg.vocab, cc->len, cc->committed, accept_len,
-                  next_anchor, cc->status, S(stream));
+                  next_anchor, cc->status, S(stream), trace_small(h, TK_ACCEPT, cdiv(cc->batch * 32, 128)));
     h->launches += 1;
     return cuda_status(cudaGetLastError());
 }
@@ -994,11 +1190,57 @@ int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* cc, const void*
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
 }
 
+int dflash_diag_step_trace(dflash_handle* h, int64_t* buf, int64_t words) {
+    if (!h || (buf && words <= 0)) return DFLASH_INVALID_ARG;
+    h->tr_buf = (long long*)buf;
+    h->tr_cap = buf ? words : 0;
+    h->tr_used = 0;
+    h->tr_recs.clear();
+    return DFLASH_OK;
+}
+
+int dflash_diag_step_trace_records(const dflash_handle* h, int32_t* recs, int64_t* offsets, int max_records,
+                                   int* n_records) {
+    if (!h || !n_records || max_records < 0 || (max_records > 0 && (!recs || !offsets))) return DFLASH_INVALID_ARG;
+    const int n = std::min((int)h->tr_recs.size(), max_records);
+    for (int i = 0; i < n; ++i) {
+        const auto& r = h->tr_recs[i];
+        recs[5 * i + 0] = r.kind;
+        recs[5 * i + 1] = r.blocks;
+        recs[5 * i + 2] = r.words;
+        recs[5 * i + 3] = r.wait_idx;
+        recs[5 * i + 4] = r.exit_idx;
+        offsets[i] = r.offset;
+    }
+    *n_records = (int)h->tr_recs.size();
+    return DFLASH_OK;
+}
+
+int dflash_diag_draft_capture(dflash_handle* h, void* x_layers, void* hf) {
+    if (!h) return DFLASH_INVALID_ARG;
+    h->cap_x = x_layers;
+    h->cap_hf = hf;
+    return DFLASH_OK;
+}
+
 int dflash_diag_wait_selftest(dflash_handle* h, int32_t* out, dflash_stream stream) {
     if (!h || !out) return DFLASH_INVALID_ARG;
     const int e = launch_wait_selftest(h->status, out, S(stream));
     h->launches += 1;
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
+}
+
+int dflash_diag_set_gemm_prefetch(int tiles) {
+    if (tiles < 0 || tiles > 256) return DFLASH_INVALID_ARG;
+    set_gemm_l2_prefetch(tiles);
+    return DFLASH_OK;
+}
+
+int dflash_diag_gemm_prefetch(void) { return gemm_l2_prefetch(); }
+
+int dflash_diag_set_norm_fold(int on) {
+    g_fold = on != 0;
+    return DFLASH_OK;
 }
 
 int dflash_diag_set_launch_mode(int programmatic) {

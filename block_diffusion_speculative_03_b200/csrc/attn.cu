@@ -96,24 +96,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                                : nullptr;
     if (trace && tid == 0) trace[0] = (long long)globaltimer_ns();
     if (tid == 0) tma_prefetch_desc(&p.tmap);
-    griddep_wait();
-    if (trace && tid == 0) trace[1] = (long long)globaltimer_ns();
+    // The kernel runs right after the QKV GEMM, which writes q and the block's own
+    // K/V rows [len, len + gamma).  len and the committed context rows [0, len)
+    // are older (the previous step's calls, complete before this step's first
+    // kernel passed its own dependency wait), so the committed-context tiles are
+    // loaded before this kernel's dependency wait, overlapping the GEMM's tail.
+    // q, the tiles holding block rows and req_ok (written by the embedding, which
+    // may still be running when this kernel starts) are read after it.  A skipped
+    // request (req_ok = 0) is attended over zero tiles: its output rows are zero.
 
     const int R = p.G * p.gamma;
     const int rows_per = (R + nsplit - 1) / nsplit;
     const int r_lo = rank * rows_per, r_hi = min(R, r_lo + rows_per);
-    if (!p.req_ok[b]) {   // skipped request: zero output rows, no cluster traffic
-        for (int r = r_lo; r < r_hi; ++r) {
-            const int j = r / p.G, hh = r % p.G;
-            __nv_bfloat16* dst = p.out + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D;
-            for (int c = tid; c < D; c += kAttnThreads) dst[c] = f2bf(0.f);
-        }
-        return;
-    }
-    const int n = p.len[b] + p.gamma;
+    const int len_b = p.len[b];
+    const int n = len_b + p.gamma;
     const int kv0 = rank * p.chunk;
     const int kv1 = min(n, kv0 + p.chunk);
-    const int ntiles = kv1 > kv0 ? (kv1 - kv0 + 63) / 64 : 0;
+    const int ntiles_all = kv1 > kv0 ? (kv1 - kv0 + 63) / 64 : 0;
+    // leading tiles made of committed context rows only (independent of the QKV GEMM)
+    const int n_early = min(min(ntiles_all, S), len_b > kv0 ? (len_b - kv0) / 64 : 0);
     const long long rowK = (long long)b * p.rows_req + (long long)p.layer * p.rows_layer + (long long)g * p.rows_kv;
     const long long rowV = rowK + p.rows_kind;
 
@@ -146,7 +147,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            for (int it = 0; it < ntiles; ++it) {
+            // first use of each ring stage: no free-slot wait needed
+            for (int it = 0; it < n_early; ++it) {
+                mbar_arrive_expect_tx(&kv_full[it], 2 * C::KV_BYTES);
+                for (int h = 0; h < C::HALVES; ++h) {
+                    tma_load_2d(sK + it * C::KV_BYTES + h * 8192, &p.tmap, &kv_full[it], h * 64,
+                                (int)(rowK + kv0 + it * 64));
+                    tma_load_2d(sV + it * C::KV_BYTES + h * 8192, &p.tmap, &kv_full[it], h * 64,
+                                (int)(rowV + kv0 + it * 64));
+                }
+            }
+        }
+        griddep_wait();
+        if (trace && lane == 0) trace[1] = (long long)globaltimer_ns();
+        const int ntiles = p.req_ok[b] ? ntiles_all : 0;
+        if (lane == 0) {
+            for (int it = n_early; it < ntiles; ++it) {
                 const int st = it % S;
                 if (!mbar_wait(&kv_empty[st], (uint32_t)(((it / S) & 1) ^ 1), abort_flag, p.status)) break;
                 mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
@@ -157,9 +173,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                                 (int)(rowV + kv0 + it * 64));
                 }
             }
+            // a skipped request consumes none of its early tiles: let them land
+            // before the CTA can exit
+            for (int it = ntiles; it < n_early; ++it) {
+                volatile int never = 0;
+                mbar_wait(&kv_full[it], 0, &never, nullptr);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        griddep_wait();
+        const int ntiles = p.req_ok[b] ? ntiles_all : 0;
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
@@ -207,6 +231,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         const int row = rl % RW, cs = rl / RW;         // query row, key slice (warp-uniform)
         const int e = tid - 64;                        // 0..127
         const uint32_t lanes = (uint32_t)(q4 * 32) << 16;
+        griddep_wait();                                // q comes from the QKV GEMM
+        const int ntiles = p.req_ok[b] ? ntiles_all : 0;
         {
             // The lane's Q row (zero past R) into the Q operand, and zeros into the
             // lane's columns of both P buffers (other slices' keys stay zero).

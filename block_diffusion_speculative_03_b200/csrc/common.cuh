@@ -88,6 +88,16 @@ DF_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
     }
 }
 
+// Step trace of the small kernels (null in normal use): thread 0 of every block
+// stamps %globaltimer (ns) into tr[2 * block + which], which = 0 once past the
+// dependency wait, 1 at exit.
+DF_DEV void trace_mark(long long* tr, int which) {
+    if (tr && threadIdx.x == 0) {
+        const size_t blk = blockIdx.x + (size_t)gridDim.x * (blockIdx.y + (size_t)gridDim.y * blockIdx.z);
+        tr[2 * blk + which] = (long long)globaltimer_ns();
+    }
+}
+
 // Named barrier over a subset of warps.
 DF_DEV void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -157,6 +167,11 @@ DF_DEV void tma_load_2d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int
         "[%0], [%1, {%2, %3}], [%4], %5;"
         ::"r"(smem_u32(dst)), "l"((uint64_t)m), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
+}
+// Prefetch a 2-D tile into L2 only (no shared-memory destination, no barrier).
+DF_DEV void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)m), "r"(x), "r"(y)
+                 : "memory");
 }
 DF_DEV uint64_t make_l2_policy_evict_first() {
     uint64_t p;

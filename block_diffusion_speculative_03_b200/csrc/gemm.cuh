@@ -48,6 +48,7 @@ struct GemmParams {
     int n_tiles, m_tiles;
     long long units;             // n_tiles * m_tiles * KB
     int ctas;
+    int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
     float* partial;              // [2 * ctas][NT][128] fp32 split-tile partials
     int* counters;               // [n_tiles * m_tiles], zero between launches
     int* status;                 // handle status word (DFLASH_TIMEOUT)
@@ -63,10 +64,26 @@ struct GemmParams {
     long long s_req, s_layer, s_kind, s_kv;
     const int* row_start;
     const int* row_count;
+    int row0;                    // EPI_INJECT: global index of this launch's first token row
     // EPI_LMHEAD
     int vocab;
-    float* logits;               // [M, vocab] or null
+    float* logits;               // [M, vocab] or null (with lm_gamma: [M / lm_gamma * (lm_gamma - 1), vocab])
     float4* records;             // [M][n_tiles]: (top1, id bits, top2, 0)
+    int lm_gamma;                // > 0: token rows are whole blocks of lm_gamma; logits skip each block's row 0
+    // RMSNorm folded into the GEMM that consumes the normalised rows: the B operand
+    // is the residual stream x, and every B stage is rewritten in shared memory as
+    // R(x * inv_rms(row) * gain[k]) before the MMA reads it.  inv_rms comes from
+    // per-tile partial sums of squares written by the producer of x.
+    const float* ssq_in;         // [ssq_tiles][ssq_ld] (null: plain B operand)
+    int ssq_tiles;
+    int ssq_ld;
+    const __nv_bfloat16* gain;   // [K]
+    float eps;
+    int norm_h;                  // features of a row (the mean's divisor)
+    __nv_bfloat16* norm_out;     // optional copy of the normalised rows [M][norm_out_ld] (written from n-tile 0)
+    int norm_out_ld;
+    // EPI_RESID / EPI_BF16: partial sums of squares of the written rows, per output n-tile
+    float* ssq_out;              // [n_tiles][ssq_ld] or null
     // Diagnostic trace (null in normal use): per CTA 8 globaltimer stamps (ns):
     // entry, producer past the dependency wait, first stage landed, last MMA
     // issued, accumulators drained, epilogue done, exit, clock64 span of the CTA.
@@ -107,6 +124,11 @@ inline int pick_nt(int M) {
     if (M <= 128) return 128;
     return 256;
 }
+
+// Weight tiles each CTA prefetches into L2 (beyond its shared-memory ring)
+// before its dependency wait; process-wide, set by dflash_diag_set_gemm_prefetch.
+int gemm_l2_prefetch();
+void set_gemm_l2_prefetch(int tiles);
 
 // Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
 // ctas) and launches on `stream`.  Returns a cudaError_t; cudaErrorInvalidValue

@@ -1,11 +1,13 @@
 // Persistent split-K tcgen05 GEMM with fused epilogues (see gemm.cuh).
 //
-// CTA = 6 warps:  warp 0 lane 0 issues TMA loads of (weight tile, token tile)
+// CTA = 7 warps:  warp 0 lane 0 issues TMA loads of (weight tile, token tile)
 // pairs into an S-stage shared-memory ring; warp 1 lane 0 issues tcgen05.mma
 // (M=128, N=NT, K=16, bf16 in, fp32 accumulate) into one of two TMEM
 // accumulator buffers; warps 2..5 (128 threads, one TMEM lane each) drain a
 // finished accumulator with tcgen05.ld, resolve split tiles, and run the
-// epilogue while the next tile accumulates in the other buffer.
+// epilogue while the next tile accumulates in the other buffer; warp 6, when
+// the GEMM consumes RMS-normalised rows, rewrites each token tile in shared
+// memory as R(x * inv_rms * gain) between its arrival and the MMA.
 #include "gemm.cuh"
 
 namespace df {
@@ -17,13 +19,14 @@ constexpr long long kGemmMaxGrid = 160;
 // that fits (two CTAs per SM with half the ring measured slower at batch 1).
 template <int NT>
 struct GemmCfg {
+    static constexpr int THREADS = 224;
     static constexpr bool TWO_PER_SM = false;
     static constexpr int A_BYTES = 128 * 128;            // 128 rows x 64 bf16
     static constexpr int B_BYTES = NT * 128;             // NT rows x 64 bf16
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int CH = NT < 32 ? NT : 32;         // epilogue column chunk
     static constexpr int XCH_FLOATS = 128 * (CH + 1);
-    static constexpr int MISC_BYTES = 4096;
+    static constexpr int MISC_BYTES = 6144;
     static constexpr int SMEM_CAP = TWO_PER_SM ? (233472 / 2 - 2048) : 232448;
     static constexpr int BUDGET = SMEM_CAP - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
     static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
@@ -55,8 +58,28 @@ DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2
     }
 }
 
+// The tile's share of each written row's sum of squares (sq: this thread's
+// feature, CH rows): over the 32 lanes of a warp (butterfly), then the four
+// warps in quadrant order, so every run adds in the same order.  Called by all
+// 128 epilogue threads (two named barriers); red: [4][CH] shared floats.
+template <int CH>
+DF_DEV void tile_ssq(float* sq, float* red, int q, int lane, int e, int mbase, int n_tile, const GemmParams& p) {
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], off);
+    if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < CH; ++i) red[q * CH + i] = sq[i];
+    named_bar_sync(1, 128);
+    if (e < CH && mbase + e < p.M)
+        p.ssq_out[(size_t)n_tile * p.ssq_ld + mbase + e] = ((red[e] + red[CH + e]) + red[2 * CH + e]) + red[3 * CH + e];
+    named_bar_sync(1, 128);
+}
+
 template <int NT>
-__global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
+    k_gemm_tc(const __grid_constant__ GemmParams p) {
     using C = GemmCfg<NT>;
     constexpr int S = C::STAGES;
     constexpr int CH = C::CH;
@@ -76,6 +99,9 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
     int* tok_b = s_flag + 1;          // [NT]
     int* tok_pos = tok_b + NT;        // [NT]
     float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
+    float* inv_s = lmred + 4 * CH * 3;       // [NT] inverse RMS of the current m-tile's rows
+    uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
+    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + NT * 4 + 8 + S * 8 <= C::MISC_BYTES, "misc");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 8 : nullptr;
@@ -90,6 +116,7 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 128);
         }
+        for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 32);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -113,9 +140,11 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
         if (lane == 0) {
             const uint64_t pol_w = make_l2_policy_evict_first();
             // Weights never depend on the previous kernel: start streaming the
-            // first S weight tiles before waiting for it to finish.
+            // first S weight tiles into the ring, and the next l2_prefetch ones
+            // into L2, before waiting for it to finish.
             int pre = 0;
-            for (long long u = u_begin; u < u_end && pre < S;) {
+            const int n_ahead = S + p.l2_prefetch;
+            for (long long u = u_begin, idx = 0; u < u_end && idx < n_ahead;) {
                 const long long t = u / KB;
                 const int kb0 = (int)(u % KB);
                 const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
@@ -124,14 +153,22 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                 if (!p.swiglu)
                     while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
                 const int arow = p.swiglu ? n_tile * 64 : (n_tile - p.amat[mi].tile0) * 128;
-                for (int kb = kb0; kb < kb1 && pre < S; ++kb, ++pre) {
-                    mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
-                    uint8_t* a = sA + pre * C::A_BYTES;
-                    if (p.swiglu) {
-                        tma_load_2d_hint(a, &p.ta[0], &full[pre], kb * 64, arow, pol_w);
-                        tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[pre], kb * 64, arow, pol_w);
+                for (int kb = kb0; kb < kb1 && idx < n_ahead; ++kb, ++idx) {
+                    if (idx < S) {
+                        mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+                        uint8_t* a = sA + pre * C::A_BYTES;
+                        if (p.swiglu) {
+                            tma_load_2d_hint(a, &p.ta[0], &full[pre], kb * 64, arow, pol_w);
+                            tma_load_2d_hint(a + 64 * 128, &p.ta[1], &full[pre], kb * 64, arow, pol_w);
+                        } else {
+                            tma_load_2d_hint(a, &p.ta[mi], &full[pre], kb * 64, arow, pol_w);
+                        }
+                        ++pre;
+                    } else if (p.swiglu) {
+                        tma_prefetch_l2_2d(&p.ta[0], kb * 64, arow);
+                        tma_prefetch_l2_2d(&p.ta[1], kb * 64, arow);
                     } else {
-                        tma_load_2d_hint(a, &p.ta[mi], &full[pre], kb * 64, arow, pol_w);
+                        tma_prefetch_l2_2d(&p.ta[mi], kb * 64, arow);
                     }
                 }
                 u += kb1 - kb0;
@@ -196,8 +233,9 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                 if (!mbar_wait(&acce[buf], (use & 1) ^ 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * NT);
+                uint64_t* const landed = p.ssq_in ? ready : full;   // normalised by warp 6 first
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(&full[stage], round & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(&landed[stage], round & 1, abort_flag, p.status)) { ok = false; break; }
                     if (trace && seg == 0 && kb == kb0) trace[2] = (long long)globaltimer_ns();
                     tc_fence_after();
                     const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
@@ -219,6 +257,64 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                 tc_commit(drain);
                 volatile int never = 0;
                 mbar_wait(drain, 0, &never, nullptr);
+            }
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ B normaliser
+        if (p.ssq_in) {
+            griddep_wait();
+            int stage = 0, cur_mt = -1;
+            uint32_t round = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const long long t = u / KB;
+                const int kb0 = (int)(u % KB);
+                const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+                const int m_tile = (int)(t % m_tiles);
+                // n-tile 0's k-blocks cover every feature once: its stages also go to norm_out
+                const bool copy_out = p.norm_out && t / m_tiles == 0;
+                if (m_tile != cur_mt) {
+                    // inverse RMS of the m-tile's rows from the producer's per-tile
+                    // partial sums, added in tile order (the same in every CTA)
+                    for (int r = lane; r < NT; r += 32) {
+                        const int m = m_tile * NT + r;
+                        float ss = 0.f;
+                        if (m < p.M)
+                            for (int j = 0; j < p.ssq_tiles; ++j) ss += __ldcg(p.ssq_in + (size_t)j * p.ssq_ld + m);
+                        inv_s[r] = 1.0f / sqrtf(ss / (float)p.norm_h + p.eps);
+                    }
+                    __syncwarp();
+                    cur_mt = m_tile;
+                }
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], round & 1, abort_flag, p.status)) { ok = false; break; }
+                    // the stage's NT x 64 tile in the 128-byte swizzle: row r at r * 128 bytes,
+                    // its 16-byte chunk j holds elements 8 (j ^ (r & 7)) .. + 7 of the k-block
+                    uint8_t* bt = sB + stage * C::B_BYTES;
+#pragma unroll 2
+                    for (int ch = lane; ch < NT * 8; ch += 32) {
+                        const int r = ch >> 3, j = ch & 7;
+                        const int f0 = kb * 64 + 8 * (j ^ (r & 7));
+                        uint4* ptr = reinterpret_cast<uint4*>(bt + r * 128 + j * 16);
+                        const uint4 xv = *ptr;
+                        const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gain + f0));
+                        const __nv_bfloat16* xe = reinterpret_cast<const __nv_bfloat16*>(&xv);
+                        const __nv_bfloat16* ge = reinterpret_cast<const __nv_bfloat16*>(&gv);
+                        const float inv = inv_s[r];
+                        uint4 out;
+                        __nv_bfloat16* oe = reinterpret_cast<__nv_bfloat16*>(&out);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) oe[k] = f2bf(bf2f(xe[k]) * inv * bf2f(ge[k]));
+                        *ptr = out;
+                        const int m = m_tile * NT + r;
+                        if (copy_out && m < p.M)
+                            *reinterpret_cast<uint4*>(p.norm_out + (size_t)m * p.norm_out_ld + f0) = out;
+                    }
+                    fence_proxy_async();   // the MMA reads the stage through the async proxy
+                    mbar_arrive(&ready[stage]);
+                    if (++stage == S) { stage = 0; ++round; }
+                }
+                u += kb1 - kb0;
             }
         }
     } else {
@@ -295,11 +391,11 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                     named_bar_sync(1, 128);
                     for (int te = e; te < NT; te += 128) tok_b[te] = -1;
                     named_bar_sync(1, 128);
-                    const int m0 = m_tile * NT;
+                    const int m0 = p.row0 + m_tile * NT;   // global row of the tile's first column
                     for (int bb = e; bb < p.batch; bb += 128) {
                         const int rs = p.row_start[bb], rc = p.row_count[bb], L0 = p.len[bb];
                         if (rc <= 0 || L0 < 0 || L0 + rc > p.cap) continue;
-                        const int lo = max(rs, m0), hi = min(min(rs + rc, m0 + NT), p.M);
+                        const int lo = max(rs, m0), hi = min(min(rs + rc, m0 + NT), p.row0 + p.M);
                         for (int m = lo; m < hi; ++m) {
                             tok_b[m - m0] = bb;
                             tok_pos[m - m0] = L0 + (m - rs);
@@ -354,10 +450,18 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
                     }
                     case EPI_BF16: {
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
-                        if (row_ok)
+                        float sq[CH];
 #pragma unroll
-                            for (int i = 0; i < CH; ++i)
-                                if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = f2bf(v[i]);
+                        for (int i = 0; i < CH; ++i) {
+                            sq[i] = 0.f;
+                            if (row_ok && mbase + i < p.M) {
+                                const __nv_bfloat16 yb = f2bf(v[i]);
+                                o[(size_t)(mbase + i) * p.ldo + lr] = yb;
+                                const float yf = bf2f(yb);
+                                sq[i] = yf * yf;
+                            }
+                        }
+                        if (p.ssq_out) tile_ssq<CH>(sq, lmred, q, lane, e, mbase, n_tile, p);
                         break;
                     }
                     case EPI_RESID: {
@@ -368,9 +472,18 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
 #pragma unroll
                         for (int i = 0; i < CH; ++i)
                             rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+                        float sq[CH];
 #pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            if (row_ok && mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = f2bf(rv[i] + v[i]);
+                        for (int i = 0; i < CH; ++i) {
+                            sq[i] = 0.f;
+                            if (row_ok && mbase + i < p.M) {
+                                const __nv_bfloat16 xb = f2bf(rv[i] + v[i]);
+                                o[(size_t)(mbase + i) * p.ldo + lr] = xb;
+                                const float xf = bf2f(xb);
+                                sq[i] = xf * xf;
+                            }
+                        }
+                        if (p.ssq_out) tile_ssq<CH>(sq, lmred, q, lane, e, mbase, n_tile, p);
                         break;
                     }
                     case EPI_SWIGLU: {
@@ -440,7 +553,14 @@ __global__ void __launch_bounds__(192, GemmCfg<NT>::MIN_BLOCKS) k_gemm_tc(const 
 #pragma unroll 1
                         for (int i = 0; i < CH; ++i) {
                             const int m = mbase + i;
-                            if (p.logits && row_ok && m < p.M) p.logits[(size_t)m * p.vocab + vid] = v[i];
+                            if (p.logits && row_ok && m < p.M) {
+                                int lrow = m;
+                                if (p.lm_gamma) {
+                                    const int j = m % p.lm_gamma;
+                                    lrow = j == 0 ? -1 : (m / p.lm_gamma) * (p.lm_gamma - 1) + j - 1;
+                                }
+                                if (lrow >= 0) p.logits[(size_t)lrow * p.vocab + vid] = v[i];
+                            }
                             float a1 = row_ok ? v[i] : -INFINITY, a2 = -INFINITY;
                             int ai = row_ok ? vid : 0x7fffffff;
 #pragma unroll
@@ -503,10 +623,14 @@ static int launch_nt(GemmParams& p, cudaStream_t stream) {
         if (e != cudaSuccess) return (int)e;
         attr_done = true;
     }
-    cudaError_t e = launch_k(k_gemm_tc<NT>, dim3(p.ctas), dim3(192), (size_t)C::SMEM, stream, p);
+    cudaError_t e = launch_k(k_gemm_tc<NT>, dim3(p.ctas), dim3(C::THREADS), (size_t)C::SMEM, stream, p);
     if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
 }
+
+static int g_l2_prefetch = 0;
+int gemm_l2_prefetch() { return g_l2_prefetch; }
+void set_gemm_l2_prefetch(int tiles) { g_l2_prefetch = tiles < 0 ? 0 : (tiles > 256 ? 256 : tiles); }
 
 int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
     p.KB = (p.K + 63) / 64;

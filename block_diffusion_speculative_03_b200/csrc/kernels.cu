@@ -10,12 +10,16 @@ namespace df {
 // len == committed, len + gamma <= capacity and the anchor is a valid token;
 // otherwise its rows are zero, req_ok[b] = 0 and the first error is recorded.
 // ---------------------------------------------------------------------------
+// With ssq non-null the block also writes its row's sum of squares ssq[m] (the
+// statistic of the first layer's input RMSNorm, which the QKV GEMM applies).
 template <typename T>
 __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anchor, int mask_id, int gamma, int H,
                         int V, const int* __restrict__ len, const int* __restrict__ committed, int cap,
-                        T* __restrict__ x, int* __restrict__ req_ok, int* __restrict__ status) {
+                        T* __restrict__ x, int* __restrict__ req_ok, int* __restrict__ status, float* __restrict__ ssq,
+                        long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     const int m = blockIdx.x, b = m / gamma, j = m % gamma;
     const int L0 = len[b], a = anchor[b];
     int err = 0;
@@ -29,13 +33,36 @@ __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anc
     T* dst = x + (size_t)m * H;
     if (err) {
         for (int i = threadIdx.x; i < H; i += blockDim.x) stf(dst + i, 0.0f);
+        if (ssq && threadIdx.x == 0) ssq[m] = 0.f;
+        trace_mark(tr, 1);
         return;
     }
     const int tok = (j == 0) ? a : mask_id;
     const T* src = embed + (size_t)tok * H;
     constexpr int VEC = 16 / sizeof(T);
-    for (int i = threadIdx.x * VEC; i < H; i += blockDim.x * VEC)
-        *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<const uint4*>(src + i);
+    float ss = 0.f;
+    for (int i = threadIdx.x * VEC; i < H; i += blockDim.x * VEC) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+        *reinterpret_cast<uint4*>(dst + i) = u;
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+            const float v = ldf(e + k);
+            ss += v * v;
+        }
+    }
+    if (ssq) {   // fixed order: each thread's chunks, the warp butterfly, then the warps in order
+        __shared__ float red[32];
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+            ssq[m] = t;
+        }
+    }
+    trace_mark(tr, 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -46,9 +73,10 @@ __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anc
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* __restrict__ y, int H, float eps,
-                          int grp, int gstride, int goff) {
+                          int grp, int gstride, int goff, long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     constexpr int VEC = 16 / sizeof(T);          // elements per 16-byte access
     const int o = blockIdx.x;
     const int in = (o / grp) * gstride + goff + o % grp;
@@ -87,6 +115,7 @@ __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* _
         for (int k = 0; k < VEC; ++k) stf(oe + k, ldf(e + k) * inv * ldf(ge + k));
         yr[i] = out;
     }
+    trace_mark(tr, 1);
 }
 
 // Top-2 merge with ties of the top value to the lower id.
@@ -109,13 +138,17 @@ constexpr int kLmReduceThreads = 512;
 
 __global__ void __launch_bounds__(kLmReduceThreads) k_lm_reduce(const float4* __restrict__ rec, int n_vt, int M,
                                                                  int gm1, const int* __restrict__ req_ok,
-                                                                 int* __restrict__ drafts, float* __restrict__ margin) {
+                                                                 int* __restrict__ drafts, float* __restrict__ margin,
+                                                                 int rec_blocks, long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     __shared__ float s1[kLmReduceThreads / 32], s2[kLmReduceThreads / 32];
     __shared__ int si[kLmReduceThreads / 32];
     const int m = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const float4* row = rec + (size_t)m * n_vt;
+    // records of draft row m: row m, or with rec_blocks (records for whole blocks of
+    // gamma = gm1 + 1 rows, anchor rows included) row m + m / gm1 + 1
+    const float4* row = rec + (size_t)(rec_blocks ? m + m / gm1 + 1 : m) * n_vt;
     float a1 = -INFINITY, a2 = -INFINITY;
     int ai = 0x7fffffff;
     for (int t = threadIdx.x; t < n_vt; t += kLmReduceThreads) {
@@ -136,6 +169,7 @@ __global__ void __launch_bounds__(kLmReduceThreads) k_lm_reduce(const float4* __
         drafts[m] = ok ? ai : -1;
         if (margin) margin[m] = ok ? a1 - a2 : 0.f;
     }
+    trace_mark(tr, 1);
 }
 
 // fp32 path: top-2 over the fp32 logits of each row; one CTA per row.
@@ -173,9 +207,10 @@ __global__ void k_top2_rows(const float* __restrict__ logits, int V, int gm1, co
 // ---------------------------------------------------------------------------
 __global__ void k_accept(const int* __restrict__ drafts, const int* __restrict__ target, int B, int gamma, int V,
                          int* __restrict__ len, int* __restrict__ committed, int* __restrict__ accept_len,
-                         int* __restrict__ next_anchor, int* __restrict__ status) {
+                         int* __restrict__ next_anchor, int* __restrict__ status, long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (b >= B) return;
     const int tg = lane < gamma ? target[(size_t)b * gamma + lane] : 0;
@@ -198,31 +233,41 @@ __global__ void k_accept(const int* __restrict__ drafts, const int* __restrict__
             if (len[b] > c) len[b] = c;
         }
     }
+    trace_mark(tr, 1);
 }
 
 // After an injection: len[b] += row_count[b] for every request that fitted.
 __global__ void k_inject_finalize(const int* __restrict__ row_count, int B, int cap, int* __restrict__ len,
-                                  int* __restrict__ status) {
+                                  int* __restrict__ status, long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= B) return;
-    const int rc = row_count[b];
-    if (rc < 0) { set_error(status, DFLASH_INVALID_ARG); return; }
-    if (len[b] + rc > cap) { set_error(status, DFLASH_CAPACITY); return; }
-    len[b] += rc;
+    if (b < B) {
+        const int rc = row_count[b];
+        if (rc < 0) set_error(status, DFLASH_INVALID_ARG);
+        else if (len[b] + rc > cap) set_error(status, DFLASH_CAPACITY);
+        else len[b] += rc;
+    }
+    trace_mark(tr, 1);
 }
 
 __global__ void k_set_len(const int* __restrict__ lens, int B, int cap, int* __restrict__ len,
-                          int* __restrict__ committed, int* __restrict__ status) {
+                          int* __restrict__ committed, int* __restrict__ status, long long* tr) {
     griddep_wait();
     griddep_launch();
+    trace_mark(tr, 0);
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= B) return;
-    const int v = lens[b];
-    if (v < 0 || v > cap) { set_error(status, DFLASH_CAPACITY); return; }
-    len[b] = v;
-    committed[b] = v;
+    if (b < B) {
+        const int v = lens[b];
+        if (v < 0 || v > cap) {
+            set_error(status, DFLASH_CAPACITY);
+        } else {
+            len[b] = v;
+            committed[b] = v;
+        }
+    }
+    trace_mark(tr, 1);
 }
 
 // Stand-in for the target's greedy verification (diagnostic).
@@ -440,41 +485,49 @@ __global__ void k_attn_f32(const float* __restrict__ q, const float* __restrict_
 // ---------------------------------------------------------------------------
 template <typename T>
 void launch_embed(const T* embed, const int* anchor, int mask_id, int B, int gamma, int H, int V, const int* len,
-                  const int* committed, int cap, T* x, int* req_ok, int* status, cudaStream_t st) {
-    launch_k(k_embed<T>, dim3(B * gamma), dim3(128), 0, st, embed, anchor, mask_id, gamma, H, V, len, committed, cap, x, req_ok, status);
+                  const int* committed, int cap, T* x, int* req_ok, int* status, cudaStream_t st, long long* tr,
+                  float* ssq) {
+    launch_k(k_embed<T>, dim3(B * gamma), dim3(128), 0, st, embed, anchor, mask_id, gamma, H, V, len, committed, cap, x,
+             req_ok, status, ssq, tr);
 }
 template <typename T>
 void launch_rmsnorm(const T* x, const T* g, T* y, int rows, int H, float eps, int grp, int gstride, int goff,
-                    cudaStream_t st) {
+                    cudaStream_t st, long long* tr) {
     if (rows <= 0) return;
-    launch_k(k_rmsnorm<T>, dim3(rows), dim3(H / (16 / (int)sizeof(T)) >= 256 ? 256 : 128), 0, st, x, g, y, H, eps, grp, gstride, goff);
+    launch_k(k_rmsnorm<T>, dim3(rows), dim3(H / (16 / (int)sizeof(T)) >= 256 ? 256 : 128), 0, st, x, g, y, H, eps,
+             grp, gstride, goff, tr);
 }
 template void launch_embed<float>(const float*, const int*, int, int, int, int, int, const int*, const int*, int,
-                                  float*, int*, int*, cudaStream_t);
+                                  float*, int*, int*, cudaStream_t, long long*, float*);
 template void launch_embed<__nv_bfloat16>(const __nv_bfloat16*, const int*, int, int, int, int, int, const int*,
-                                          const int*, int, __nv_bfloat16*, int*, int*, cudaStream_t);
-template void launch_rmsnorm<float>(const float*, const float*, float*, int, int, float, int, int, int, cudaStream_t);
+                                          const int*, int, __nv_bfloat16*, int*, int*, cudaStream_t, long long*,
+                                          float*);
+template void launch_rmsnorm<float>(const float*, const float*, float*, int, int, float, int, int, int, cudaStream_t,
+                                    long long*);
 template void launch_rmsnorm<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*, __nv_bfloat16*, int, int,
-                                            float, int, int, int, cudaStream_t);
+                                            float, int, int, int, cudaStream_t, long long*);
 
 void launch_lm_reduce(const float4* rec, int n_vt, int M, int gm1, const int* req_ok, int* drafts, float* margin,
-                      cudaStream_t st) {
-    launch_k(k_lm_reduce, dim3(M), dim3(kLmReduceThreads), 0, st, rec, n_vt, M, gm1, req_ok, drafts, margin);
+                      cudaStream_t st, long long* tr, int rec_blocks) {
+    launch_k(k_lm_reduce, dim3(M), dim3(kLmReduceThreads), 0, st, rec, n_vt, M, gm1, req_ok, drafts, margin,
+             rec_blocks, tr);
 }
 void launch_top2_rows(const float* logits, int M, int V, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st) {
     launch_k(k_top2_rows, dim3(M), dim3(256), 0, st, logits, V, gm1, req_ok, drafts, margin);
 }
 void launch_accept(const int* drafts, const int* target, int B, int gamma, int V, int* len, int* committed,
-                   int* accept_len, int* next_anchor, int* status, cudaStream_t st) {
-    launch_k(k_accept, dim3((B * 32 + 127) / 128), dim3(128), 0, st, drafts, target, B, gamma, V, len, committed, accept_len,
-                                                   next_anchor, status);
+                   int* accept_len, int* next_anchor, int* status, cudaStream_t st, long long* tr) {
+    launch_k(k_accept, dim3((B * 32 + 127) / 128), dim3(128), 0, st, drafts, target, B, gamma, V, len, committed,
+             accept_len, next_anchor, status, tr);
 }
-void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st) {
-    launch_k(k_inject_finalize, dim3((B + 127) / 128), dim3(128), 0, st, row_count, B, cap, len, status);
+void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st,
+                            long long* tr) {
+    launch_k(k_inject_finalize, dim3((B + 127) / 128), dim3(128), 0, st, row_count, B, cap, len, status, tr);
 }
-void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st) {
-    launch_k(k_set_len, dim3((B + 127) / 128), dim3(128), 0, st, lens, B, cap, len, committed, status);
+void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st,
+                    long long* tr) {
+    launch_k(k_set_len, dim3((B + 127) / 128), dim3(128), 0, st, lens, B, cap, len, committed, status, tr);
 }
 void launch_synth_target(const int* drafts, const int* a_plan, const int* rnd, int B, int gamma, int V, int* target,
                          cudaStream_t st) {

@@ -12,18 +12,21 @@ struct XSegs {            // X = concat_s seg[s] along k; seg s is [rows, width]
 
 template <typename T>
 void launch_embed(const T* embed, const int* anchor, int mask_id, int B, int gamma, int H, int V, const int* len,
-                  const int* committed, int cap, T* x, int* req_ok, int* status, cudaStream_t st);
+                  const int* committed, int cap, T* x, int* req_ok, int* status, cudaStream_t st,
+                  long long* tr = nullptr, float* ssq = nullptr);
 template <typename T>
 void launch_rmsnorm(const T* x, const T* g, T* y, int rows, int H, float eps, int grp, int gstride, int goff,
-                    cudaStream_t st);
+                    cudaStream_t st, long long* tr = nullptr);
 void launch_lm_reduce(const float4* rec, int n_vt, int M, int gm1, const int* req_ok, int* drafts, float* margin,
-                      cudaStream_t st);
+                      cudaStream_t st, long long* tr = nullptr, int rec_blocks = 0);
 void launch_top2_rows(const float* logits, int M, int V, int gm1, const int* req_ok, int* drafts, float* margin,
                       cudaStream_t st);
 void launch_accept(const int* drafts, const int* target, int B, int gamma, int V, int* len, int* committed,
-                   int* accept_len, int* next_anchor, int* status, cudaStream_t st);
-void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st);
-void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st);
+                   int* accept_len, int* next_anchor, int* status, cudaStream_t st, long long* tr = nullptr);
+void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st,
+                            long long* tr = nullptr);
+void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st,
+                    long long* tr = nullptr);
 int launch_wait_selftest(int* status, int* out, cudaStream_t st);
 void launch_synth_target(const int* drafts, const int* a_plan, const int* rnd, int B, int gamma, int V, int* target,
                          cudaStream_t st);

@@ -89,6 +89,7 @@ def lib():
         "dflash_cache_status": (i32, [vp, vp, vp]),
         "dflash_fuse_context": (i32, [vp, C.POINTER(vp), i64, i32, vp, vp]),
         "dflash_inject_kv": (i32, [vp, vp, vp, vp, vp, i32, vp]),
+        "dflash_fuse_inject": (i32, [vp, vp, C.POINTER(vp), i64, vp, vp, i32, vp, vp]),
         "dflash_draft_block": (i32, [vp, vp, vp, i32, vp, vp, vp, vp]),
         "dflash_accept": (i32, [vp, vp, vp, vp, i32, vp, vp, vp]),
         "dflash_status_string": (C.c_char_p, [i32]),
@@ -103,11 +104,18 @@ def lib():
         "dflash_diag_timing_disable": (i32, [vp]),
         "dflash_diag_timed_name": (C.c_char_p, [i32]),
         "dflash_diag_set_launch_mode": (i32, [i32]),
+        "dflash_diag_set_gemm_prefetch": (i32, [i32]),
+        "dflash_diag_gemm_prefetch": (i32, []),
+        "dflash_diag_set_norm_fold": (i32, [i32]),
         "dflash_diag_wait_selftest": (i32, [vp, vp, vp]),
         "dflash_diag_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
         "dflash_diag_gemm_bf16_traced": (i32, [vp, vp, vp, i32, i32, i32, vp, sz, i32, vp, vp]),
         "dflash_diag_attention_traced": (i32, [vp, vp, vp, vp, i32, i32, vp, C.POINTER(i32), vp]),
         "dflash_diag_gemm_bf16_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
+        "dflash_diag_draft_capture": (i32, [vp, vp, vp]),
+        "dflash_diag_step_trace": (i32, [vp, vp, i64]),
+        "dflash_diag_step_trace_records": (i32, [vp, C.POINTER(C.c_int32), C.POINTER(i64), i32, C.POINTER(i32)]),
+        "dflash_diag_gemm_bf16_noalloc_status": (i32, [C.POINTER(C.c_int32), vp]),
         "dflash_gamma_policy_init": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(i32), i32, C.c_double,
                                            C.c_double, C.c_double, C.c_double, C.c_double]),
         "dflash_gamma_policy_observe": (i32, [C.POINTER(dflash_gamma_policy), C.POINTER(C.c_int32), i32, i32]),
@@ -126,13 +134,16 @@ def lib():
 def exported_symbols() -> list:
     return ["dflash_workspace_bytes", "dflash_create", "dflash_destroy", "dflash_cache_bytes", "dflash_cache_init",
             "dflash_cache_release", "dflash_cache_get_info", "dflash_cache_set_len", "dflash_cache_status",
-            "dflash_fuse_context", "dflash_inject_kv", "dflash_draft_block", "dflash_accept",
+            "dflash_fuse_context", "dflash_inject_kv", "dflash_fuse_inject", "dflash_draft_block", "dflash_accept",
             "dflash_status_string", "dflash_launch_count", "dflash_diag_gemm_scratch_bytes",
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
-            "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_wait_selftest",
+            "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_set_gemm_prefetch", "dflash_diag_gemm_prefetch",
+            "dflash_diag_set_norm_fold",
+            "dflash_diag_wait_selftest",
             "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
-            "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc",
+            "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc", "dflash_diag_draft_capture",
+            "dflash_diag_gemm_bf16_noalloc_status", "dflash_diag_step_trace", "dflash_diag_step_trace_records",
             "dflash_gamma_policy_init", "dflash_gamma_policy_observe", "dflash_gamma_policy_alpha",
             "dflash_gamma_policy_expected_tokens", "dflash_gamma_policy_choose"]
 
@@ -204,6 +215,13 @@ def dflash_inject_kv(h: int, c: int, ctx: int, row_start: int, row_count: int, t
     return _chk(lib().dflash_inject_kv(h, c, ctx, row_start, row_count, total_rows, stream), "dflash_inject_kv", check)
 
 
+def dflash_fuse_inject(h: int, c: int, hiddens: Sequence[int], row_stride: int, row_start: int, row_count: int,
+                       total_rows: int, ctx_out: Optional[int] = None, stream: int = 0, check: bool = True) -> int:
+    arr = (C.c_void_p * max(1, len(hiddens)))(*hiddens)
+    return _chk(lib().dflash_fuse_inject(h, c, arr, row_stride, row_start, row_count, total_rows, ctx_out, stream),
+                "dflash_fuse_inject", check)
+
+
 def dflash_draft_block(h: int, c: int, anchor: int, gamma: int, drafts: int, logits: Optional[int] = None,
                        margin: Optional[int] = None, stream: int = 0, check: bool = True) -> int:
     return _chk(lib().dflash_draft_block(h, c, anchor, gamma, drafts, logits, margin, stream),
@@ -244,6 +262,13 @@ def dflash_diag_gemm_bf16_noalloc(X: int, W: int, Y: int, M: int, N: int, K: int
     """The same GEMM with its scratch in the library's static device array (no allocation)."""
     return _chk(lib().dflash_diag_gemm_bf16_noalloc(X, W, Y, M, N, K, grid, stream),
                 "dflash_diag_gemm_bf16_noalloc", check)
+
+
+def dflash_diag_gemm_bf16_noalloc_status(stream: int = 0) -> int:
+    """Status word of the last no-allocation GEMM on this device (syncs `stream`)."""
+    v = C.c_int32(0)
+    _chk(lib().dflash_diag_gemm_bf16_noalloc_status(C.byref(v), stream), "dflash_diag_gemm_bf16_noalloc_status")
+    return v.value
 
 
 def dflash_diag_partition(units: int, kb: int, ctas: int, tile: int):
@@ -287,6 +312,40 @@ def dflash_diag_timed_name(kind: int) -> str:
 
 def dflash_diag_set_launch_mode(programmatic: bool) -> int:
     return _chk(lib().dflash_diag_set_launch_mode(1 if programmatic else 0), "dflash_diag_set_launch_mode")
+
+
+def dflash_diag_step_trace(h: int, buf: Optional[int], words: int = 0) -> int:
+    return _chk(lib().dflash_diag_step_trace(h, buf, words if buf else 0), "dflash_diag_step_trace")
+
+
+def dflash_diag_step_trace_records(h: int, max_records: int = 4096):
+    """List of dicts (kind name, blocks, words, wait_idx, exit_idx, offset) in launch order."""
+    recs = (C.c_int32 * (5 * max_records))()
+    offs = (C.c_int64 * max_records)()
+    n = C.c_int(0)
+    _chk(lib().dflash_diag_step_trace_records(h, recs, offs, max_records, C.byref(n)),
+         "dflash_diag_step_trace_records")
+    out = []
+    for i in range(min(n.value, max_records)):
+        out.append({"kind": dflash_diag_timed_name(recs[5 * i]), "blocks": recs[5 * i + 1], "words": recs[5 * i + 2],
+                    "wait_idx": recs[5 * i + 3], "exit_idx": recs[5 * i + 4], "offset": offs[i]})
+    return out
+
+
+def dflash_diag_draft_capture(h: int, x_layers: Optional[int], hf: Optional[int]) -> int:
+    return _chk(lib().dflash_diag_draft_capture(h, x_layers, hf), "dflash_diag_draft_capture")
+
+
+def dflash_diag_set_gemm_prefetch(tiles: int) -> int:
+    return _chk(lib().dflash_diag_set_gemm_prefetch(int(tiles)), "dflash_diag_set_gemm_prefetch")
+
+
+def dflash_diag_gemm_prefetch() -> int:
+    return lib().dflash_diag_gemm_prefetch()
+
+
+def dflash_diag_set_norm_fold(on: bool) -> int:
+    return _chk(lib().dflash_diag_set_norm_fold(1 if on else 0), "dflash_diag_set_norm_fold")
 
 
 def dflash_diag_wait_selftest(h: int, out: int, stream: int = 0) -> int:

@@ -145,6 +145,18 @@ class Drafter:
         D.dflash_inject_kv(self.handle, cache.handle, ctx.data_ptr(), row_start.data_ptr(), row_count.data_ptr(),
                            ctx.shape[0], _stream())
 
+    def fuse_inject(self, cache: Cache, hiddens: Sequence[torch.Tensor], row_start: torch.Tensor,
+                    row_count: torch.Tensor, ctx_out: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
+        """fuse_context + inject_kv of the same rows in one library call."""
+        rows = hiddens[0].shape[0]
+        stride = hiddens[0].stride(0)
+        for h in hiddens:
+            assert h.dtype == self.torch_dtype and h.stride(1) == 1 and h.stride(0) == stride and h.shape[0] == rows
+        D.dflash_fuse_inject(self.handle, cache.handle, [h.data_ptr() for h in hiddens], stride, row_start.data_ptr(),
+                             row_count.data_ptr(), rows, ctx_out.data_ptr() if ctx_out is not None else None,
+                             _stream())
+        return ctx_out
+
     def draft_block(self, cache: Cache, anchor: torch.Tensor, gamma: int, drafts: Optional[torch.Tensor] = None,
                     logits: Optional[torch.Tensor] = None, margin: Optional[torch.Tensor] = None) -> torch.Tensor:
         if drafts is None:

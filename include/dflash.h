@@ -204,6 +204,25 @@ int dflash_fuse_context(dflash_handle* h, const void* const* hiddens, int64_t ro
 int dflash_inject_kv(dflash_handle* h, dflash_cache* c, const void* ctx, const int32_t* row_start,
                      const int32_t* row_count, int total_rows, dflash_stream stream);
 
+/* a1 + a2 in one call: the verify-side pre-step.  DFlash-ja §2.2, context-feature
+ * bullet (the verified rows' hidden states of the selected target layers are
+ * concatenated and projected) and KV-injection bullet (the feature goes into every
+ * draft layer's K/V cache), taken straight from the target's verification output.
+ * Computes exactly dflash_fuse_context followed by dflash_inject_kv of the same
+ * rows (the same rounding points: ctx = R(RMSNorm(R(y)) * g_fc) is what the K/V
+ * projections read), but with small batches of rows (at most 64 per call) the
+ * RMSNorm is folded into the injection GEMM: the W_fc GEMM also writes its rows'
+ * partial sums of squares, and the injection GEMM normalises its token tiles in
+ * shared memory, so no separate normalisation kernel runs and the feature is not
+ * re-read from memory.  Larger calls (prefill) run the two calls one after the other.
+ * hiddens, row_stride: as dflash_fuse_context; row_start, row_count (device),
+ * total_rows: as dflash_inject_kv (rows index the hidden-state rows).
+ * ctx_out: NULL, or device [total_rows, H] storage type receiving the context
+ * feature as dflash_fuse_context would write it.  Errors: as the two calls. */
+int dflash_fuse_inject(dflash_handle* h, dflash_cache* c, const void* const* hiddens, int64_t row_stride,
+                       const int32_t* row_start, const int32_t* row_count, int total_rows, void* ctx_out,
+                       dflash_stream stream);
+
 /* a3..a7. Draft one block per request.  anchor: device int32[batch].
  * 1 <= gamma <= max_gamma.  drafts: device int32[batch, gamma-1].
  * logits_opt: NULL or device fp32[batch, gamma-1, V]; margin_opt: NULL or device

@@ -51,22 +51,35 @@ int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, 
  * [M, K], W device bf16 [N, K], Y device fp32 [M, N] (all owned by the caller),
  * K % 8 == 0, 1 <= M <= 4096; grid = persistent CTAs (0 = one per SM).
  *
- * Size limit: the scratch needed is the tile counters (4 bytes per 128 x nt
- * output tile, nt = 16/32/64/128/256 from M) plus 2 * CTAs * nt * 512 bytes of
- * partials.  M <= 32 always fits; a larger M fits only with a smaller grid.  A
- * call whose need exceeds the array returns DFLASH_WORKSPACE and launches
- * nothing.  Other returns: DFLASH_INVALID_ARG (bad sizes, pointers or
+ * Size limit: the scratch needed is a 256-byte status word, the tile counters
+ * (4 bytes per 128 x nt output tile, nt = 16/32/64/128/256 from M, rounded up
+ * to 256 bytes) and 2 * CTAs * nt * 512 bytes of partials.  At the largest grid
+ * (160 CTAs), M <= 32 fits for N up to 33.5 million and M <= 16 for N up to 117
+ * million; a larger M fits only with a smaller grid.  A call whose need exceeds
+ * the array returns DFLASH_WORKSPACE and launches nothing.  Other returns: DFLASH_INVALID_ARG (bad sizes, pointers or
  * alignment), DFLASH_CUDA (the symbol lookup, the counter clear or the launch
  * failed).
  *
  * The first call on each device looks up the array's address with that device
  * current (this may load the module); make that first call before any stream
- * capture begins.  Each call clears the counters on `stream` before the launch.
+ * capture begins.  The address is kept together with the CUDA context it was
+ * looked up in and looked up again when the current context differs (after a
+ * device reset).  Each call clears the status word and the counters on `stream`
+ * before the launch; a wait that runs out is reported by
+ * dflash_diag_gemm_bf16_noalloc_status, not by this call's return value.
  * One array serves every caller on a device: calls that may overlap on the same
  * device (other streams, other host threads) race on it and must be serialised
  * by the caller. */
 int dflash_diag_gemm_bf16_noalloc(const void* X, const void* W, float* Y, int M, int N, int K, int grid,
                                   dflash_stream stream);
+
+/* Status of the last dflash_diag_gemm_bf16_noalloc on this device: synchronises
+ * `stream` (the stream of that call) and writes to *status (host) DFLASH_OK, or
+ * DFLASH_TIMEOUT when a bounded wait inside the kernel ran out, in which case Y
+ * is incomplete.  The word lives in the same static array and is cleared by the
+ * next dflash_diag_gemm_bf16_noalloc.  Allocates nothing.  Returns DFLASH_OK,
+ * DFLASH_INVALID_ARG (status NULL) or DFLASH_CUDA. */
+int dflash_diag_gemm_bf16_noalloc_status(int32_t* status, dflash_stream stream);
 
 /* Work partition of the persistent split-K GEMM (host only, no CUDA call).
  * `units` k-blocks in total, `kb` k-blocks per output tile, `ctas` CTAs.  For
@@ -111,6 +124,40 @@ int dflash_diag_attention(dflash_handle* h, dflash_cache* c, const void* q, void
 int dflash_diag_attention_traced(dflash_handle* h, dflash_cache* c, const void* q, void* out, int layer, int gamma,
                                  int64_t* trace, int* splits_out, dflash_stream stream);
 
+/* Step trace: per-block %globaltimer stamps (ns) of every kernel the handle's
+ * bf16 calls launch while it is set, for attributing a captured step's time to
+ * its kernels.  buf: device int64[words], zero-filled by the caller; each traced
+ * launch takes the next blocks * words_per_block words (a launch that does not fit
+ * is not traced).  Block b of a launch stamps word b * words_per_block + wait_idx
+ * once past its dependency wait and word b * words_per_block + exit_idx when it is
+ * done; blocks a launch does not use stay zero.  The pointers are fixed at launch
+ * time, so a step captured in a CUDA graph with tracing set writes the same words
+ * on every replay.  dflash_diag_step_trace(h, NULL, 0) stops tracing; setting a
+ * buffer restarts the record list.  Launches outside the handle's calls (the
+ * verification stand-in) are not traced. */
+int dflash_diag_step_trace(dflash_handle* h, int64_t* buf, int64_t words);
+
+/* The launches traced since dflash_diag_step_trace was set, in launch order:
+ * recs (host int32[max_records][5]) = (kind, blocks, words_per_block, wait_idx,
+ * exit_idx), offsets (host int64[max_records]) = first word of the launch in buf;
+ * kind names come from dflash_diag_timed_name.  *n_records = the number traced
+ * (may exceed max_records; only max_records are written). */
+int dflash_diag_step_trace_records(const dflash_handle* h, int32_t* recs, int64_t* offsets, int max_records,
+                                   int* n_records);
+
+/* Capture of the draft step's intermediate states, for call-local parity checks
+ * (each stage compared with the oracle run on the GPU's own input to it).  While
+ * set, every dflash_draft_block on the handle also copies (on its stream):
+ *   x_layers: device [(n_layers+1)][batch*gamma][hidden], storage type: the
+ *             residual stream after the embedding (slot 0) and after each layer l
+ *             (slot l+1), rows b*gamma + j;
+ *   hf:       device [batch*(gamma-1)][hidden], storage type: the final-norm rows
+ *             that the LM head reads, rows b*(gamma-1) + j-1.
+ * Either may be NULL; dflash_diag_draft_capture(h, NULL, NULL) stops capturing.
+ * The buffers are borrowed and must hold the largest batch*gamma drafted while set.
+ * Not for use under CUDA-graph capture of a timed step (the copies are extra work). */
+int dflash_diag_draft_capture(dflash_handle* h, void* x_layers, void* hf);
+
 /* Self-test of the device-side bounded wait used by the pipelined kernels: a
  * one-warp kernel waits on a shared-memory barrier that nothing arrives at.  The
  * wait gives up after its limit (about 2 s), records DFLASH_TIMEOUT in the
@@ -125,6 +172,24 @@ int dflash_diag_wait_selftest(dflash_handle* h, int32_t* out, dflash_stream stre
  * results in-kernel, and the GEMM streams its first weight tiles before that
  * wait), 0 = plain stream-ordered launches. */
 int dflash_diag_set_launch_mode(int programmatic);
+
+/* Weight tiles (128 x 64 bf16 each) that every CTA of the tensor-core GEMM
+ * prefetches into L2, beyond the tiles it loads into its shared-memory ring,
+ * before waiting for the previous kernel of the stream (process-wide, 0..256;
+ * applies to launches enqueued afterwards).  The weights never depend on the
+ * previous kernel, so this keeps HBM streaming across kernel boundaries. */
+int dflash_diag_set_gemm_prefetch(int tiles);
+/* The current setting of dflash_diag_set_gemm_prefetch. */
+int dflash_diag_gemm_prefetch(void);
+
+/* Whether the draft step folds each RMSNorm into the GEMM that consumes its
+ * output (process-wide, default 1; applies to calls enqueued afterwards).  When
+ * on and the token tile is at most 64 wide, the producer of the residual stream
+ * (the embedding, the O-projection and the down-projection) also writes per-tile
+ * partial sums of squares of its rows, and the QKV, gate/up and LM-head GEMMs
+ * read x itself and normalise each token tile in shared memory; no separate
+ * normalisation kernel runs.  0 = one RMSNorm kernel before each of them. */
+int dflash_diag_set_norm_fold(int on);
 
 /* "sm_100a" for this build. */
 const char* dflash_diag_arch(void);

@@ -26,9 +26,10 @@ def rel_err(g: np.ndarray, r: np.ndarray) -> float:
     return float(np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-30))
 
 
-def check_float(w: I.Workload, got: np.ndarray, ref: np.ndarray, what: str, bf16_rel: float = 2.0 ** -6):
-    """fp32: relative 1e-4; bf16 storage values: within a couple of bf16 ulps of the row scale,
-    with almost all elements identical."""
+def check_float(w: I.Workload, got: np.ndarray, ref: np.ndarray, what: str, bf16_rel: float = 2.0 ** -6,
+                min_same: float = 0.9):
+    """fp32: relative 1e-4; bf16 storage values: within 2^-6 of the tensor's scale, with at
+    least 90 % of elements identical (the rest single rounding flips)."""
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     if got.size == 0:
         return
@@ -40,7 +41,7 @@ def check_float(w: I.Workload, got: np.ndarray, ref: np.ndarray, what: str, bf16
         e = float(np.max(np.abs(got - ref)))
         assert e <= bf16_rel * scale, (what, e, scale)
         same = float(np.mean(got == ref))
-        assert same > 0.75, (what, same)   # differences are single rounding flips, not systematic
+        assert same >= min_same, (what, same)   # differences are single rounding flips, not systematic
 
 
 MAX_SEEN = {"logits": 0.0}
@@ -107,7 +108,9 @@ class Pair:
             ctx_o = self.ora.fuse_context([to_np(h[s0:s0 + T]) for h in hid])
             if check:
                 check_float(w, ctx_g_np[s0:s0 + T], ctx_o, "ctx[%d]" % b)
-            self.ora.inject_kv(self.ocache[b], ctx_o)
+            # the oracle injects the GPU's ctx (compared just above), so that the
+            # cache comparison tests the injection and not an inherited ctx flip
+            self.ora.inject_kv(self.ocache[b], ctx_g_np[s0:s0 + T])
             self.ocache[b]["committed"] = self.ocache[b]["len"]
         self.cache.set_len(torch.tensor(w.context, dtype=torch.int32))
         if check:
@@ -180,9 +183,12 @@ class Pair:
         torch.cuda.synchronize()
         assert self.cache.status() == 0
         acc_g, nxt_g = acc.cpu().numpy(), nxt.cpu().numpy()
+        ctx_g_np = ctx_g.double().cpu().numpy()
         out = []
         for b in range(B):
             ctx_o = self.ora.fuse_context([to_np(h[b * gamma:(b + 1) * gamma]) for h in hid])
+            check_float(w, ctx_g_np[b * gamma:(b + 1) * gamma], ctx_o, "ctx rows [%d]" % b)
+            ctx_o = ctx_g_np[b * gamma:(b + 1) * gamma]   # the oracle injects the GPU's ctx
             oc = self.ocache[b]
             if order == "speculative":
                 self.ora.inject_kv(oc, ctx_o)

@@ -1,13 +1,17 @@
-"""Parity at the full workload sizes, in the launch configuration the benchmark
-uses: the GPU runs the whole batch; the oracle recomputes sampled requests.
+"""Chained parity at the full workload sizes, in the launch configuration the
+benchmark uses: the GPU runs the whole batch; the oracle runs sampled requests
+end to end through its own draft step (each layer on its own previous layer's
+output), so rounding flips compound over the five bf16 layers.
 
-Logit tolerance at these sizes: five bf16-rounded layers of width 4096 are
-chaotic with respect to rounding, so two oracles that differ only in their
-accumulation precision (fp64 vs fp32) already disagree by ~0.06 in max logit
-(0.012 rms) on these inputs.  The GPU's logits must be within
-max(3e-2, 1.5 x that oracle-vs-oracle gap measured on the same request); the
-draft tokens must still match exactly wherever the oracle's top-1 margin
-exceeds 0.1, and every length exactly.
+The stated bf16 logit bound (3e-2) is held call-locally, stage by stage, in
+test_gpu_call_local.py.  Chained end to end it is not reachable at these sizes:
+five bf16-rounded layers of width 4096 are chaotic with respect to rounding, so
+two oracles that differ only in their accumulation precision (fp64 vs fp32)
+already disagree by ~0.06 in max logit on these inputs, and the GPU's chained
+logits land 0.065-0.077 from the fp64 oracle (2.2-2.6 x the bound).  Here the
+logits must be within max(3e-2, 1.5 x that oracle-vs-oracle gap measured on the
+same request); the draft tokens must still match exactly wherever the oracle's
+top-1 margin exceeds 0.1, and every length exactly.
 
 The committed context of every request is filled with seeded K/V rows from the
 input generator (the spread of injected keys/values), so the oracle needs no
@@ -128,7 +132,9 @@ def _run(name, sample, cycles, gammas=None):
             rows = [h[b * g:(b + 1) * g].cpu() for h in hid]
             ctx_o = od.fuse_context([to_np(r) for r in rows])
             check_float(w, ctx_np[b * g:(b + 1) * g], ctx_o, "ctx[%d]" % b)
-            od.inject_kv(ocache[b], ctx_o)
+            # the oracle injects the GPU's ctx (compared just above): the K/V check
+            # then tests the injection, not a ctx rounding flip it inherited
+            od.inject_kv(ocache[b], ctx_np[b * g:(b + 1) * g])
             st, a, nx = od.accept(ocache[b], o_drafts[b], target[b])
             assert st == 0 and a == plan[b] and nx == nxt_np[b]
             new = slice(T0, T0 + a + 1)

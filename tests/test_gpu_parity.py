@@ -38,8 +38,16 @@ def test_tiny_fp32_chain():
     assert n > 0
 
 
-def test_small_bf16_chain_speculative_order():
-    n = _chain("small_bf16")
+@pytest.mark.parametrize("fold", [True, False])
+def test_small_bf16_chain_speculative_order(fold):
+    # fold: each RMSNorm applied inside the GEMM that consumes it (the default for
+    # token tiles up to 64 wide); not fold: one normalisation kernel before each
+    from block_diffusion_speculative_03_b200 import dflash as D
+    D.dflash_diag_set_norm_fold(fold)
+    try:
+        n = _chain("small_bf16")
+    finally:
+        D.dflash_diag_set_norm_fold(True)
     assert n > 0
 
 

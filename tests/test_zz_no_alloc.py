@@ -1,8 +1,9 @@
 """The GEMM entry point that keeps its scratch in the library's static device
 array (dflash_diag_gemm_bf16_noalloc), called through the C ABI: two calls in
 a row must agree with the caller-scratch entry point (dflash_diag_gemm_bf16)
-and with an fp64 product of the same bf16 inputs, must not change the device's
-free memory, and sizes whose scratch exceeds the array must be refused.
+and with an fp64 product of the same bf16 inputs, must report a clear status
+word, must not change the device's free memory, and sizes whose scratch
+exceeds the array must be refused.
 
 The file name sorts last so that the test also runs after every other GPU test
 has used the library in the same process."""
@@ -42,6 +43,8 @@ def test_noalloc_matches_caller_scratch_gemm(M, N, K, grid):
     free_before = torch.cuda.mem_get_info()[0]
     for Y in Ys:
         D.dflash_diag_gemm_bf16_noalloc(Xd.data_ptr(), Wd.data_ptr(), Y.data_ptr(), M, N, K, grid, st)
+        # the status word in the static array: no bounded wait ran out
+        assert D.dflash_diag_gemm_bf16_noalloc_status(st) == 0
     torch.cuda.synchronize()
     free_after = torch.cuda.mem_get_info()[0]
     # the first call on this device may have loaded the module (and with it the
