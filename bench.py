@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--no-profile-pass", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
+    ap.add_argument("--conditioning", choices=["kv-injection", "input-fusion"], default="kv-injection",
+                    help="how the verified rows condition the drafter: injected into every layer's K/V (DFlash), "
+                         "or passed through the draft layers as input hidden states (the ablation)")
     ap.add_argument("--separate-pre-step", action="store_true",
                     help="fuse_context + inject_kv as two calls instead of one fuse_inject call")
     ap.add_argument("--no-fold", action="store_true", help="separate RMSNorm kernels in the draft step")
@@ -154,6 +157,7 @@ def traced_step(D, h, step, i0, K, st, ab, dump=None):
 def workload_description(w, B, T, g):
     family = ("LLaMA-3.1-8B-shaped" if w.name.startswith("llama")
               else "Qwen3-4B-shaped" if w.name.startswith("qwen3_4b")
+              else "Qwen3-Coder-30B-A3B-target-shaped" if w.name.startswith("qwen3_coder")
               else "Qwen3-8B-shaped" if w.name.startswith(("qwen3_8b", "long_ctx"))
               else "%s (%s, parity-size)" % (w.name, w.dtype))
     return ("%s drafter (hidden %d, %d layers, %d/%d heads, d %d, intermediate %d, vocab %d, %s LM head), "
@@ -235,11 +239,17 @@ def algorithmic_bytes(w, B, gamma, ctx_len):
     }
 
 
-def step_algorithmic_bytes(w, B, gamma, ctx_len):
+def step_algorithmic_bytes(w, B, gamma, ctx_len, conditioning="kv-injection"):
     ab = algorithmic_bytes(w, B, gamma, ctx_len)
     L = w.n_layers
-    return (L * (ab["gemm_qkv"] + ab["gemm_o"] + ab["gemm_swiglu"] + ab["gemm_down"] + ab["attention"])
-            + ab["gemm_lmhead"] + ab["gemm_fuse"] + ab["gemm_inject"])
+    draft = (L * (ab["gemm_qkv"] + ab["gemm_o"] + ab["gemm_swiglu"] + ab["gemm_down"] + ab["attention"])
+             + ab["gemm_lmhead"] + ab["gemm_fuse"])
+    if conditioning == "input-fusion":
+        # the gamma verified rows through every layer's QKV, and all but the last
+        # layer's attention, O-projection and MLP (causal over the context)
+        return draft + L * ab["gemm_qkv"] + (L - 1) * (ab["gemm_o"] + ab["gemm_swiglu"] + ab["gemm_down"]
+                                                       + ab["attention"])
+    return draft + ab["gemm_inject"]
 
 
 def step_flops(w, B, gamma, ctx_len):
@@ -478,7 +488,10 @@ def run_gpu(args):
         D.dflash_diag_synth_target(drafts.data_ptr(), a_plan[j].data_ptr(), rnd[j].data_ptr(), B, g, w.vocab,
                                    target.data_ptr(), sp)
         hl = hid_list if hid_list is not None else step_hid[i % POOL]
-        if args.separate_pre_step:
+        if args.conditioning == "input-fusion":
+            D.dflash_fuse_context(h, [x.data_ptr() for x in hl], w.target_hidden, B * g, ctx_step.data_ptr(), sp)
+            D.dflash_ingest_fused_input(h, c, ctx_step.data_ptr(), g, None, sp)
+        elif args.separate_pre_step:
             D.dflash_fuse_context(h, [x.data_ptr() for x in hl], w.target_hidden, B * g, ctx_step.data_ptr(), sp)
             D.dflash_inject_kv(h, c, ctx_step.data_ptr(), rs.data_ptr(), rc.data_ptr(), B * g, sp)
         else:   # the verify-side pre-step: fuse + inject of the verified rows in one call
@@ -548,7 +561,7 @@ def run_gpu(args):
 
     hbm_peak, tc_peak, peak_src = measured_peaks()
     ab = algorithmic_bytes(w, B, g, T)
-    step_bytes = step_algorithmic_bytes(w, B, g, T)
+    step_bytes = step_algorithmic_bytes(w, B, g, T, args.conditioning)
     t_roof_ms = step_bytes / (hbm_peak * 1e9) * 1e3
 
     # ---- traced pass: the same step captured in one CUDA graph with the library's
@@ -668,7 +681,9 @@ def run_gpu(args):
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) target hiddens; benchmark datasets not used)",
-            "config": config_of(w, world, B, T, g, step_bytes),
+            "config": dict(config_of(w, world, B, T, g, step_bytes),
+                           **({"conditioning": "input fusion (the ablation KV injection is compared against)"}
+                              if args.conditioning == "input-fusion" else {})),
             "drafted_tok_per_s": round(blocks_per_s * (g - 1), 1),
             "roofline": roofline,
             "step_roofline": {"algorithmic_bytes": step_bytes, "flops": step_flops(w, B, g, T),
@@ -684,7 +699,9 @@ def run_gpu(args):
             "prefill": prefill,
             "e2e": e2e,
             "gpu_launches": launches,
-            "step_options": {"pre_step": "two calls" if args.separate_pre_step else "fuse_inject (one call)",
+            "step_options": {"conditioning": args.conditioning,
+                             "pre_step": ("fuse_context + ingest_fused_input" if args.conditioning == "input-fusion"
+                                          else "two calls" if args.separate_pre_step else "fuse_inject (one call)"),
                              "norm_fold": not args.no_fold, "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch()},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
                                                                               else ", programmatic dependent launch"),

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "../../include/dflash.h"
+#include "../../include/dflash_ablation.h"
 #include "../../include/dflash_diag.h"
 #include "attn.cuh"
 #include "common.cuh"
@@ -141,7 +142,7 @@ int validate_config(const dflash_config* c) {
     if (c->dtype == DFLASH_BF16) {
         if (c->head_dim != 64 && c->head_dim != 128) return DFLASH_UNSUPPORTED;
         if (c->hidden % 64 || c->intermediate % 64 || c->target_hidden % 64) return DFLASH_UNSUPPORTED;
-        if ((c->n_q_heads / c->n_kv_heads) * c->max_gamma > 64) return DFLASH_UNSUPPORTED;
+        if ((c->n_q_heads / c->n_kv_heads) * c->max_gamma > 128) return DFLASH_UNSUPPORTED;
     } else {
         if (c->max_position > 12000) return DFLASH_UNSUPPORTED;   // fp32 attention keeps a row of scores in smem
     }
@@ -747,20 +748,25 @@ static void fold_in(dflash_handle* h, GemmParams& p, const void* gain, int ssq_t
     p.norm_h = h->cfg.hidden;
 }
 
-static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* drafts, float* logits, float* margin,
-                      cudaStream_t st) {
+// The draft layers over the block rows in h->x ([B * gamma][H], rows b * gamma +
+// j at positions len[b] + j), every request validated in h->req_ok.  Each layer
+// writes the rows' own K/V at cache rows [len, len + gamma).  draft: attention
+// without a mask (the block is bidirectional) and the rows' K/V are scratch.
+// ingest (input fusion): causal attention (row j sees positions <= len + j), and
+// the last layer stops once its K/V are written (its attention and MLP change no
+// cached value); the caller then appends the rows to the cache.
+static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool ingest, cudaStream_t st) {
     const dflash_config& c = h->cfg;
-    const int B = cc->batch, M = B * gamma, Mlm = B * (gamma - 1);
+    const int B = cc->batch, M = B * gamma;
     const int H = c.hidden, d = c.head_dim, Nq = c.n_q_heads * d, Nkv = c.n_kv_heads * d, I = c.intermediate;
     typedef __nv_bfloat16 bf;
     const int nt = pick_nt(M);
     const bool fold = fold_norms(h, M);
     const int nH = cdiv(H, 128);                 // producer n-tiles of x: partial sums per row
     const int ssq_ld = c.max_batch * c.max_gamma;
-    CUtensorMap tm_h, tm_o, tm_act, tm_hf, tm_x;
+    CUtensorMap tm_h, tm_o, tm_act, tm_x;
     if (!act_map(&tm_h, h->h, M, H, H, nt) || !act_map(&tm_o, h->o, M, Nq, Nq, nt) ||
-        !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)) ||
-        !act_map(&tm_x, h->x, M, H, H, nt))
+        !act_map(&tm_act, h->act, M, I, I, nt) || !act_map(&tm_x, h->x, M, H, H, nt))
         return DFLASH_CUDA;
     int splits, chunk;
     attn_plan(B, c.n_kv_heads, cc->capacity, h->num_sms, attn_max_cluster(d), splits, chunk);
@@ -783,6 +789,7 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
     ap.rows_req = cc->s_req / d;
     ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     ap.status = h->status;
+    ap.causal = ingest ? 1 : 0;
     const int attn_blocks = splits * c.n_kv_heads * B;
 
     capture_x(h, 0, M, st);
@@ -828,6 +835,7 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
             int r = run_gemm(h, p, nt, st, TK_GEMM_QKV);
             if (r) return r;
         }
+        if (ingest && l == c.n_layers - 1) break;   // the last layer's K/V are written
         ap.layer = l;
         // attention trace: 8 stamps per CTA (attn.cuh), past the wait at 1, merge done at 7
         ap.trace = trace_slot(h, TK_ATTENTION, attn_blocks, 8, 1, 7);
@@ -906,6 +914,22 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
         }
         capture_x(h, l + 1, M, st);
     }
+    return DFLASH_OK;
+}
+
+static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* drafts, float* logits, float* margin,
+                      cudaStream_t st) {
+    const dflash_config& c = h->cfg;
+    const int B = cc->batch, M = B * gamma, Mlm = B * (gamma - 1);
+    const int H = c.hidden;
+    typedef __nv_bfloat16 bf;
+    const int nt = pick_nt(M);
+    const bool fold = fold_norms(h, M);
+    const int nH = cdiv(H, 128);
+    int r = layers_bf16(h, cc, gamma, false, st);
+    if (r) return r;
+    CUtensorMap tm_hf, tm_x;
+    if (!act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)) || !act_map(&tm_x, h->x, M, H, H, nt)) return DFLASH_CUDA;
     if (!fold) {
         Timed t(h, TK_RMSNORM, st);
         launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_final, (bf*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1,
@@ -1015,6 +1039,27 @@ int dflash_draft_block(dflash_handle* h, dflash_cache* cc, const int32_t* anchor
     int r = c.dtype == DFLASH_BF16 ? draft_bf16(h, cc, gamma, drafts, logits_opt, margin_opt, st)
                                    : draft_f32(h, cc, gamma, drafts, logits_opt, margin_opt, st);
     if (r) return r;
+    return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// Input-fusion ablation: the context rows through the draft layers
+// ---------------------------------------------------------------------------
+int dflash_ingest_fused_input(dflash_handle* h, dflash_cache* cc, const void* ctx, int rows,
+                              const int32_t* row_count, dflash_stream stream) {
+    if (!h || !cc || cc->h != h || !ctx || rows < 1 || rows > h->cfg.max_gamma) return DFLASH_INVALID_ARG;
+    const dflash_config& c = h->cfg;
+    if (c.dtype != DFLASH_BF16) return DFLASH_UNSUPPORTED;
+    if (!aligned16(ctx)) return DFLASH_INVALID_ARG;
+    cudaStream_t st = S(stream);
+    const int B = cc->batch, M = B * rows;
+    launch_ingest_begin((const __nv_bfloat16*)ctx, B, rows, c.hidden, cc->len, cc->capacity, (__nv_bfloat16*)h->x,
+                        h->req_ok, cc->status, fold_norms(h, M) ? h->ssq : nullptr, st);
+    h->launches += 1;
+    int r = layers_bf16(h, cc, rows, true, st);
+    if (r) return r;
+    launch_ingest_end(row_count, rows, B, h->req_ok, cc->len, cc->status, st);
+    h->launches += 1;
     return cuda_status(cudaGetLastError());
 }
 

@@ -6,9 +6,9 @@
 // QKV epilogue wrote at [len, len+gamma): no mask.  CTA `rank` of the cluster
 // (b, g) takes keys [rank*chunk, (rank+1)*chunk).
 //
-// The R <= 64 query rows fill CS = 2 (R > 32) or 4 copies of a window of
-// RW = 128/CS lanes of an M = 128 tile: TMEM lane l holds query row l % RW and
-// takes key slice l / RW (64/CS keys) of every 64-key tile.  Q and P are MMA
+// The R <= 128 query rows fill CS = 1 (R > 64), 2 (R > 32) or 4 copies of a
+// window of RW = 128/CS lanes of an M = 128 tile: TMEM lane l holds query row
+// l % RW and takes key slice l / RW (64/CS keys) of every 64-key tile.  Q and P are MMA
 // operands in tensor memory, so the tensor cores read only K and V from
 // shared memory.
 //
@@ -55,7 +55,7 @@ struct AttnCfg {
     static constexpr uint32_t T_S = 0, T_Q = 192, T_O = 256, T_P = 384, TMEM_COLS = 512;
     static_assert(T_S + NS * 64 <= T_Q && T_Q + D / 2 <= T_O && T_O + D <= T_P && T_P + 64 <= TMEM_COLS, "TMEM");
     // the split's partial, written over the ring once the key loop is done
-    static_assert(128 * PO_LD * 4 + 64 * 8 + 3 * 64 * kAttnMaxSplits * 4 <= RING, "partial");
+    static_assert(128 * PO_LD * 4 + 128 * 8 + 3 * 128 * kAttnMaxSplits * 4 <= RING, "partial");
 };
 
 template <int D, int CS>
@@ -82,10 +82,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     float* xch = (float*)(smem + C::RING + 256);   // [128] per TMEM lane: running max, then row sum
     // After the key loop the ring holds this CTA's partial.
     float* po = (float*)smem;                      // [128][PO_LD] lanes' O, then rows 0..RW-1 summed
-    float2* pml = (float2*)(po + 128 * PO_LD);     // [64] (integer base, row sum)
-    float* cm = (float*)(pml + 64);                // [64][splits] peers' bases
-    float* cl = cm + 64 * kAttnMaxSplits;          // [64][splits] peers' sums
-    float* cw = cl + 64 * kAttnMaxSplits;          // [64][splits] merge weights
+    float2* pml = (float2*)(po + 128 * PO_LD);     // [128] (integer base, row sum)
+    float* cm = (float*)(pml + 128);               // [128][splits] peers' bases
+    float* cl = cm + 128 * kAttnMaxSplits;         // [128][splits] peers' sums
+    float* cw = cl + 128 * kAttnMaxSplits;         // [128][splits] merge weights
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         const int row = rl % RW, cs = rl / RW;         // query row, key slice (warp-uniform)
         const int e = tid - 64;                        // 0..127
         const uint32_t lanes = (uint32_t)(q4 * 32) << 16;
+        const int jrow = row < R ? row / p.G : 0;      // block position of this thread's query row
         griddep_wait();                                // q comes from the QKV GEMM
         const int ntiles = p.req_ok[b] ? ntiles_all : 0;
         {
@@ -276,8 +277,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             // is applied to the maximum (rounding is monotonic, so this equals the
             // maximum of the scaled scores) and inside the exponent's FMA.
             float t[KC];
-            if constexpr (KC == 32) tmem_ld32w(ts, t); else tmem_ld16w(ts, t);
-            const int nvalid = kv1 - kvb;
+            if constexpr (KC == 64) {
+                tmem_ld32w(ts, t);
+                tmem_ld32w(ts + 32, t + 32);
+            } else if constexpr (KC == 32) {
+                tmem_ld32w(ts, t);
+            } else {
+                tmem_ld16w(ts, t);
+            }
+            // keys past the split's end, and with a causal mask past the row's own position
+            const int nvalid = (p.causal ? min(kv1, len_b + jrow + 1) : kv1) - kvb;
             if (nvalid < KC) {
 #pragma unroll
                 for (int i = 0; i < KC; ++i) t[i] = (i < nvalid) ? t[i] : -INFINITY;
@@ -359,7 +368,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
                 ls[c0 >> 4] = s2;
             }
             const uint32_t tp = tP + lanes + sb * 32 + cs * (KC / 2);
-            if constexpr (KC == 32) {
+            if constexpr (KC == 64) {
+                float pv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pv[i] = __uint_as_float(pk[i]);
+                tmem_st16(tp, pv);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pv[i] = __uint_as_float(pk[16 + i]);
+                tmem_st16(tp + 16, pv);
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            } else if constexpr (KC == 32) {
                 float pv[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) pv[i] = __uint_as_float(pk[i]);
@@ -517,12 +535,14 @@ void attn_plan(int B, int nkv, int cap, int num_sms, int max_cluster, int& split
 
 int launch_attention(const AttnParams& p, int d, int B, cudaStream_t stream, long long* launches) {
     const int smem = attn_smem_bytes(d);
-    // Row copies: 4 when the R = G * gamma query rows fit 32 lanes, else 2 (R <= 64).
-    const bool four = p.G * p.gamma <= 32;
-    void (*kern)(AttnParams) = (d == 128) ? (four ? k_attn_tc<128, 4> : k_attn_tc<128, 2>)
-                                          : (four ? k_attn_tc<64, 4> : k_attn_tc<64, 2>);
-    static bool done_v[2][2] = {{false, false}, {false, false}};
-    bool& done = done_v[d == 128 ? 1 : 0][four ? 1 : 0];
+    // Row copies: 4 when the R = G * gamma query rows fit 32 lanes, 2 when they fit
+    // 64, else 1 (R <= 128: one lane per row, each softmax thread takes all 64 keys).
+    const int R = p.G * p.gamma;
+    const int cs = R <= 32 ? 4 : (R <= 64 ? 2 : 1);
+    void (*kern)(AttnParams) = (d == 128) ? (cs == 4 ? k_attn_tc<128, 4> : cs == 2 ? k_attn_tc<128, 2> : k_attn_tc<128, 1>)
+                                          : (cs == 4 ? k_attn_tc<64, 4> : cs == 2 ? k_attn_tc<64, 2> : k_attn_tc<64, 1>);
+    static bool done_v[2][3] = {{false, false, false}, {false, false, false}};
+    bool& done = done_v[d == 128 ? 1 : 0][cs == 4 ? 2 : cs - 1];
     if (!done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return (int)e;

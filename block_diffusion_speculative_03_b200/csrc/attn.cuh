@@ -11,6 +11,7 @@ struct AttnParams {
     const int* len;
     const int* req_ok;
     int gamma, G, nq, nkv, layer, splits, chunk;
+    int causal;                  // 0: every row sees all len + gamma keys; 1: row j sees keys [0, len + j]
     long long rows_req, rows_layer, rows_kind, rows_kv;
     float scale_log2;            // log2(e) / sqrt(d)
     int* status;

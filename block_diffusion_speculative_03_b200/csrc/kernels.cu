@@ -66,6 +66,65 @@ __global__ void k_embed(const T* __restrict__ embed, const int* __restrict__ anc
 }
 
 // ---------------------------------------------------------------------------
+// Input fusion, first step: the context rows become the block's input hidden
+// states.  One CTA per row m = b * rows + j: x[m] = ctx[m], ssq[m] = its sum of
+// squares (when ssq is set), req_ok[b] = (len[b] + rows <= capacity); a request
+// that does not fit records DFLASH_CAPACITY and is skipped.
+// ---------------------------------------------------------------------------
+__global__ void k_ingest_begin(const __nv_bfloat16* __restrict__ ctx, int rows, int H, const int* __restrict__ len,
+                               int cap, __nv_bfloat16* __restrict__ x, int* __restrict__ req_ok,
+                               int* __restrict__ status, float* __restrict__ ssq) {
+    griddep_wait();
+    griddep_launch();
+    const int m = blockIdx.x, b = m / rows, j = m % rows;
+    const bool fits = len[b] >= 0 && len[b] + rows <= cap;
+    if (j == 0 && threadIdx.x == 0) {
+        req_ok[b] = fits ? 1 : 0;
+        if (!fits) set_error(status, DFLASH_CAPACITY);
+    }
+    const __nv_bfloat16* src = ctx + (size_t)m * H;
+    __nv_bfloat16* dst = x + (size_t)m * H;
+    float ss = 0.f;
+    for (int i = threadIdx.x * 8; i < H; i += blockDim.x * 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+        *reinterpret_cast<uint4*>(dst + i) = u;
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float v = bf2f(e[k]);
+            ss += v * v;
+        }
+    }
+    if (ssq) {   // the same fixed order as the embedding's
+        __shared__ float red[32];
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+            ssq[m] = t;
+        }
+    }
+}
+
+// Input fusion, last step: append the ingested rows, len[b] += row_count[b]
+// (all `rows` when row_count is null) for every request that was processed.
+__global__ void k_ingest_end(const int* __restrict__ row_count, int rows, int B, const int* __restrict__ req_ok,
+                             int* __restrict__ len, int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch();
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B || !req_ok[b]) return;
+    const int n = row_count ? row_count[b] : rows;
+    if (n < 0 || n > rows) {
+        set_error(status, DFLASH_INVALID_ARG);
+        return;
+    }
+    len[b] += n;
+}
+
+// ---------------------------------------------------------------------------
 // RMSNorm: y[o] = R(x[in(o)] / sqrt(mean(x^2) + eps) * g), fp32 math.
 // in(o) = (o / grp) * gstride + goff + o % grp selects the rows (grp = rows,
 // gstride = 0, goff = 0 is the identity; grp = gamma-1, gstride = gamma,
@@ -520,6 +579,14 @@ void launch_accept(const int* drafts, const int* target, int B, int gamma, int V
                    int* accept_len, int* next_anchor, int* status, cudaStream_t st, long long* tr) {
     launch_k(k_accept, dim3((B * 32 + 127) / 128), dim3(128), 0, st, drafts, target, B, gamma, V, len, committed,
              accept_len, next_anchor, status, tr);
+}
+void launch_ingest_begin(const __nv_bfloat16* ctx, int B, int rows, int H, const int* len, int cap, __nv_bfloat16* x,
+                         int* req_ok, int* status, float* ssq, cudaStream_t st) {
+    launch_k(k_ingest_begin, dim3(B * rows), dim3(128), 0, st, ctx, rows, H, len, cap, x, req_ok, status, ssq);
+}
+void launch_ingest_end(const int* row_count, int rows, int B, const int* req_ok, int* len, int* status,
+                       cudaStream_t st) {
+    launch_k(k_ingest_end, dim3((B + 127) / 128), dim3(128), 0, st, row_count, rows, B, req_ok, len, status);
 }
 void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st,
                             long long* tr) {

@@ -23,6 +23,10 @@ void launch_top2_rows(const float* logits, int M, int V, int gm1, const int* req
                       cudaStream_t st);
 void launch_accept(const int* drafts, const int* target, int B, int gamma, int V, int* len, int* committed,
                    int* accept_len, int* next_anchor, int* status, cudaStream_t st, long long* tr = nullptr);
+void launch_ingest_begin(const __nv_bfloat16* ctx, int B, int rows, int H, const int* len, int cap, __nv_bfloat16* x,
+                         int* req_ok, int* status, float* ssq, cudaStream_t st);
+void launch_ingest_end(const int* row_count, int rows, int B, const int* req_ok, int* len, int* status,
+                       cudaStream_t st);
 void launch_inject_finalize(const int* row_count, int B, int cap, int* len, int* status, cudaStream_t st,
                             long long* tr = nullptr);
 void launch_set_len(const int* lens, int B, int cap, int* len, int* committed, int* status, cudaStream_t st,

@@ -1,5 +1,5 @@
-"""ctypes binding of libdflash (include/dflash.h, include/dflash_diag.h,
-include/dflash_policy.h).
+"""ctypes binding of libdflash (include/dflash.h, include/dflash_ablation.h,
+include/dflash_diag.h, include/dflash_policy.h).
 
 Functions carry the C names and only marshal arguments: every step of the
 draft step runs in the library's CUDA kernels.  Pointers are passed as ints
@@ -90,6 +90,7 @@ def lib():
         "dflash_fuse_context": (i32, [vp, C.POINTER(vp), i64, i32, vp, vp]),
         "dflash_inject_kv": (i32, [vp, vp, vp, vp, vp, i32, vp]),
         "dflash_fuse_inject": (i32, [vp, vp, C.POINTER(vp), i64, vp, vp, i32, vp, vp]),
+        "dflash_ingest_fused_input": (i32, [vp, vp, vp, i32, vp, vp]),
         "dflash_draft_block": (i32, [vp, vp, vp, i32, vp, vp, vp, vp]),
         "dflash_accept": (i32, [vp, vp, vp, vp, i32, vp, vp, vp]),
         "dflash_status_string": (C.c_char_p, [i32]),
@@ -135,6 +136,7 @@ def exported_symbols() -> list:
     return ["dflash_workspace_bytes", "dflash_create", "dflash_destroy", "dflash_cache_bytes", "dflash_cache_init",
             "dflash_cache_release", "dflash_cache_get_info", "dflash_cache_set_len", "dflash_cache_status",
             "dflash_fuse_context", "dflash_inject_kv", "dflash_fuse_inject", "dflash_draft_block", "dflash_accept",
+            "dflash_ingest_fused_input",
             "dflash_status_string", "dflash_launch_count", "dflash_diag_gemm_scratch_bytes",
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
@@ -220,6 +222,12 @@ def dflash_fuse_inject(h: int, c: int, hiddens: Sequence[int], row_stride: int, 
     arr = (C.c_void_p * max(1, len(hiddens)))(*hiddens)
     return _chk(lib().dflash_fuse_inject(h, c, arr, row_stride, row_start, row_count, total_rows, ctx_out, stream),
                 "dflash_fuse_inject", check)
+
+
+def dflash_ingest_fused_input(h: int, c: int, ctx: int, rows: int, row_count: Optional[int] = None, stream: int = 0,
+                              check: bool = True) -> int:
+    return _chk(lib().dflash_ingest_fused_input(h, c, ctx, rows, row_count, stream), "dflash_ingest_fused_input",
+                check)
 
 
 def dflash_draft_block(h: int, c: int, anchor: int, gamma: int, drafts: int, logits: Optional[int] = None,

@@ -157,6 +157,14 @@ class Drafter:
                              _stream())
         return ctx_out
 
+    def ingest_fused_input(self, cache: Cache, ctx: torch.Tensor, rows: int,
+                           row_count: Optional[torch.Tensor] = None) -> None:
+        """Input-fusion ablation: append `rows` context rows per request (ctx [batch*rows, H])
+        through the draft layers instead of injecting them."""
+        assert ctx.is_contiguous() and ctx.dtype == self.torch_dtype and ctx.shape[0] == cache.batch * rows
+        D.dflash_ingest_fused_input(self.handle, cache.handle, ctx.data_ptr(), rows,
+                                    row_count.data_ptr() if row_count is not None else None, _stream())
+
     def draft_block(self, cache: Cache, anchor: torch.Tensor, gamma: int, drafts: Optional[torch.Tensor] = None,
                     logits: Optional[torch.Tensor] = None, margin: Optional[torch.Tensor] = None) -> torch.Tensor:
         if drafts is None:

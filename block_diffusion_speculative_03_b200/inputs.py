@@ -191,6 +191,14 @@ def preset(name: str) -> Workload:
     if name == "qwen3_4b":
         return Workload("qwen3_4b", 2560, 5, 32, 8, 128, 9728, 151936, 5, 2560, 1e6, 1e-6, "bf16",
                         batch=1, gamma=16, context=[2048], seed=0xDF1A5 + 6)
+    # A drafter for a Qwen3-Coder-30B-A3B-shaped target: the target's hidden size
+    # (2048), 32 query heads of 128 over 4 key/value heads (8 query heads per kv
+    # head: 128 query rows per kv head at gamma 16), a dense SwiGLU of 3 x hidden
+    # (the target's experts are not part of the drafter), the Qwen3 vocabulary and
+    # a long-context RoPE base.
+    if name == "qwen3_coder_30b":
+        return Workload("qwen3_coder_30b", 2048, 5, 32, 4, 128, 6144, 151936, 5, 2048, 1e7, 1e-6, "bf16",
+                        batch=1, gamma=16, context=[2048], seed=0xDF1A5 + 7)
     # Reduced bf16 shapes that span several GEMM tiles and ragged tails but
     # that the oracle finishes in seconds.
     if name == "small_bf16":
@@ -204,7 +212,7 @@ def preset(name: str) -> Workload:
 
 
 PRESETS = ["tiny", "qwen3_8b", "qwen3_8b_b32", "long_ctx", "llama31_8b", "qwen3_8b_depth8", "qwen3_4b",
-           "small_bf16", "small_bf16_untied"]
+           "qwen3_coder_30b", "small_bf16", "small_bf16_untied"]
 
 
 # Tensor ids of the generator streams.

@@ -145,7 +145,7 @@ int dflash_workspace_bytes(const dflash_config* cfg, size_t* bytes);
  * and initialises the workspace (synchronously, on the legacy stream).
  * workspace: device memory, 1024-byte aligned, borrowed for the handle's life.
  * bf16 needs: H, I, H_t multiples of 64; head_dim 64 or 128;
- * (n_q_heads/n_kv_heads) * max_gamma <= 64.  Requires an sm_100 device. */
+ * (n_q_heads/n_kv_heads) * max_gamma <= 128.  Requires an sm_100 device. */
 int dflash_create(const dflash_config* cfg, const dflash_weights* w, void* workspace,
                   size_t ws_bytes, dflash_handle** out);
 void dflash_destroy(dflash_handle* h);

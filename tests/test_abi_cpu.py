@@ -24,7 +24,8 @@ def _declared(header):
 
 
 def test_exports_every_declared_symbol(lib):
-    names = _declared("dflash.h") + _declared("dflash_diag.h") + _declared("dflash_policy.h")
+    names = (_declared("dflash.h") + _declared("dflash_ablation.h") + _declared("dflash_diag.h")
+             + _declared("dflash_policy.h"))
     assert len(names) >= 20
     for n in names:
         assert hasattr(lib, n), n
@@ -55,7 +56,7 @@ def test_workspace_and_config_validation(lib):
            dict(max_gamma=0), dict(rope_theta=0.0)]
     for kw in bad:
         assert D.dflash_workspace_bytes(_cfg(**kw), check=False) == -1, kw
-    unsup = [dict(head_dim=96), dict(max_gamma=33), dict(hidden=4000), dict(max_gamma=32),
+    unsup = [dict(head_dim=96), dict(max_gamma=33), dict(hidden=4000), dict(max_gamma=32, n_kv_heads=4),
              dict(dtype=D.DFLASH_F32, max_position=20000)]
     for kw in unsup:
         assert D.dflash_workspace_bytes(_cfg(**kw), check=False) == -2, kw

@@ -19,7 +19,9 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("lens,gamma,nq,nkv,d", [([2048], 16, 32, 8, 128), ([100, 3000], 16, 8, 2, 128),
                                                  ([5000, 17, 700], 8, 6, 3, 64), ([64], 4, 8, 2, 128),
                                                  ([32768], 16, 32, 8, 128), ([4000], 8, 32, 8, 128),
-                                                 ([1500, 250], 11, 12, 4, 128)])
+                                                 ([1500, 250], 11, 12, 4, 128),
+                                                 # 8 and 12 query heads per kv head: 128 and 120 query rows
+                                                 ([2048, 300], 16, 32, 4, 128), ([700], 10, 24, 2, 64)])
 def test_attention_kernel_matches_oracle(lens, gamma, nq, nkv, d):
     B = len(lens)
     w = I.Workload("attn", 512, 1, nq, nkv, d, 1024, 1024, 1, 512, 1e6, 1e-6, "bf16", batch=B, gamma=gamma,

@@ -231,3 +231,7 @@ def test_call_local_long_context_gamma_sweep():
 
 def test_call_local_llama31_8b_batch16():
     assert _cycles("llama31_8b", sample=[5], cycles=1, check_cycles={0}) > 0
+
+
+def test_call_local_qwen3_coder_30b_shaped():
+    assert _cycles("qwen3_coder_30b", sample=[0], cycles=2, check_cycles={0, 1}, gammas=[16, 8]) > 0

@@ -176,3 +176,8 @@ def test_depth8_drafter():
 def test_qwen3_4b_shaped_drafter():
     # hidden 2560 with 32 x 128 query width: the O-proj reduces over 4096 into 2560
     assert _run("qwen3_4b", sample=[0], cycles=2) > 0
+
+
+def test_qwen3_coder_30b_shaped_drafter():
+    # hidden 2048, 32 query heads over 4 kv heads: 128 query rows per kv head at gamma 16
+    assert _run("qwen3_coder_30b", sample=[0], cycles=2, gammas=[16, 8]) > 0

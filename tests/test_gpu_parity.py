@@ -135,3 +135,21 @@ def test_small_bf16_long_context_multi_tile_splits():
     for cyc in range(w.cycles):
         o_dr, g_dr, n = pr.draft(anchors, w.gamma)
         anchors = pr.verify_and_accept(o_dr, w.gamma, plan[cyc], cyc)
+
+
+def test_small_bf16_wide_gqa_128_query_rows():
+    # 8 query heads on one kv head at gamma 16: 128 query rows per kv head (one copy
+    # of each row in the attention tile), through draft / verify / accept cycles
+    import dataclasses
+    w = dataclasses.replace(I.preset("small_bf16"), n_kv_heads=1, cycles=2)
+    pr = Pair(w)
+    pr.prefill()
+    anchors = I.make_anchors(w).numpy()
+    plan = I.plan_accept(w, w.cycles).numpy()
+    compared = 0
+    for cyc in range(w.cycles):
+        o_dr, g_dr, n = pr.draft(anchors, w.gamma)
+        compared += n
+        anchors = pr.verify_and_accept(o_dr, w.gamma, plan[cyc], cyc)
+        pr.check_cache()
+    assert compared > 0
