@@ -137,21 +137,36 @@ def traced_step(D, h, step, i0, K, st, ab, dump=None):
                                            for r in recs], dtype=np.int64))
     kern = {}
     for r in range(R):
-        prev_end = None
-        for rec in recs:
-            blk = H[r, rec["offset"]:rec["offset"] + rec["blocks"] * rec["words"]].reshape(rec["blocks"], rec["words"])
-            used = blk[:, rec["exit_idx"]] != 0
-            if not used.any():
-                continue
-            start = int(blk[used, rec["wait_idx"]].min())
-            end = int(blk[used, rec["exit_idx"]].max())
-            t = end - (prev_end if prev_end is not None else start)
-            prev_end = end
-            e = kern.setdefault(rec["kind"], [0, 0.0])
+        for kind, start, end, excl in attribute_launches(recs, H[r]):
+            e = kern.setdefault(kind, [0, 0.0])
             e[0] += 1
-            e[1] += max(t, 0) / 1e6
+            e[1] += excl / 1e6
     info = {"replays": R, "traced_ms_per_step": tot / R, "launches": len(recs)}
     return kern, info
+
+
+def attribute_launches(recs, stamps):
+    """Per traced launch (kind, start, end, exclusive ns) from one replay's stamps.
+
+    start = the earliest block's stamp past its dependency wait, end = the latest
+    block's exit stamp (blocks a launch did not use hold 0 and are ignored).  A
+    launch's exclusive time runs from the previous launch's end to its own end
+    (the first launch: from its own start), so kernels that overlap under
+    programmatic dependent launch are charged once and the exclusive times add up
+    to the traced span (first start to last end)."""
+    out = []
+    prev_end = None
+    for rec in recs:
+        blk = stamps[rec["offset"]:rec["offset"] + rec["blocks"] * rec["words"]].reshape(rec["blocks"], rec["words"])
+        used = blk[:, rec["exit_idx"]] != 0
+        if not used.any():
+            continue
+        start = int(blk[used, rec["wait_idx"]].min())
+        end = int(blk[used, rec["exit_idx"]].max())
+        excl = end - (prev_end if prev_end is not None else start)
+        prev_end = max(end, prev_end) if prev_end is not None else end
+        out.append((rec["kind"], start, end, max(excl, 0)))
+    return out
 
 
 def workload_description(w, B, T, g):

@@ -32,3 +32,31 @@ def test_reference_arm_prints_one_contract_line():
     w = I.preset("tiny")
     assert d["config"] == bench.config_of(w, 1, w.batch, w.context[0], w.gamma,
                                           bench.step_algorithmic_bytes(w, w.batch, w.gamma, w.context[0]))
+
+
+def test_trace_attribution_partitions_the_traced_span():
+    """bench.attribute_launches charges each launch from the previous launch's end to
+    its own end: overlapping launches (programmatic dependent launch) are charged
+    once, unused blocks (zero stamps) are ignored, and the shares add up to the span."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    recs, words, off = [], [], 0
+    # (kind, blocks, words per block, wait idx, exit idx, [(wait, exit) per used block])
+    plan = [("embed", 2, 2, 0, 1, [(100, 400), (120, 380)]),
+            ("gemm_qkv", 4, 8, 1, 6, [(300, 2000), (350, 2100), (0, 0), (500, 1900)]),   # starts before embed ends
+            ("attention", 2, 8, 1, 7, [(2050, 2600), (2100, 2700)]),
+            ("gemm_o", 3, 8, 1, 6, [(2400, 3500), (2600, 3300), (2500, 3600)])]
+    buf = []
+    for kind, blocks, w, wi, ei, st in plan:
+        recs.append({"kind": kind, "blocks": blocks, "words": w, "wait_idx": wi, "exit_idx": ei, "offset": off})
+        for a, b in st:
+            row = [0] * w
+            row[wi], row[ei] = a, b
+            buf.extend(row)
+        off += blocks * w
+    out = bench.attribute_launches(recs, np.array(buf, dtype=np.int64))
+    assert [o[0] for o in out] == ["embed", "gemm_qkv", "attention", "gemm_o"]
+    assert [(o[1], o[2]) for o in out] == [(100, 400), (300, 2100), (2050, 2700), (2400, 3600)]
+    assert [o[3] for o in out] == [300, 1700, 600, 900]
+    assert sum(o[3] for o in out) == 3600 - 100
