@@ -172,6 +172,13 @@ struct dflash_handle {
     // embedding and after every layer, and the final-norm rows.
     void* cap_x = nullptr;
     void* cap_hf = nullptr;
+    // per-layer stage captures (dflash_diag_draft_capture_stages), each [L][M][width]
+    void* cap_h = nullptr;     // normalised layer input (width H)
+    void* cap_q = nullptr;     // q (n_q_heads * d)
+    void* cap_o = nullptr;     // attention output (n_q_heads * d)
+    void* cap_xm = nullptr;    // residual stream after the O-projection (H)
+    void* cap_h2 = nullptr;    // normalised MLP input (H)
+    void* cap_act = nullptr;   // SwiGLU output (intermediate)
     // Diagnostic step trace (dflash_diag_step_trace): per-block %globaltimer
     // stamps of every traced launch, laid out one launch after the other.
     long long* tr_buf = nullptr;
@@ -268,6 +275,13 @@ void capture_x(dflash_handle* h, int slot, int M, cudaStream_t st) {
     const size_t es = h->cfg.dtype == DFLASH_BF16 ? 2 : 4;
     const size_t row = (size_t)M * h->cfg.hidden * es;
     cudaMemcpyAsync((uint8_t*)h->cap_x + (size_t)slot * row, h->x, row, cudaMemcpyDeviceToDevice, st);
+}
+// Diagnostic stage capture: rows x width elements of `src` into slot `layer` of dst.
+void capture_stage(dflash_handle* h, void* dst, const void* src, int layer, int M, int width, cudaStream_t st) {
+    if (!dst) return;
+    const size_t es = h->cfg.dtype == DFLASH_BF16 ? 2 : 4;
+    const size_t bytes = (size_t)M * width * es;
+    cudaMemcpyAsync((uint8_t*)dst + (size_t)layer * bytes, src, bytes, cudaMemcpyDeviceToDevice, st);
 }
 void capture_hf(dflash_handle* h, int Mlm, cudaStream_t st) {
     if (!h->cap_hf) return;
@@ -799,6 +813,7 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_in[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st,
                                trace_small(h, TK_RMSNORM, M));
             h->launches += 1;
+            capture_stage(h, h->cap_h, h->h, l, M, H, st);
         }
         {   // QKV + RoPE; block K/V to cache scratch rows [len, len + gamma)
             GemmParams p;
@@ -812,6 +827,10 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             p.n_amat = 3;
             p.tb[0] = fold ? tm_x : tm_h;
             if (fold) fold_in(h, p, h->w.g_in[l], l == 0 ? 1 : nH);   // layer 0: the embedding's row sums
+            if (fold && h->cap_h) {   // diagnostic: the normaliser also writes the rows it normalised
+                p.norm_out = (bf*)h->cap_h + (size_t)l * M * H;
+                p.norm_out_ld = H;
+            }
             p.kb_per_b = cdiv(H, 64);
             p.M = M;
             p.K = H;
@@ -835,6 +854,7 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             int r = run_gemm(h, p, nt, st, TK_GEMM_QKV);
             if (r) return r;
         }
+        capture_stage(h, h->cap_q, h->q, l, M, Nq, st);
         if (ingest && l == c.n_layers - 1) break;   // the last layer's K/V are written
         ap.layer = l;
         // attention trace: 8 stamps per CTA (attn.cuh), past the wait at 1, merge done at 7
@@ -844,6 +864,7 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             int e = launch_attention(ap, d, B, st, &h->launches);
             if (e) return DFLASH_CUDA;
         }
+        capture_stage(h, h->cap_o, h->o, l, M, Nq, st);
         {   // O-proj + residual
             GemmParams p;
             std::memset(&p, 0, sizeof(p));
@@ -865,11 +886,13 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             int r = run_gemm(h, p, nt, st, TK_GEMM_O);
             if (r) return r;
         }
+        capture_stage(h, h->cap_xm, h->x, l, M, H, st);
         if (!fold) {
             Timed t(h, TK_RMSNORM, st);
             launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_post[l], (bf*)h->h, M, H, (float)c.rms_eps, M, 0, 0, st,
                                trace_small(h, TK_RMSNORM, M));
             h->launches += 1;
+            capture_stage(h, h->cap_h2, h->h, l, M, H, st);
         }
         {   // gate/up + SwiGLU
             GemmParams p;
@@ -881,6 +904,10 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             p.n_tiles = I / 64;
             p.tb[0] = fold ? tm_x : tm_h;
             if (fold) fold_in(h, p, h->w.g_post[l], nH);
+            if (fold && h->cap_h2) {
+                p.norm_out = (bf*)h->cap_h2 + (size_t)l * M * H;
+                p.norm_out_ld = H;
+            }
             p.kb_per_b = cdiv(H, 64);
             p.M = M;
             p.K = H;
@@ -891,6 +918,7 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
             int r = run_gemm(h, p, nt, st, TK_GEMM_SWIGLU);
             if (r) return r;
         }
+        capture_stage(h, h->cap_act, h->act, l, M, I, st);
         {   // down + residual
             GemmParams p;
             std::memset(&p, 0, sizeof(p));
@@ -1258,6 +1286,18 @@ int dflash_diag_step_trace_records(const dflash_handle* h, int32_t* recs, int64_
         offsets[i] = r.offset;
     }
     *n_records = (int)h->tr_recs.size();
+    return DFLASH_OK;
+}
+
+int dflash_diag_draft_capture_stages(dflash_handle* h, void* h_in, void* q, void* o, void* x_mid, void* h2,
+                                     void* act) {
+    if (!h) return DFLASH_INVALID_ARG;
+    h->cap_h = h_in;
+    h->cap_q = q;
+    h->cap_o = o;
+    h->cap_xm = x_mid;
+    h->cap_h2 = h2;
+    h->cap_act = act;
     return DFLASH_OK;
 }
 

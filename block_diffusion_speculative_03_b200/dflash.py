@@ -114,6 +114,7 @@ def lib():
         "dflash_diag_attention_traced": (i32, [vp, vp, vp, vp, i32, i32, vp, C.POINTER(i32), vp]),
         "dflash_diag_gemm_bf16_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
         "dflash_diag_draft_capture": (i32, [vp, vp, vp]),
+        "dflash_diag_draft_capture_stages": (i32, [vp, vp, vp, vp, vp, vp, vp]),
         "dflash_diag_step_trace": (i32, [vp, vp, i64]),
         "dflash_diag_step_trace_records": (i32, [vp, C.POINTER(C.c_int32), C.POINTER(i64), i32, C.POINTER(i32)]),
         "dflash_diag_gemm_bf16_noalloc_status": (i32, [C.POINTER(C.c_int32), vp]),
@@ -145,6 +146,7 @@ def exported_symbols() -> list:
             "dflash_diag_wait_selftest",
             "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
             "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc", "dflash_diag_draft_capture",
+            "dflash_diag_draft_capture_stages",
             "dflash_diag_gemm_bf16_noalloc_status", "dflash_diag_step_trace", "dflash_diag_step_trace_records",
             "dflash_gamma_policy_init", "dflash_gamma_policy_observe", "dflash_gamma_policy_alpha",
             "dflash_gamma_policy_expected_tokens", "dflash_gamma_policy_choose"]
@@ -354,6 +356,11 @@ def dflash_diag_gemm_prefetch() -> int:
 
 def dflash_diag_set_norm_fold(on: bool) -> int:
     return _chk(lib().dflash_diag_set_norm_fold(1 if on else 0), "dflash_diag_set_norm_fold")
+
+
+def dflash_diag_draft_capture_stages(h: int, h_in=None, q=None, o=None, x_mid=None, h2=None, act=None) -> int:
+    return _chk(lib().dflash_diag_draft_capture_stages(h, h_in, q, o, x_mid, h2, act),
+                "dflash_diag_draft_capture_stages")
 
 
 def dflash_diag_wait_selftest(h: int, out: int, stream: int = 0) -> int:

@@ -158,6 +158,22 @@ int dflash_diag_step_trace_records(const dflash_handle* h, int32_t* recs, int64_
  * Not for use under CUDA-graph capture of a timed step (the copies are extra work). */
 int dflash_diag_draft_capture(dflash_handle* h, void* x_layers, void* hf);
 
+/* Capture of every layer's intermediate states (bf16 handles), for per-stage
+ * parity checks.  While set, every dflash_draft_block also writes, for each layer
+ * l, slot l (rows b*gamma + j, storage type) of:
+ *   h_in:  [n_layers][batch*gamma][hidden]       the normalised layer input R(RMSNorm(x) g_in)
+ *   q:     [n_layers][batch*gamma][n_q_heads*d]  the queries after RoPE
+ *   o:     [n_layers][batch*gamma][n_q_heads*d]  the attention output
+ *   x_mid: [n_layers][batch*gamma][hidden]       the residual stream after the O-projection
+ *   h2:    [n_layers][batch*gamma][hidden]       the normalised MLP input R(RMSNorm(x_mid) g_post)
+ *   act:   [n_layers][batch*gamma][intermediate] the SwiGLU output
+ * The block's own K/V of each layer stay in the cache rows [len, len + gamma).
+ * With the norms folded into the GEMMs, h_in and h2 are written by the GEMMs'
+ * normalising warp from the tiles the MMAs read.  Any pointer may be NULL;
+ * dflash_diag_draft_capture_stages(h, NULL, ...) stops.  Not for timed steps. */
+int dflash_diag_draft_capture_stages(dflash_handle* h, void* h_in, void* q, void* o, void* x_mid, void* h2,
+                                     void* act);
+
 /* Self-test of the device-side bounded wait used by the pipelined kernels: a
  * one-warp kernel waits on a shared-memory barrier that nothing arrives at.  The
  * wait gives up after its limit (about 2 s), records DFLASH_TIMEOUT in the

@@ -397,49 +397,50 @@ void oracle_ingest_fused_input(const oracle_config* c, const oracle_weights* w, 
 }
 
 // ---------------------------------------------------------------------------
-// a4..a6: one draft layer l on the block's hidden states x [gamma][H], in place.
-// Block position j sits at absolute position len + j.  Every block query sees
-// the whole committed context [0, len) of layer l (k_cache/v_cache, this
-// oracle's [L][nkv][cap][d] layout) and every block position (no mask).  The
-// block's own K/V are used for this pass only and are not written to the cache.
-//   h = R(RMSNorm(x) * g_in);  q = R(RoPE(h . Wq^T)), k = R(RoPE(h . Wk^T)), v = R(h . Wv^T)
-//   o = R(attention(q, [context K; k], [context V; v]))  (bf16 P when storage is bf16)
-//   x = R(x + o . Wo^T);  h2 = R(RMSNorm(x) * g_post)
-//   m = R(silu(h2 . Wg^T) * (h2 . Wu^T));  x = R(x + m . Wd^T)
+// a4..a6, one stage at a time (each exported, so a test can feed a stage its
+// input from elsewhere).  rows of the block: j = 0..gamma-1 at absolute
+// position len + j.
 // ---------------------------------------------------------------------------
-void oracle_draft_layer(const oracle_config* c, const oracle_weights* w, int l,
-                        const double* k_cache, const double* v_cache, int cap, int len,
-                        int gamma, double* x) {
+
+// RMSNorm of `rows` rows of width H with gain g (storage type), rounded:
+// out = R(RMSNorm(x) * g).
+void oracle_norm_rows(const oracle_config* c, const void* g_w, const double* x, int rows, double* out) {
+    int S = c->storage, H = c->hidden;
+    std::vector<double> g(H), tmp(H);
+    load_vec(g_w, H, S, g.data());
+    for (int j = 0; j < rows; ++j) {
+        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
+        for (int t = 0; t < H; ++t) out[(size_t)j * H + t] = R(tmp[t], S);
+    }
+}
+
+// a4: q = R(RoPE(h . Wq^T)), k = R(RoPE(h . Wk^T)), v = R(h . Wv^T) of layer l for
+// the normalised rows h [gamma][H]; q [gamma][nq*d], k, v [gamma][nkv*d].
+void oracle_layer_qkv(const oracle_config* c, const oracle_weights* w, int l, const double* h, int len,
+                      int gamma, double* q, double* k, double* v) {
     g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
-    int Nq = nq * d, Nkv = nkv * d, I = c->intermediate;
-    int n = len + gamma;
-    std::vector<double> g(H), h((size_t)gamma * H), tmp(H);
-    std::vector<double> q((size_t)gamma * Nq), kb((size_t)gamma * Nkv), vb((size_t)gamma * Nkv);
-    std::vector<double> K((size_t)nkv * n * d), Vv((size_t)nkv * n * d), o((size_t)gamma * Nq);
-    std::vector<double> y((size_t)gamma * H);
-    std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I);
-    size_t xs = (size_t)gamma * H;
-
-    // a4: h = R(RMSNorm(x) * g_in); q, k with RoPE at len + j; v.
-    load_vec(w->g_in[l], H, S, g.data());
-    for (int j = 0; j < gamma; ++j) {
-        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
-        for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
-    }
-    linear(h.data(), gamma, H, w->wq[l], Nq, S, q.data());
-    linear(h.data(), gamma, H, w->wk[l], Nkv, S, kb.data());
-    linear(h.data(), gamma, H, w->wv[l], Nkv, S, vb.data());
+    int Nq = nq * d, Nkv = nkv * d;
+    linear(h, gamma, H, w->wq[l], Nq, S, q);
+    linear(h, gamma, H, w->wk[l], Nkv, S, k);
+    linear(h, gamma, H, w->wv[l], Nkv, S, v);
     for (int j = 0; j < gamma; ++j) {
         long p = (long)len + j;
-        for (int hq = 0; hq < nq; ++hq) oracle_rope(q.data() + (size_t)j * Nq + (size_t)hq * d, d, p, c->rope_theta);
-        for (int g2 = 0; g2 < nkv; ++g2) oracle_rope(kb.data() + (size_t)j * Nkv + (size_t)g2 * d, d, p, c->rope_theta);
+        for (int hq = 0; hq < nq; ++hq) oracle_rope(q + (size_t)j * Nq + (size_t)hq * d, d, p, c->rope_theta);
+        for (int g2 = 0; g2 < nkv; ++g2) oracle_rope(k + (size_t)j * Nkv + (size_t)g2 * d, d, p, c->rope_theta);
     }
-    for (auto& e : q) e = R(e, S);
-    for (auto& e : kb) e = R(e, S);
-    for (auto& e : vb) e = R(e, S);
+    for (long i = 0; i < (long)gamma * Nq; ++i) q[i] = R(q[i], S);
+    for (long i = 0; i < (long)gamma * Nkv; ++i) { k[i] = R(k[i], S); v[i] = R(v[i], S); }
+}
 
-    // a5: keys/values = injected context rows [0, len) then the block rows.
+// a5: o = R(attention) of the block's queries q [gamma][nq*d] over layer l's
+// committed context rows [0, len) (k_cache/v_cache, [L][nkv][cap][d]) followed by
+// the block's own rows kb, vb [gamma][nkv*d] (no mask; bf16 P with bf16 storage).
+void oracle_layer_attention(const oracle_config* c, int l, const double* q, const double* kb, const double* vb,
+                            const double* k_cache, const double* v_cache, int cap, int len, int gamma, double* o) {
+    int S = c->storage, d = c->head_dim, nq = c->n_q_heads, nkv = c->n_kv_heads;
+    int Nkv = nkv * d, n = len + gamma;
+    std::vector<double> K((size_t)nkv * n * d), Vv((size_t)nkv * n * d);
     for (int g2 = 0; g2 < nkv; ++g2) {
         for (int i = 0; i < len; ++i)
             for (int t = 0; t < d; ++t) {
@@ -453,27 +454,59 @@ void oracle_draft_layer(const oracle_config* c, const oracle_weights* w, int l,
                 Vv[((size_t)g2 * n + len + j) * d + t] = vb[(size_t)j * Nkv + (size_t)g2 * d + t];
             }
     }
-    oracle_attention(q.data(), gamma, nq, K.data(), Vv.data(), n, nkv, d, S == 1, o.data());
-    for (auto& e : o) e = R(e, S);
+    oracle_attention(q, gamma, nq, K.data(), Vv.data(), n, nkv, d, S == 1, o);
+    for (long i = 0; i < (long)gamma * nq * d; ++i) o[i] = R(o[i], S);
+}
 
-    // a6: x = R(x + o.Wo^T); h2 = R(RMSNorm(x) * g_post);
-    //     m = R(silu(h2.Wg^T) * (h2.Wu^T)); x = R(x + m.Wd^T)
-    linear(o.data(), gamma, Nq, w->wo[l], H, S, y.data());
-    for (size_t i = 0; i < xs; ++i) x[i] = R(x[i] + y[i], S);
-    load_vec(w->g_post[l], H, S, g.data());
-    for (int j = 0; j < gamma; ++j) {
-        oracle_rmsnorm(x + (size_t)j * H, g.data(), H, c->rms_eps, tmp.data());
-        for (int t = 0; t < H; ++t) h[(size_t)j * H + t] = R(tmp[t], S);
-    }
-    linear(h.data(), gamma, H, w->w_gate[l], I, S, gt.data());
-    linear(h.data(), gamma, H, w->w_up[l], I, S, up.data());
+// a6, first half: x_out = R(x + o . Wo^T) for rows [gamma].
+void oracle_layer_oproj(const oracle_config* c, const oracle_weights* w, int l, const double* o, const double* x,
+                        int gamma, double* x_out) {
+    g_acc32 = c->acc32;
+    int S = c->storage, H = c->hidden, Nq = c->n_q_heads * c->head_dim;
+    std::vector<double> y((size_t)gamma * H);
+    linear(o, gamma, Nq, w->wo[l], H, S, y.data());
+    for (size_t i = 0; i < y.size(); ++i) x_out[i] = R(x[i] + y[i], S);
+}
+
+// a6, second half: m = R(silu(h2 . Wg^T) * (h2 . Wu^T)) for the normalised rows
+// h2 [gamma][H] (m [gamma][I] optional), then x_out = R(x + m . Wd^T).
+void oracle_layer_mlp(const oracle_config* c, const oracle_weights* w, int l, const double* h2, const double* x,
+                      int gamma, double* m_out, double* x_out) {
+    g_acc32 = c->acc32;
+    int S = c->storage, H = c->hidden, I = c->intermediate;
+    std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I), y((size_t)gamma * H);
+    linear(h2, gamma, H, w->w_gate[l], I, S, gt.data());
+    linear(h2, gamma, H, w->w_up[l], I, S, up.data());
     for (size_t i = 0; i < mm.size(); ++i) {
         double a = gt[i];
         double silu = a / (1.0 + std::exp(-a));
         mm[i] = R(silu * up[i], S);
     }
+    if (m_out) std::memcpy(m_out, mm.data(), sizeof(double) * mm.size());
     linear(mm.data(), gamma, I, w->w_down[l], H, S, y.data());
-    for (size_t i = 0; i < xs; ++i) x[i] = R(x[i] + y[i], S);
+    for (size_t i = 0; i < y.size(); ++i) x_out[i] = R(x[i] + y[i], S);
+}
+
+// ---------------------------------------------------------------------------
+// a4..a6: one draft layer l on the block's hidden states x [gamma][H], in place:
+//   h = R(RMSNorm(x) * g_in); q, k, v (oracle_layer_qkv); o (oracle_layer_attention);
+//   x = R(x + o . Wo^T); h2 = R(RMSNorm(x) * g_post); x = R(x + m . Wd^T) with the
+//   SwiGLU m (oracle_layer_mlp).  The block's own K/V are used for this pass only
+//   and are not written to the cache.
+// ---------------------------------------------------------------------------
+void oracle_draft_layer(const oracle_config* c, const oracle_weights* w, int l,
+                        const double* k_cache, const double* v_cache, int cap, int len,
+                        int gamma, double* x) {
+    int H = c->hidden, Nq = c->n_q_heads * c->head_dim, Nkv = c->n_kv_heads * c->head_dim;
+    size_t xs = (size_t)gamma * H;
+    std::vector<double> h(xs), q((size_t)gamma * Nq), kb((size_t)gamma * Nkv), vb((size_t)gamma * Nkv);
+    std::vector<double> o((size_t)gamma * Nq), xm(xs);
+    oracle_norm_rows(c, w->g_in[l], x, gamma, h.data());
+    oracle_layer_qkv(c, w, l, h.data(), len, gamma, q.data(), kb.data(), vb.data());
+    oracle_layer_attention(c, l, q.data(), kb.data(), vb.data(), k_cache, v_cache, cap, len, gamma, o.data());
+    oracle_layer_oproj(c, w, l, o.data(), x, gamma, xm.data());
+    oracle_norm_rows(c, w->g_post[l], xm.data(), gamma, h.data());
+    oracle_layer_mlp(c, w, l, h.data(), xm.data(), gamma, nullptr, x);
 }
 
 // a7 (second half): the shared LM head and argmax on already-normalised rows

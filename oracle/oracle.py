@@ -60,6 +60,12 @@ def lib():
                                          C.c_int, C.c_int, ip, dp, dp]
         L.oracle_draft_layer.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, C.c_int,
                                          C.c_int, dp]
+        L.oracle_norm_rows.argtypes = [C.POINTER(_Cfg), C.c_void_p, dp, C.c_int, dp]
+        L.oracle_layer_qkv.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, C.c_int, C.c_int, dp, dp, dp]
+        L.oracle_layer_attention.argtypes = [C.POINTER(_Cfg), C.c_int, dp, dp, dp, dp, dp, C.c_int, C.c_int,
+                                             C.c_int, dp]
+        L.oracle_layer_oproj.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, dp]
+        L.oracle_layer_mlp.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, dp, dp]
         L.oracle_embed_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, C.c_int, dp]
         L.oracle_final_norm.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, dp]
         L.oracle_lm_head.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, ip, dp, dp]
@@ -257,6 +263,55 @@ class OracleDrafter:
         lib().oracle_draft_layer(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(cache["k"]), _dp(cache["v"]),
                                  cache["cap"], cache["len"], gamma, _dp(y))
         return y
+
+    # -- one layer one stage at a time --------------------------------------
+    def norm_rows(self, gain: str, layer: int, x: np.ndarray) -> np.ndarray:
+        """R(RMSNorm(x) * g) of rows x [rows, hidden]; gain one of g_in, g_post (per
+        layer), g_final, g_fc."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        gp = getattr(self.w, gain)[layer] if gain in ("g_in", "g_post") else getattr(self.w, gain)
+        out = np.empty_like(x)
+        lib().oracle_norm_rows(C.byref(self.cfg), gp, _dp(x), x.shape[0], _dp(out))
+        return out
+
+    def layer_qkv(self, layer: int, h: np.ndarray, pos0: int):
+        """q [rows, nq*d], k, v [rows, nkv*d] of normalised rows h at positions pos0 + j."""
+        s = self.shape
+        h = np.ascontiguousarray(h, dtype=np.float64)
+        g = h.shape[0]
+        q = np.empty((g, s["n_q_heads"] * s["head_dim"]))
+        k = np.empty((g, s["n_kv_heads"] * s["head_dim"]))
+        v = np.empty_like(k)
+        lib().oracle_layer_qkv(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(h), int(pos0), g, _dp(q),
+                               _dp(k), _dp(v))
+        return q, k, v
+
+    def layer_attention(self, cache: Dict, layer: int, q: np.ndarray, kb: np.ndarray, vb: np.ndarray) -> np.ndarray:
+        """o [rows, nq*d]: the block queries over the cache's committed rows then the block's kb, vb."""
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        kb = np.ascontiguousarray(kb, dtype=np.float64)
+        vb = np.ascontiguousarray(vb, dtype=np.float64)
+        o = np.empty_like(q)
+        lib().oracle_layer_attention(C.byref(self.cfg), int(layer), _dp(q), _dp(kb), _dp(vb), _dp(cache["k"]),
+                                     _dp(cache["v"]), cache["cap"], cache["len"], q.shape[0], _dp(o))
+        return o
+
+    def layer_oproj(self, layer: int, o: np.ndarray, x: np.ndarray) -> np.ndarray:
+        o = np.ascontiguousarray(o, dtype=np.float64)
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty_like(x)
+        lib().oracle_layer_oproj(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(o), _dp(x), x.shape[0], _dp(out))
+        return out
+
+    def layer_mlp(self, layer: int, h2: np.ndarray, x: np.ndarray):
+        """(m [rows, intermediate], x_out [rows, hidden])."""
+        h2 = np.ascontiguousarray(h2, dtype=np.float64)
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        m = np.empty((x.shape[0], self.shape["intermediate"]))
+        out = np.empty_like(x)
+        lib().oracle_layer_mlp(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(h2), _dp(x), x.shape[0], _dp(m),
+                               _dp(out))
+        return m, out
 
     def final_norm(self, x: np.ndarray) -> np.ndarray:
         """hf rows of the mask positions 1..gamma-1 of x [gamma, hidden]."""

@@ -10,9 +10,17 @@ run on the GPU's own input to that stage, so that a rounding flip inherited
 from an earlier stage cannot hide, or be mistaken for, a fault in the stage
 under test.  The draft step is captured through dflash_diag_draft_capture (the
 residual stream after the embedding and after every layer, and the final-norm
-rows the LM head reads):
+rows the LM head reads) and dflash_diag_draft_capture_stages (every layer's
+normalised input, q, attention output, residual after the O-projection,
+normalised MLP input and SwiGLU output; the block's own K/V stay in the cache):
   embedding          oracle embed of the anchor/mask tokens      vs GPU x_0 (exact)
-  layer l            oracle layer l on GPU x_l and the GPU cache  vs GPU x_{l+1}
+  layer l, stage by stage, each from the GPU's input to it:
+    input norm       oracle norm of GPU x_l                       vs GPU h
+    QKV + RoPE       oracle QKV of GPU h                          vs GPU q, block k, v
+    attention        oracle attention of GPU q, k, v + GPU cache  vs GPU o
+    O-proj + resid.  oracle O-proj of GPU o onto GPU x_l          vs GPU x_mid
+    MLP norm         oracle norm of GPU x_mid                     vs GPU h2
+    SwiGLU MLP       oracle MLP of GPU h2 onto GPU x_mid          vs GPU act, x_{l+1}
   final norm         oracle final norm of GPU x_L                 vs GPU hf
   LM head + argmax   oracle LM head on GPU hf                     vs GPU logits / drafts
   fuse               oracle fuse of the same target hidden rows   vs GPU ctx
@@ -102,28 +110,60 @@ class Rig:
         Returns the GPU's drafts [B, g-1] and the number of draft tokens compared."""
         w, dr = self.w, self.dr
         B, H, L, nd = w.batch, w.hidden, w.n_layers, g - 1
-        X = torch.empty(L + 1, B * g, H, dtype=torch.bfloat16, device="cuda")
-        HF = torch.empty(max(B * nd, 1), H, dtype=torch.bfloat16, device="cuda")
+        Nq, Nkv, d = w.n_q_heads * w.head_dim, w.n_kv_heads * w.head_dim, w.head_dim
+        M = B * g
+        bf = dict(dtype=torch.bfloat16, device="cuda")
+        X = torch.empty(L + 1, M, H, **bf)
+        HF = torch.empty(max(B * nd, 1), H, **bf)
+        ST = {"h": torch.empty(L, M, H, **bf), "q": torch.empty(L, M, Nq, **bf), "o": torch.empty(L, M, Nq, **bf),
+              "x_mid": torch.empty(L, M, H, **bf), "h2": torch.empty(L, M, H, **bf),
+              "act": torch.empty(L, M, w.intermediate, **bf)}
         logits = torch.empty(B, nd, w.vocab, dtype=torch.float32, device="cuda")
         margin = torch.empty(B, nd, dtype=torch.float32, device="cuda")
         D.dflash_diag_draft_capture(dr.handle, X.data_ptr(), HF.data_ptr())
+        D.dflash_diag_draft_capture_stages(dr.handle, *[ST[k].data_ptr() for k in ("h", "q", "o", "x_mid", "h2",
+                                                                                   "act")])
         try:
             drafts = dr.draft_block(self.cache, torch.tensor(anchors, dtype=torch.int32, device="cuda"), g,
                                     logits=logits, margin=margin)
             torch.cuda.synchronize()
         finally:
             D.dflash_diag_draft_capture(dr.handle, None, None)
+            D.dflash_diag_draft_capture_stages(dr.handle)
         assert self.cache.status() == 0
         g_dr = drafts.cpu().numpy()[:, :nd]
         assert np.all((g_dr >= 0) & (g_dr < w.vocab))
+        slab = self.cache.slab()
+        lens = self.cache.len.cpu().numpy()
         compared = 0
         for b in sample:
             oc = self.oracle_cache(b)
-            xs = X[:, b * g:(b + 1) * g].double().cpu().numpy()          # [L+1, g, H]
+            rows = slice(b * g, (b + 1) * g)
+            xs = X[:, rows].double().cpu().numpy()          # [L+1, g, H]
+            st = {k: v[:, rows].double().cpu().numpy() for k, v in ST.items()}
             assert np.array_equal(xs[0], self.od.embed_block(int(anchors[b]), g)), "embedding"
+            n0 = int(lens[b])
             for l in range(L):
-                y = self.od.draft_layer(oc, l, xs[l])
-                check_state(xs[l + 1], y, "x[layer %d, b %d, gamma %d]" % (l, b, g))
+                tag = "[layer %d, b %d, gamma %d]" % (l, b, g)
+                od = self.od
+                # every stage of the layer from the GPU's own input to it
+                check_state(st["h"][l], od.norm_rows("g_in", l, xs[l]), "h" + tag)
+                q_o, k_o, v_o = od.layer_qkv(l, st["h"][l], n0)
+                kb = slab[b, l, 0, :, n0:n0 + g].double().cpu().numpy().transpose(1, 0, 2).reshape(g, Nkv)
+                vb = slab[b, l, 1, :, n0:n0 + g].double().cpu().numpy().transpose(1, 0, 2).reshape(g, Nkv)
+                check_state(st["q"][l], q_o, "q" + tag)
+                check_state(kb, k_o, "k" + tag)
+                check_state(vb, v_o, "v" + tag)
+                check_state(st["o"][l], od.layer_attention(oc, l, st["q"][l], kb, vb), "o" + tag)
+                check_state(st["x_mid"][l], od.layer_oproj(l, st["o"][l], xs[l]), "x_mid" + tag)
+                check_state(st["h2"][l], od.norm_rows("g_post", l, st["x_mid"][l]), "h2" + tag)
+                m_o, x_o = od.layer_mlp(l, st["h2"][l], st["x_mid"][l])
+                check_state(st["act"][l], m_o, "act" + tag)
+                check_state(xs[l + 1], x_o, "x" + tag)
+                # the whole layer from its input: bf16 flips inside the layer cascade
+                # through the MLP (fp64 vs fp32 accumulation alone leaves ~70 % of the
+                # outputs identical), so only the error bound is held here
+                check_state(xs[l + 1], od.draft_layer(oc, l, xs[l]), "layer" + tag, min_same=0.0)
             hf_g = HF[b * nd:(b + 1) * nd].double().cpu().numpy()
             check_state(hf_g, self.od.final_norm(xs[L]), "hf[b %d]" % b)
             d_o, m_o, l_o = self.od.lm_head(hf_g)

@@ -304,3 +304,22 @@ def test_piecewise_draft_equals_one_call(dtype):
     hf = od.final_norm(x)
     d2, m2, l2 = od.lm_head(hf)
     assert np.array_equal(d2, drafts) and np.array_equal(m2, margin) and np.array_equal(l2, logits)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layer_stages_compose_to_the_layer(dtype):
+    # norm -> qkv -> attention -> O-proj -> norm -> MLP, one stage at a time (the form
+    # the per-stage GPU parity tests feed the GPU's own inputs to), equals one layer call
+    w = micro(dtype)
+    W = I.make_weights(w)
+    hid = I.make_hiddens(w, 20)
+    od, ctx, cache, drafts, margin, logits = _run_oracle(w, W, hid, 5, 11)
+    x = od.embed_block(11, 5)
+    for l in range(w.n_layers):
+        h = od.norm_rows("g_in", l, x)
+        q, k, v = od.layer_qkv(l, h, cache["len"])
+        o = od.layer_attention(cache, l, q, k, v)
+        xm = od.layer_oproj(l, o, x)
+        m, x2 = od.layer_mlp(l, od.norm_rows("g_post", l, xm), xm)
+        assert np.array_equal(x2, od.draft_layer(cache, l, x))
+        x = x2
