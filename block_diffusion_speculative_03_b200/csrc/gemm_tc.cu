@@ -26,7 +26,8 @@ struct GemmCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int CH = NT < 32 ? NT : 32;         // epilogue column chunk
     static constexpr int XCH_FLOATS = 128 * (CH + 1);
-    static constexpr int MISC_BYTES = 6144;
+    static constexpr int GAIN_MAX = 4096;                // RMSNorm gain elements staged in shared memory
+    static constexpr int MISC_BYTES = 6144 + GAIN_MAX * 2;
     static constexpr int SMEM_CAP = TWO_PER_SM ? (233472 / 2 - 2048) : 232448;
     static constexpr int BUDGET = SMEM_CAP - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
     static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
@@ -101,7 +102,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
     float* inv_s = lmred + 4 * CH * 3;       // [NT] inverse RMS of the current m-tile's rows
     uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
-    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + NT * 4 + 8 + S * 8 <= C::MISC_BYTES, "misc");
+    __nv_bfloat16* sgain = (__nv_bfloat16*)(((uintptr_t)(ready + S) + 15) & ~(uintptr_t)15);   // [GAIN_MAX]
+    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+                      C::MISC_BYTES, "misc");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 8 : nullptr;
@@ -262,6 +265,15 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     } else if (warp == 6) {
         // ------------------------------------------------------------ B normaliser
         if (p.ssq_in) {
+            // The gain is a weight (independent of the previous kernel): stage it in
+            // shared memory before the dependency wait, so no stage waits on a
+            // global load of its slice.
+            const bool gain_smem = p.K <= C::GAIN_MAX;
+            if (gain_smem) {
+                for (int i = lane * 8; i < p.K; i += 32 * 8)
+                    *reinterpret_cast<uint4*>(sgain + i) = __ldg(reinterpret_cast<const uint4*>(p.gain + i));
+                __syncwarp();
+            }
             griddep_wait();
             int stage = 0, cur_mt = -1;
             uint32_t round = 0;
@@ -297,7 +309,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                         const int f0 = kb * 64 + 8 * (j ^ (r & 7));
                         uint4* ptr = reinterpret_cast<uint4*>(bt + r * 128 + j * 16);
                         const uint4 xv = *ptr;
-                        const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gain + f0));
+                        const uint4 gv = gain_smem ? *reinterpret_cast<const uint4*>(sgain + f0)
+                                                   : __ldg(reinterpret_cast<const uint4*>(p.gain + f0));
                         const __nv_bfloat16* xe = reinterpret_cast<const __nv_bfloat16*>(&xv);
                         const __nv_bfloat16* ge = reinterpret_cast<const __nv_bfloat16*>(&gv);
                         const float inv = inv_s[r];
@@ -324,6 +337,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
         const int row = q * 32 + lane;          // weight-tile row = TMEM lane
         const int e = threadIdx.x - 64;         // 0..127
         int seg = 0;
+        int tok_mt = -1;                        // m-tile whose token map tok_b / tok_pos holds
         for (long long u = u_begin; u < u_end;) {
             const long long t = u / KB;
             const int kb0 = (int)(u % KB);
@@ -331,6 +345,72 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
             const int n_tile = (int)(t / m_tiles), m_tile = (int)(t % m_tiles);
             const int buf = seg & 1;
             const uint32_t use = (uint32_t)(seg >> 1);
+            // Everything the epilogue needs that does not depend on this tile's sums is
+            // gathered while the tile still accumulates, so that the finishing path
+            // after the last MMA holds as few dependent memory round trips as possible:
+            // the per-token request / position map of the cache-writing epilogues ...
+            if ((p.epi == EPI_QKV || p.epi == EPI_INJECT) && m_tile != tok_mt) {
+                named_bar_sync(1, 128);   // the previous tile's readers of the map are done
+                if (p.epi == EPI_QKV) {
+                    for (int te = e; te < NT; te += 128) {   // NT may exceed the 128 epilogue threads
+                        const int m = m_tile * NT + te;
+                        int b = -1, pos = -1;
+                        if (m < p.M) {
+                            const int bb = m / p.gamma;
+                            if (p.req_ok[bb]) { b = bb; pos = p.len[bb] + (m - bb * p.gamma); }
+                        }
+                        if (pos < 0 || pos >= p.cap) b = -1;   // never write outside the request's slab
+                        tok_b[te] = b;
+                        tok_pos[te] = pos;
+                    }
+                } else {
+                    // one thread per request marks the rows it owns in this m-tile
+                    for (int te = e; te < NT; te += 128) tok_b[te] = -1;
+                    named_bar_sync(1, 128);
+                    const int m0 = p.row0 + m_tile * NT;   // global row of the tile's first column
+                    for (int bb = e; bb < p.batch; bb += 128) {
+                        const int rs = p.row_start[bb], rc = p.row_count[bb], L0 = p.len[bb];
+                        if (rc <= 0 || L0 < 0 || L0 + rc > p.cap) continue;
+                        const int lo = max(rs, m0), hi = min(min(rs + rc, m0 + NT), p.row0 + p.M);
+                        for (int m = lo; m < hi; ++m) {
+                            tok_b[m - m0] = bb;
+                            tok_pos[m - m0] = L0 + (m - rs);
+                        }
+                    }
+                }
+                named_bar_sync(1, 128);
+                tok_mt = m_tile;
+            }
+            // ... the weight-row -> output-feature mapping of this tile ...
+            int mi = 0;
+            if (!p.swiglu)
+                while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
+            const int lr = p.swiglu ? 0 : (n_tile - p.amat[mi].tile0) * 128 + row;
+            const bool row_ok = p.swiglu ? true : (lr < p.amat[mi].rows);
+            // ... and, for single-chunk tiles, the residual rows or the RoPE cos/sin
+            // of the thread's output feature (only a finisher uses them).
+            constexpr bool PRE = NT <= 16;
+            float pre_x[PRE ? CH : 1];
+            float2 pre_cs[PRE ? CH : 1];
+            if constexpr (PRE) {
+                if (p.epi == EPI_RESID) {
+                    const __nv_bfloat16* o = (const __nv_bfloat16*)p.out;
+#pragma unroll
+                    for (int i = 0; i < CH; ++i) {
+                        const int m = m_tile * NT + i;
+                        pre_x[i] = (row_ok && m < p.M) ? bf2f(o[(size_t)m * p.ldo + lr]) : 0.f;
+                    }
+                } else if (p.epi == EPI_QKV || p.epi == EPI_INJECT) {
+                    // rotated sections: q and k of the QKV GEMM (matrices 0, 1), K of each layer in
+                    // the injection GEMM (even matrices); the same rule as the epilogue's `rotate`
+                    const bool rot = p.epi == EPI_QKV ? mi <= 1 : (mi & 1) == 0;
+                    const int half = p.d >> 1, ih = (lr % p.d) % half;
+#pragma unroll
+                    for (int i = 0; i < CH; ++i)
+                        pre_cs[i] = (rot && row_ok && tok_b[i] >= 0) ? __ldg(&p.rope[(size_t)tok_pos[i] * half + ih])
+                                                                     : make_float2(1.f, 0.f);
+                }
+            }
             const bool ok = mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
             if (named_bar_or(1, 128, !ok)) break;   // leave together: later named barriers stay matched
             if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
@@ -353,56 +433,22 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) __stcg(dst + (c0 + i) * 128 + row, v[i]);
                 }
-                __threadfence();
+                // Release the CTA's partial and count it: the barrier orders every
+                // thread's stores before one thread's gpu-scope fence and atomic; the
+                // last arriver's fence (acquire side) and the barrier after it make the
+                // other contributors' partials visible to all its threads.
                 named_bar_sync(1, 128);
                 if (e == 0) {
-                    int old = atomicAdd(&p.counters[t], 1);
-                    *s_flag = (old == nc - 1) ? 1 : 0;
+                    __threadfence();
+                    const int old = atomicAdd(&p.counters[t], 1);
+                    const bool last = old == nc - 1;
+                    if (last) __threadfence();
+                    *s_flag = last ? 1 : 0;
                 }
                 named_bar_sync(1, 128);
                 finish = (*s_flag != 0);
-                if (finish) __threadfence();
             }
             if (finish) {
-                // Weight-row -> output-feature mapping of this tile.
-                int mi = 0;
-                if (!p.swiglu)
-                    while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
-                const int lr = p.swiglu ? 0 : (n_tile - p.amat[mi].tile0) * 128 + row;
-                const bool row_ok = p.swiglu ? true : (lr < p.amat[mi].rows);
-                // Per-token request / position for the cache-writing epilogues.
-                if (p.epi == EPI_QKV) {
-                    named_bar_sync(1, 128);
-                    for (int te = e; te < NT; te += 128) {   // NT may exceed the 128 epilogue threads
-                        const int m = m_tile * NT + te;
-                        int b = -1, pos = -1;
-                        if (m < p.M) {
-                            const int bb = m / p.gamma;
-                            if (p.req_ok[bb]) { b = bb; pos = p.len[bb] + (m - bb * p.gamma); }
-                        }
-                        if (pos < 0 || pos >= p.cap) b = -1;   // never write outside the request's slab
-                        tok_b[te] = b;
-                        tok_pos[te] = pos;
-                    }
-                    named_bar_sync(1, 128);
-                } else if (p.epi == EPI_INJECT) {
-                    // One thread per request marks the rows it owns in this m-tile
-                    // (independent loads; no per-token search over the batch).
-                    named_bar_sync(1, 128);
-                    for (int te = e; te < NT; te += 128) tok_b[te] = -1;
-                    named_bar_sync(1, 128);
-                    const int m0 = p.row0 + m_tile * NT;   // global row of the tile's first column
-                    for (int bb = e; bb < p.batch; bb += 128) {
-                        const int rs = p.row_start[bb], rc = p.row_count[bb], L0 = p.len[bb];
-                        if (rc <= 0 || L0 < 0 || L0 + rc > p.cap) continue;
-                        const int lo = max(rs, m0), hi = min(min(rs + rc, m0 + NT), p.row0 + p.M);
-                        for (int m = lo; m < hi; ++m) {
-                            tok_b[m - m0] = bb;
-                            tok_pos[m - m0] = L0 + (m - rs);
-                        }
-                    }
-                    named_bar_sync(1, 128);
-                }
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += CH) {
                     float v[CH];
@@ -469,9 +515,14 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                         // so the loads are not serialised behind the stores.
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
                         float rv[CH];
+                        if constexpr (PRE) {
 #pragma unroll
-                        for (int i = 0; i < CH; ++i)
-                            rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+                            for (int i = 0; i < CH; ++i) rv[i] = pre_x[i];
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < CH; ++i)
+                                rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+                        }
                         float sq[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) {
@@ -520,11 +571,17 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                         if (row_ok) {
                             // cos/sin of every column first (independent loads), then the stores
                             float2 cs[CH];
+                            if constexpr (PRE) {
 #pragma unroll
-                            for (int i = 0; i < CH; ++i) {
-                                const int b = tok_b[c0 + i];
-                                cs[i] = (rotate && b >= 0) ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
-                                                           : make_float2(1.f, 0.f);
+                                for (int i = 0; i < CH; ++i) cs[i] = pre_cs[i];
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < CH; ++i) {
+                                    const int b = tok_b[c0 + i];
+                                    cs[i] = (rotate && b >= 0)
+                                                ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
+                                                : make_float2(1.f, 0.f);
+                                }
                             }
 #pragma unroll
                             for (int i = 0; i < CH; ++i) {
