@@ -83,9 +83,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     // After the key loop the ring holds this CTA's partial.
     float* po = (float*)smem;                      // [128][PO_LD] lanes' O, then rows 0..RW-1 summed
     float2* pml = (float2*)(po + 128 * PO_LD);     // [128] (integer base, row sum)
-    float* cm = (float*)(pml + 128);               // [128][splits] peers' bases
-    float* cl = cm + 128 * kAttnMaxSplits;         // [128][splits] peers' sums
-    float* cw = cl + 128 * kAttnMaxSplits;         // [128][splits] merge weights
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -240,12 +237,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             const __nv_bfloat16* qsrc =
                 row < R ? p.q + ((size_t)(b * p.gamma + row / p.G) * p.nq + (size_t)(g * p.G + row % p.G)) * D
                         : nullptr;
-#pragma unroll 1
+            // the whole row in one batch of independent loads (one memory round trip),
+            // then into tensor memory 16 columns (32 elements) at a time
+            uint4 qv[D / 8];
+#pragma unroll
+            for (int k = 0; k < D / 8; ++k)
+                qv[k] = qsrc ? *reinterpret_cast<const uint4*>(qsrc + 8 * k) : make_uint4(0, 0, 0, 0);
+#pragma unroll
             for (int c0 = 0; c0 < D / 2; c0 += 16) {   // columns c0..c0+15 = elements 2*c0..2*c0+31
                 float v[16];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint4 u = qsrc ? *reinterpret_cast<const uint4*>(qsrc + 2 * c0 + 8 * k) : make_uint4(0, 0, 0, 0);
+                    const uint4 u = qv[c0 / 4 + k];
                     v[4 * k + 0] = __uint_as_float(u.x);
                     v[4 * k + 1] = __uint_as_float(u.y);
                     v[4 * k + 2] = __uint_as_float(u.z);
@@ -453,45 +456,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         rpo[s2] = s2 < nsplit ? cluster.map_shared_rank(po, s2) : po;
         rpml[s2] = s2 < nsplit ? cluster.map_shared_rank(pml, s2) : pml;
     }
+    // One round of distributed-shared-memory reads per output chunk: each thread
+    // fetches every split's (base, sum) of its row and O chunk together, and forms
+    // the row's merge weights itself (exact powers of two times 1 / the merged sum).
     const int nr = r_hi - r_lo;
-    for (int idx = tid; idx < nr * nsplit; idx += kAttnThreads) {
-        const int r = r_lo + idx / nsplit, s2 = idx % nsplit;
-        const float2 ml = rpml[s2][r];
-        cm[idx] = ml.x;
-        cl[idx] = ml.y;
-    }
-    __syncthreads();
-    for (int rr = tid; rr < nr; rr += kAttnThreads) {
-        float M = -INFINITY;
-        for (int s2 = 0; s2 < nsplit; ++s2)
-            if (cl[rr * nsplit + s2] > 0.f) M = fmaxf(M, cm[rr * nsplit + s2]);
-        const float bm = (M == -INFINITY) ? 0.f : M;
-        float L = 0.f;
-        for (int s2 = 0; s2 < nsplit; ++s2) {
-            const float lv = cl[rr * nsplit + s2];
-            const float wv = lv > 0.f ? exp2f(cm[rr * nsplit + s2] - bm) : 0.f;
-            cw[rr * nsplit + s2] = wv;
-            L += wv * lv;
-        }
-        const float inv = L > 0.f ? 1.0f / L : 0.f;
-        for (int s2 = 0; s2 < nsplit; ++s2) cw[rr * nsplit + s2] *= inv;
-    }
-    __syncthreads();
     for (int idx = tid; idx < nr * (D / 4); idx += kAttnThreads) {
         const int rr = idx / (D / 4), c = (idx % (D / 4)) * 4, r = r_lo + rr;
+        float2 ml[kAttnMaxSplits];
         float4 v[kAttnMaxSplits];
 #pragma unroll
-        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+            ml[s2] = s2 < nsplit ? rpml[s2][r] : make_float2(0.f, 0.f);
             v[s2] = s2 < nsplit ? *reinterpret_cast<const float4*>(rpo[s2] + r * PO_LD + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
+            if (s2 < nsplit && ml[s2].y > 0.f) M = fmaxf(M, ml[s2].x);
+        const float bm = (M == -INFINITY) ? 0.f : M;
+        float wv[kAttnMaxSplits];
+        float L = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+            wv[s2] = (s2 < nsplit && ml[s2].y > 0.f) ? exp2f(ml[s2].x - bm) : 0.f;
+            L += wv[s2] * ml[s2].y;
+        }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
             if (s2 < nsplit) {
-                const float wv = cw[rr * nsplit + s2];
-                acc.x += wv * v[s2].x;
-                acc.y += wv * v[s2].y;
-                acc.z += wv * v[s2].z;
-                acc.w += wv * v[s2].w;
+                const float w = wv[s2] * inv;
+                acc.x += w * v[s2].x;
+                acc.y += w * v[s2].y;
+                acc.z += w * v[s2].z;
+                acc.w += w * v[s2].w;
             }
         }
         const int j = r / p.G, hh = r % p.G;

@@ -48,6 +48,8 @@ struct GemmParams {
     int n_tiles, m_tiles;
     long long units;             // n_tiles * m_tiles * KB
     int ctas;
+    int whole_tiles;             // 1: CTAs take whole output tiles (no split-K): every output is one
+                                 //    in-order accumulation over all of K, whatever M and the grid
     int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
     float* partial;              // [2 * ctas][NT][128] fp32 split-tile partials
     int* counters;               // [n_tiles * m_tiles], zero between launches

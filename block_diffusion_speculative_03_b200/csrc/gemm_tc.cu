@@ -1,12 +1,12 @@
 // Persistent split-K tcgen05 GEMM with fused epilogues (see gemm.cuh).
 //
-// CTA = 7 warps:  warp 0 lane 0 issues TMA loads of (weight tile, token tile)
+// CTA = 8 warps:  warp 0 lane 0 issues TMA loads of (weight tile, token tile)
 // pairs into an S-stage shared-memory ring; warp 1 lane 0 issues tcgen05.mma
 // (M=128, N=NT, K=16, bf16 in, fp32 accumulate) into one of two TMEM
 // accumulator buffers; warps 2..5 (128 threads, one TMEM lane each) drain a
 // finished accumulator with tcgen05.ld, resolve split tiles, and run the
-// epilogue while the next tile accumulates in the other buffer; warp 6, when
-// the GEMM consumes RMS-normalised rows, rewrites each token tile in shared
+// epilogue while the next tile accumulates in the other buffer; warps 6 and 7,
+// when the GEMM consumes RMS-normalised rows, rewrite each token tile in shared
 // memory as R(x * inv_rms * gain) between its arrival and the MMA.
 #include "gemm.cuh"
 
@@ -19,7 +19,7 @@ constexpr long long kGemmMaxGrid = 160;
 // that fits (two CTAs per SM with half the ring measured slower at batch 1).
 template <int NT>
 struct GemmCfg {
-    static constexpr int THREADS = 224;
+    static constexpr int THREADS = 256;
     static constexpr bool TWO_PER_SM = false;
     static constexpr int A_BYTES = 128 * 128;            // 128 rows x 64 bf16
     static constexpr int B_BYTES = NT * 128;             // NT rows x 64 bf16
@@ -100,10 +100,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     int* tok_b = s_flag + 1;          // [NT]
     int* tok_pos = tok_b + NT;        // [NT]
     float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
-    float* inv_s = lmred + 4 * CH * 3;       // [NT] inverse RMS of the current m-tile's rows
-    uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
+    float* inv_s = lmred + 4 * CH * 3;       // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
+    uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + 2 * NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
     __nv_bfloat16* sgain = (__nv_bfloat16*)(((uintptr_t)(ready + S) + 15) & ~(uintptr_t)15);   // [GAIN_MAX]
-    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
                       C::MISC_BYTES, "misc");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 128);
         }
-        for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 32);
+        for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 2);   // one arrival per normaliser warp
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -135,7 +135,12 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
 
     const long long U = p.units;
     const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
-    const long long u_begin = sk_begin(cta, U, P), u_end = sk_begin(cta + 1, U, P);
+    long long u_begin = sk_begin(cta, U, P), u_end = sk_begin(cta + 1, U, P);
+    if (p.whole_tiles) {   // tile-granular ranges: no tile is split, no partials
+        const long long T = U / KB;
+        u_begin = (T * cta / P) * KB;
+        u_end = (T * (cta + 1) / P) * KB;
+    }
 
     griddep_launch();
     if (warp == 0) {
@@ -262,18 +267,19 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                 mbar_wait(drain, 0, &never, nullptr);
             }
         }
-    } else if (warp == 6) {
-        // ------------------------------------------------------------ B normaliser
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ B normalisers (warps 6, 7)
         if (p.ssq_in) {
+            const int nl = (warp - 6) * 32 + lane;   // 0..63 over the two warps
+            float* inv_w = inv_s + (warp - 6) * NT;
             // The gain is a weight (independent of the previous kernel): stage it in
             // shared memory before the dependency wait, so no stage waits on a
             // global load of its slice.
             const bool gain_smem = p.K <= C::GAIN_MAX;
-            if (gain_smem) {
-                for (int i = lane * 8; i < p.K; i += 32 * 8)
+            if (gain_smem)
+                for (int i = nl * 8; i < p.K; i += 64 * 8)
                     *reinterpret_cast<uint4*>(sgain + i) = __ldg(reinterpret_cast<const uint4*>(p.gain + i));
-                __syncwarp();
-            }
+            named_bar_sync(2, 64);   // the staged gain; the only barrier between the two warps
             griddep_wait();
             int stage = 0, cur_mt = -1;
             uint32_t round = 0;
@@ -287,13 +293,16 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                 const bool copy_out = p.norm_out && t / m_tiles == 0;
                 if (m_tile != cur_mt) {
                     // inverse RMS of the m-tile's rows from the producer's per-tile
-                    // partial sums, added in tile order (the same in every CTA)
+                    // partial sums, added in tile order (the same in every CTA); each
+                    // warp keeps its own copy, so the two warps never wait for each other
+                    // inside the stage loop
+                    __syncwarp();
                     for (int r = lane; r < NT; r += 32) {
                         const int m = m_tile * NT + r;
                         float ss = 0.f;
                         if (m < p.M)
                             for (int j = 0; j < p.ssq_tiles; ++j) ss += __ldcg(p.ssq_in + (size_t)j * p.ssq_ld + m);
-                        inv_s[r] = 1.0f / sqrtf(ss / (float)p.norm_h + p.eps);
+                        inv_w[r] = 1.0f / sqrtf(ss / (float)p.norm_h + p.eps);
                     }
                     __syncwarp();
                     cur_mt = m_tile;
@@ -304,7 +313,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                     // its 16-byte chunk j holds elements 8 (j ^ (r & 7)) .. + 7 of the k-block
                     uint8_t* bt = sB + stage * C::B_BYTES;
 #pragma unroll 2
-                    for (int ch = lane; ch < NT * 8; ch += 32) {
+                    for (int ch = nl; ch < NT * 8; ch += 64) {
                         const int r = ch >> 3, j = ch & 7;
                         const int f0 = kb * 64 + 8 * (j ^ (r & 7));
                         uint4* ptr = reinterpret_cast<uint4*>(bt + r * 128 + j * 16);
@@ -313,7 +322,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                                                    : __ldg(reinterpret_cast<const uint4*>(p.gain + f0));
                         const __nv_bfloat16* xe = reinterpret_cast<const __nv_bfloat16*>(&xv);
                         const __nv_bfloat16* ge = reinterpret_cast<const __nv_bfloat16*>(&gv);
-                        const float inv = inv_s[r];
+                        const float inv = inv_w[r];
                         uint4 out;
                         __nv_bfloat16* oe = reinterpret_cast<__nv_bfloat16*>(&out);
 #pragma unroll
@@ -324,7 +333,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                             *reinterpret_cast<uint4*>(p.norm_out + (size_t)m * p.norm_out_ld + f0) = out;
                     }
                     fence_proxy_async();   // the MMA reads the stage through the async proxy
-                    mbar_arrive(&ready[stage]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ready[stage]);
                     if (++stage == S) { stage = 0; ++round; }
                 }
                 u += kb1 - kb0;
@@ -707,6 +717,7 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
     if (p.units * (long long)kGemmMaxGrid >= (1LL << 32)) return (int)cudaErrorInvalidValue;   // 32-bit partition arithmetic
     if (p.ctas <= 0 || p.ctas > num_sms) p.ctas = num_sms;
     if ((long long)p.ctas > p.units) p.ctas = (int)p.units;
+    if (p.whole_tiles && (long long)p.ctas > p.units / p.KB) p.ctas = (int)(p.units / p.KB);
     if (p.units == 0) return 0;
     switch (nt) {
     case 16: return launch_nt<16>(p, stream);
