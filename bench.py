@@ -61,6 +61,7 @@ def parse_args():
     ap.add_argument("--separate-pre-step", action="store_true",
                     help="fuse_context + inject_kv as two calls instead of one fuse_inject call")
     ap.add_argument("--no-fold", action="store_true", help="separate RMSNorm kernels in the draft step")
+    ap.add_argument("--inject-whole", type=int, default=None, help="1: injection GEMM over whole tiles, 0: split-K slabs")
     ap.add_argument("--trace-dump", default=None,
                     help="write the traced step's raw per-block stamps and launch records to this .npz file")
     ap.add_argument("--l2-prefetch", type=int, default=None,
@@ -458,6 +459,13 @@ def run_gpu(args):
     lens = torch.full((B,), T, dtype=torch.int32, device=dev)
     zeros = torch.zeros(B, dtype=torch.int32, device=dev)
     starts = torch.arange(0, B * T, T, dtype=torch.int32, device=dev)
+    # library switches (process-wide) before any call, the prefill included
+    D.dflash_diag_set_launch_mode(not args.no_pdl)
+    D.dflash_diag_set_norm_fold(not args.no_fold)
+    if args.inject_whole is not None:
+        D.dflash_diag_set_inject_partition(bool(args.inject_whole))
+    if args.l2_prefetch is not None:
+        D.dflash_diag_set_gemm_prefetch(args.l2_prefetch)
     pre_ms = []
     for rep in range(3):
         cache.set_len(zeros)
@@ -491,10 +499,6 @@ def run_gpu(args):
     rs = torch.arange(0, B * g, g, dtype=torch.int32, device=dev)
     rc = torch.full((B,), g, dtype=torch.int32, device=dev)
     h, c = drafter.handle, cache.handle
-    D.dflash_diag_set_launch_mode(not args.no_pdl)
-    D.dflash_diag_set_norm_fold(not args.no_fold)
-    if args.l2_prefetch is not None:
-        D.dflash_diag_set_gemm_prefetch(args.l2_prefetch)
 
     def step(i, hid_list=None):
         sp = torch.cuda.current_stream().cuda_stream

@@ -21,6 +21,9 @@ static bool g_pdl = true;
 // RMSNorm folded into the GEMMs that consume the normalised rows (draft step,
 // token tiles up to kFoldMaxNT wide); dflash_diag_set_norm_fold switches it.
 static bool g_fold = true;
+// Injection GEMM partition: whole output tiles (every K/V element one in-order
+// sum over all of K) instead of split-K per slab of tile rows.
+static bool g_inject_whole = false;
 constexpr int kFoldMaxNT = 64;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -332,8 +335,10 @@ static int inject_gemms(dflash_handle* h, dflash_cache* cc, const void* src, con
     const dflash_config& c = h->cfg;
     const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
     const int nt = pick_nt(total_rows);
-    for (int row0 = 0; row0 < total_rows; row0 += nt) {
-        const int rows = std::min(nt, total_rows - row0);
+    const bool whole = g_inject_whole;
+    const int slab = whole ? total_rows : nt;   // whole tiles: one launch over all rows
+    for (int row0 = 0; row0 < total_rows; row0 += slab) {
+        const int rows = std::min(slab, total_rows - row0);
         CUtensorMap tb;
         if (!act_map(&tb, (const uint8_t*)src + (size_t)row0 * H * 2, rows, H, H, nt)) return DFLASH_INVALID_ARG;
         for (int l0 = 0; l0 < c.n_layers; l0 += kMaxAMats / 2) {
@@ -351,6 +356,7 @@ static int inject_gemms(dflash_handle* h, dflash_cache* cc, const void* src, con
             p.kb_per_b = cdiv(H, 64);
             p.M = rows;
             p.row0 = row0;
+            p.whole_tiles = whole ? 1 : 0;
             p.K = H;
             p.epi = EPI_INJECT;
             p.d = d;
@@ -1322,6 +1328,11 @@ int dflash_diag_set_gemm_prefetch(int tiles) {
 }
 
 int dflash_diag_gemm_prefetch(void) { return gemm_l2_prefetch(); }
+
+int dflash_diag_set_inject_partition(int whole_tiles) {
+    g_inject_whole = whole_tiles != 0;
+    return DFLASH_OK;
+}
 
 int dflash_diag_set_norm_fold(int on) {
     g_fold = on != 0;

@@ -2,8 +2,10 @@
 DFlash-ja section 2.2, KV-injection bullet: the context feature of every
 verified row is appended to every layer's cache): a 2048-row context of the
 Qwen3-8B-shaped drafter injected in one call, in 16-row chunks, and in ragged
-chunks writes identical K/V bits.  The injection GEMM's k-split points depend
-only on the weight shape and the grid, never on the number of rows."""
+chunks writes identical K/V bits.  Under either work partition of the injection
+GEMM (split-K per slab of tile rows, or whole output tiles) the summation order
+of every element depends only on the weight shape and the grid, never on the
+number of rows."""
 import pytest
 import torch
 
@@ -23,7 +25,17 @@ def _inject(dr, cache, ctx, pieces):
     assert cache.status() == 0
 
 
-def test_inject_2048_rows_in_chunks_is_bit_exact():
+@pytest.mark.parametrize("whole_tiles", [False, True])
+def test_inject_2048_rows_in_chunks_is_bit_exact(whole_tiles):
+    from block_diffusion_speculative_03_b200 import dflash as D
+    D.dflash_diag_set_inject_partition(whole_tiles)
+    try:
+        _chunked(whole_tiles)
+    finally:
+        D.dflash_diag_set_inject_partition(False)
+
+
+def _chunked(whole_tiles):
     w = I.preset("qwen3_8b")
     T = w.context[0]
     W = I.make_weights(w, device="cuda")
