@@ -21,9 +21,11 @@ static bool g_pdl = true;
 // RMSNorm folded into the GEMMs that consume the normalised rows (draft step,
 // token tiles up to kFoldMaxNT wide); dflash_diag_set_norm_fold switches it.
 static bool g_fold = true;
-// Injection GEMM partition: whole output tiles (every K/V element one in-order
-// sum over all of K) instead of split-K per slab of tile rows.
-static bool g_inject_whole = false;
+// Partition of dflash_inject_kv's GEMM: whole output tiles (every K/V element one
+// in-order sum over all of K), or split-K per slab of tile rows.  Whole tiles are
+// faster for wide token tiles (prefill); the fused per-cycle call
+// dflash_fuse_inject always uses split-K slabs (all SMs stream at batch 1).
+static bool g_inject_whole = true;
 constexpr int kFoldMaxNT = 64;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -321,21 +323,25 @@ bool act_map(CUtensorMap* m, const void* base, int rows, int K, long long stride
 
 // The injection GEMMs of rows [0, total_rows) of `src` ([total_rows, H] bf16):
 // all layers' Wk/Wv stacked as one A operand (up to kMaxAMats matrices per
-// launch), RoPE and the cache write in the epilogue.  One launch per slab of nt
-// rows: every launch then has a single m-tile, so the split-K partition (k-ranges
-// per CTA over n_tiles x k-blocks) and with it the fp32 summation order of every
-// K/V element are the same whatever the number of rows: injecting rows in chunks
-// writes the same bits as injecting them at once.
+// launch), RoPE and the cache write in the epilogue.  Either partition keeps the
+// fp32 summation order of every K/V element independent of the number of rows,
+// so injecting rows in chunks writes the same bits as injecting them at once:
+//  - whole: one launch, CTAs take whole output tiles (each element one in-order
+//    sum over all of K); at batch 1 only n-tiles CTAs stream the weights, but
+//    wide token tiles (prefill) run without split-K partials;
+//  - split: one launch per slab of nt rows, each with a single m-tile, so the
+//    split-K partition over n_tiles x k-blocks is the same for every slab; all
+//    SMs stream the weights (the per-cycle injection of a few rows).
 // With ssq (the projected rows' per-tile sums of squares, [cdiv(H,128)][max_rows]),
 // src holds the un-normalised rows and each launch applies RMSNorm * g_fc to its
 // token tiles in shared memory (and copies the normalised rows to ctx_out when it
 // is not null).
 static int inject_gemms(dflash_handle* h, dflash_cache* cc, const void* src, const int32_t* row_start,
-                 const int32_t* row_count, int total_rows, const float* ssq, void* ctx_out, cudaStream_t st) {
+                 const int32_t* row_count, int total_rows, const float* ssq, void* ctx_out, bool whole,
+                 cudaStream_t st) {
     const dflash_config& c = h->cfg;
     const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
     const int nt = pick_nt(total_rows);
-    const bool whole = g_inject_whole;
     const int slab = whole ? total_rows : nt;   // whole tiles: one launch over all rows
     for (int row0 = 0; row0 < total_rows; row0 += slab) {
         const int rows = std::min(slab, total_rows - row0);
@@ -687,7 +693,7 @@ int dflash_inject_kv(dflash_handle* h, dflash_cache* cc, const void* ctx, const 
     const int H = c.hidden, d = c.head_dim, Nkv = c.n_kv_heads * d;
     if (c.dtype == DFLASH_BF16) {
         if (!aligned16(ctx)) return DFLASH_INVALID_ARG;
-        int r = inject_gemms(h, cc, ctx, row_start, row_count, total_rows, nullptr, nullptr, st);
+        int r = inject_gemms(h, cc, ctx, row_start, row_count, total_rows, nullptr, nullptr, g_inject_whole, st);
         if (r) return r;
     } else {
         Timed t(h, TK_SIMT_F32, st);
@@ -733,7 +739,7 @@ int dflash_fuse_inject(dflash_handle* h, dflash_cache* cc, const void* const* hi
         // memory: the context feature never goes through a separate kernel.
         int r = fuse_gemm(h, hiddens, row_stride, total_rows, h->ssq_ctx, st);
         if (r) return r;
-        r = inject_gemms(h, cc, h->y, row_start, row_count, total_rows, h->ssq_ctx, ctx_out, st);
+        r = inject_gemms(h, cc, h->y, row_start, row_count, total_rows, h->ssq_ctx, ctx_out, false, st);
         if (r) return r;
         Timed t(h, TK_INJECT_FINALIZE, st);
         launch_inject_finalize(row_count, cc->batch, cc->capacity, cc->len, cc->status, st,

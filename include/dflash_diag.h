@@ -207,11 +207,13 @@ int dflash_diag_gemm_prefetch(void);
  * normalisation kernel runs.  0 = one RMSNorm kernel before each of them. */
 int dflash_diag_set_norm_fold(int on);
 
-/* Work partition of the injection GEMM (process-wide, applies to calls enqueued
- * afterwards).  0: split-K with one launch per slab of token-tile rows; 1: whole
- * output tiles in one launch (no tile is split across CTAs).  Either way the fp32
- * summation order of every K/V element does not depend on the number of rows
- * injected, so chunked injection writes the same bits as one call. */
+/* Work partition of dflash_inject_kv's GEMM (process-wide, applies to calls
+ * enqueued afterwards).  1 (default): whole output tiles in one launch (no tile is
+ * split across CTAs; the fast choice for many rows, e.g. prefill); 0: split-K with
+ * one launch per slab of token-tile rows.  Either way the fp32 summation order of
+ * every K/V element does not depend on the number of rows injected, so chunked
+ * injection writes the same bits as one call.  dflash_fuse_inject always uses the
+ * split-K slabs (its few rows per call stream the weights on every SM). */
 int dflash_diag_set_inject_partition(int whole_tiles);
 
 /* "sm_100a" for this build. */

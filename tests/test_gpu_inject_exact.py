@@ -32,7 +32,7 @@ def test_inject_2048_rows_in_chunks_is_bit_exact(whole_tiles):
     try:
         _chunked(whole_tiles)
     finally:
-        D.dflash_diag_set_inject_partition(False)
+        D.dflash_diag_set_inject_partition(True)
 
 
 def _chunked(whole_tiles):
