@@ -26,6 +26,8 @@ static bool g_fold = true;
 // faster for wide token tiles (prefill); the fused per-cycle call
 // dflash_fuse_inject always uses split-K slabs (all SMs stream at batch 1).
 static bool g_inject_whole = true;
+// Whether the final norm is folded into the LM-head GEMM too (see draft_bf16).
+static bool g_fold_head = false;
 constexpr int kFoldMaxNT = 64;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -970,7 +972,12 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
     if (r) return r;
     CUtensorMap tm_hf, tm_x;
     if (!act_map(&tm_hf, h->hf, Mlm, H, H, pick_nt(Mlm)) || !act_map(&tm_x, h->x, M, H, H, nt)) return DFLASH_CUDA;
-    if (!fold) {
+    // The LM head streams the largest weight at the HBM roofline, where the folded
+    // normaliser's per-stage work measured slower than one final-norm kernel: the
+    // final norm stays a kernel of its own unless g_fold_head is set.
+    const bool fold_head = fold && g_fold_head;
+    (void)nt;
+    if (!fold_head) {
         Timed t(h, TK_RMSNORM, st);
         launch_rmsnorm<bf>((const bf*)h->x, (const bf*)h->w.g_final, (bf*)h->hf, Mlm, H, (float)c.rms_eps, gamma - 1,
                            gamma, 1, st, trace_small(h, TK_RMSNORM, Mlm));
@@ -988,25 +995,25 @@ static int draft_bf16(dflash_handle* h, dflash_cache* cc, int gamma, int32_t* dr
         p.ta[0] = h->tm_lm;
         p.amat[0].rows = c.vocab;
         p.n_amat = 1;
-        p.tb[0] = fold ? tm_x : tm_hf;
+        p.tb[0] = fold_head ? tm_x : tm_hf;
         p.kb_per_b = cdiv(H, 64);
-        p.M = fold ? M : Mlm;
+        p.M = fold_head ? M : Mlm;
         p.K = H;
         p.epi = EPI_LMHEAD;
         p.vocab = c.vocab;
         p.logits = logits;
         p.records = h->rec;
-        if (fold) {
+        if (fold_head) {
             fold_in(h, p, h->w.g_final, nH);
             p.lm_gamma = gamma;
         }
         Timed t(h, TK_GEMM_LMHEAD, st);
-        int r = run_gemm(h, p, fold ? nt : pick_nt(Mlm), st, TK_GEMM_LMHEAD);
+        int r = run_gemm(h, p, fold_head ? nt : pick_nt(Mlm), st, TK_GEMM_LMHEAD);
         if (r) return r;
     }
     Timed t(h, TK_LM_REDUCE, st);
     launch_lm_reduce(h->rec, cdiv(c.vocab, 128), Mlm, gamma - 1, h->req_ok, drafts, margin, st,
-                     trace_small(h, TK_LM_REDUCE, Mlm), fold ? 1 : 0);
+                     trace_small(h, TK_LM_REDUCE, Mlm), fold_head ? 1 : 0);
     h->launches += 1;
     return DFLASH_OK;
 }
@@ -1342,6 +1349,7 @@ int dflash_diag_set_inject_partition(int whole_tiles) {
 
 int dflash_diag_set_norm_fold(int on) {
     g_fold = on != 0;
+    g_fold_head = on > 1;
     return DFLASH_OK;
 }
 

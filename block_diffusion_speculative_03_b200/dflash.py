@@ -359,8 +359,9 @@ def dflash_diag_set_inject_partition(whole_tiles: bool) -> int:
     return _chk(lib().dflash_diag_set_inject_partition(1 if whole_tiles else 0), "dflash_diag_set_inject_partition")
 
 
-def dflash_diag_set_norm_fold(on: bool) -> int:
-    return _chk(lib().dflash_diag_set_norm_fold(1 if on else 0), "dflash_diag_set_norm_fold")
+def dflash_diag_set_norm_fold(on) -> int:
+    """0: no fold; 1 / True: fold the layer norms; 2: also fold the final norm into the LM head."""
+    return _chk(lib().dflash_diag_set_norm_fold(int(on)), "dflash_diag_set_norm_fold")
 
 
 def dflash_diag_draft_capture_stages(h: int, h_in=None, q=None, o=None, x_mid=None, h2=None, act=None) -> int:

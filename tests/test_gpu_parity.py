@@ -38,16 +38,17 @@ def test_tiny_fp32_chain():
     assert n > 0
 
 
-@pytest.mark.parametrize("fold", [True, False])
+@pytest.mark.parametrize("fold", [1, 2, 0])
 def test_small_bf16_chain_speculative_order(fold):
-    # fold: each RMSNorm applied inside the GEMM that consumes it (the default for
-    # token tiles up to 64 wide); not fold: one normalisation kernel before each
+    # fold 1: each layer RMSNorm applied inside the GEMM that consumes it (the
+    # default for token tiles up to 64 wide); 2: the final norm folded into the LM
+    # head as well; 0: one normalisation kernel before each consumer
     from block_diffusion_speculative_03_b200 import dflash as D
     D.dflash_diag_set_norm_fold(fold)
     try:
         n = _chain("small_bf16")
     finally:
-        D.dflash_diag_set_norm_fold(True)
+        D.dflash_diag_set_norm_fold(1)
     assert n > 0
 
 
