@@ -64,6 +64,10 @@ def parse_args():
     ap.add_argument("--inject-whole", type=int, default=None, help="1: injection GEMM over whole tiles, 0: split-K slabs")
     ap.add_argument("--trace-dump", default=None,
                     help="write the traced step's raw per-block stamps and launch records to this .npz file")
+    ap.add_argument("--o-beside", type=int, default=None,
+                    help="1: O-projection on the SMs the attention leaves free (default), 0: on all SMs")
+    ap.add_argument("--pre-stages", type=int, default=None,
+                    help="ring stages each GEMM CTA fills with weights before its dependency wait (0 = all)")
     ap.add_argument("--l2-prefetch", type=int, default=None,
                     help="weight tiles each GEMM CTA prefetches into L2 before its dependency wait")
     return ap.parse_args()
@@ -466,6 +470,10 @@ def run_gpu(args):
         D.dflash_diag_set_inject_partition(bool(args.inject_whole))
     if args.l2_prefetch is not None:
         D.dflash_diag_set_gemm_prefetch(args.l2_prefetch)
+    if args.pre_stages is not None:
+        D.dflash_diag_set_gemm_pre_stages(args.pre_stages)
+    if args.o_beside is not None:
+        D.dflash_diag_set_o_beside_attention(bool(args.o_beside))
     pre_ms = []
     for rep in range(3):
         cache.set_len(zeros)

@@ -28,6 +28,8 @@ static bool g_fold = true;
 static bool g_inject_whole = true;
 // Whether the final norm is folded into the LM-head GEMM too (see draft_bf16).
 static bool g_fold_head = false;
+// O-projection on the SMs the attention does not hold (see layers_bf16).
+static bool g_o_beside_attention = true;
 constexpr int kFoldMaxNT = 64;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -299,14 +301,17 @@ void capture_hf(dflash_handle* h, int Mlm, cudaStream_t st) {
 // Common GEMM plumbing.
 void gemm_common(dflash_handle* h, GemmParams& p) {
     p.l2_prefetch = gemm_l2_prefetch();
+    p.pre_stages = gemm_pre_stages();
     p.partial = h->gpart;
     p.counters = h->gcnt;
     p.status = h->status;
     p.ctas = 0;
 }
 
-int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st, int kind) {
+int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st, int kind, int ctas = 0, int l2_prefetch = -1) {
     gemm_common(h, p);
+    if (ctas > 0) p.ctas = ctas;
+    if (l2_prefetch >= 0) p.l2_prefetch = l2_prefetch;
     // GEMM trace: 8 stamps per CTA (gemm.cuh), past the wait at 1, exit at 6;
     // room for the largest grid, CTAs the launch does not use stay zero.
     p.trace = trace_slot(h, kind, kMaxCtas, 8, 1, 6);
@@ -897,7 +902,14 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
                 p.ssq_ld = ssq_ld;
             }
             Timed t(h, TK_GEMM_O, st);
-            int r = run_gemm(h, p, nt, st, TK_GEMM_O);
+            // The attention holds attn_blocks SMs until it ends; O-projection CTAs
+            // placed there would start a whole attention later than the rest and
+            // finish last.  Run the O-projection on the other SMs only, and let those
+            // CTAs, idle until the attention is done, prefetch their whole weight
+            // range into L2 (the attention leaves HBM nearly idle).
+            const bool beside = g_o_beside_attention && attn_blocks * 4 <= h->num_sms * 3;
+            int r = beside ? run_gemm(h, p, nt, st, TK_GEMM_O, h->num_sms - attn_blocks, 64)
+                           : run_gemm(h, p, nt, st, TK_GEMM_O);
             if (r) return r;
         }
         capture_stage(h, h->cap_xm, h->x, l, M, H, st);
@@ -1341,6 +1353,17 @@ int dflash_diag_set_gemm_prefetch(int tiles) {
 }
 
 int dflash_diag_gemm_prefetch(void) { return gemm_l2_prefetch(); }
+
+int dflash_diag_set_gemm_pre_stages(int stages) {
+    if (stages < 0 || stages > 64) return DFLASH_INVALID_ARG;
+    set_gemm_pre_stages(stages);
+    return DFLASH_OK;
+}
+
+int dflash_diag_set_o_beside_attention(int on) {
+    g_o_beside_attention = on != 0;
+    return DFLASH_OK;
+}
 
 int dflash_diag_set_inject_partition(int whole_tiles) {
     g_inject_whole = whole_tiles != 0;

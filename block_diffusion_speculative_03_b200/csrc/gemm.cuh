@@ -51,6 +51,7 @@ struct GemmParams {
     int whole_tiles;             // 1: CTAs take whole output tiles (no split-K): every output is one
                                  //    in-order accumulation over all of K, whatever M and the grid
     int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
+    int pre_stages;              // ring stages filled with weights before the wait (0: the whole ring)
     float* partial;              // [2 * ctas][NT][128] fp32 split-tile partials
     int* counters;               // [n_tiles * m_tiles], zero between launches
     int* status;                 // handle status word (DFLASH_TIMEOUT)
@@ -131,6 +132,9 @@ inline int pick_nt(int M) {
 // before its dependency wait; process-wide, set by dflash_diag_set_gemm_prefetch.
 int gemm_l2_prefetch();
 void set_gemm_l2_prefetch(int tiles);
+// Ring stages each CTA fills with weight tiles before its dependency wait (0 = all).
+int gemm_pre_stages();
+void set_gemm_pre_stages(int stages);
 
 // Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
 // ctas) and launches on `stream`.  Returns a cudaError_t; cudaErrorInvalidValue

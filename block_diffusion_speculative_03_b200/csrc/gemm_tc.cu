@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
             // first S weight tiles into the ring, and the next l2_prefetch ones
             // into L2, before waiting for it to finish.
             int pre = 0;
-            const int n_ahead = S + p.l2_prefetch;
+            const int s_pre = (p.pre_stages > 0 && p.pre_stages < S) ? p.pre_stages : S;
+            const int n_ahead = s_pre + p.l2_prefetch;
             for (long long u = u_begin, idx = 0; u < u_end && idx < n_ahead;) {
                 const long long t = u / KB;
                 const int kb0 = (int)(u % KB);
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                     while (mi + 1 < p.n_amat && n_tile >= p.amat[mi + 1].tile0) ++mi;
                 const int arow = p.swiglu ? n_tile * 64 : (n_tile - p.amat[mi].tile0) * 128;
                 for (int kb = kb0; kb < kb1 && idx < n_ahead; ++kb, ++idx) {
-                    if (idx < S) {
+                    if (idx < s_pre) {
                         mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
                         uint8_t* a = sA + pre * C::A_BYTES;
                         if (p.swiglu) {
@@ -696,6 +697,9 @@ static int launch_nt(GemmParams& p, cudaStream_t stream) {
 }
 
 static int g_l2_prefetch = 0;
+static int g_pre_stages = 0;
+int gemm_pre_stages() { return g_pre_stages; }
+void set_gemm_pre_stages(int stages) { g_pre_stages = stages < 0 ? 0 : stages; }
 int gemm_l2_prefetch() { return g_l2_prefetch; }
 void set_gemm_l2_prefetch(int tiles) { g_l2_prefetch = tiles < 0 ? 0 : (tiles > 256 ? 256 : tiles); }
 

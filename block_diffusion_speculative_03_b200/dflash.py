@@ -107,8 +107,10 @@ def lib():
         "dflash_diag_set_launch_mode": (i32, [i32]),
         "dflash_diag_set_gemm_prefetch": (i32, [i32]),
         "dflash_diag_gemm_prefetch": (i32, []),
+        "dflash_diag_set_gemm_pre_stages": (i32, [i32]),
         "dflash_diag_set_norm_fold": (i32, [i32]),
         "dflash_diag_set_inject_partition": (i32, [i32]),
+        "dflash_diag_set_o_beside_attention": (i32, [i32]),
         "dflash_diag_wait_selftest": (i32, [vp, vp, vp]),
         "dflash_diag_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
         "dflash_diag_gemm_bf16_traced": (i32, [vp, vp, vp, i32, i32, i32, vp, sz, i32, vp, vp]),
@@ -143,7 +145,9 @@ def exported_symbols() -> list:
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_set_gemm_prefetch", "dflash_diag_gemm_prefetch",
+            "dflash_diag_set_gemm_pre_stages",
             "dflash_diag_set_norm_fold", "dflash_diag_set_inject_partition",
+            "dflash_diag_set_o_beside_attention",
             "dflash_diag_wait_selftest",
             "dflash_diag_attention", "dflash_diag_gemm_bf16_traced",
             "dflash_diag_attention_traced", "dflash_diag_gemm_bf16_noalloc", "dflash_diag_draft_capture",
@@ -351,8 +355,16 @@ def dflash_diag_set_gemm_prefetch(tiles: int) -> int:
     return _chk(lib().dflash_diag_set_gemm_prefetch(int(tiles)), "dflash_diag_set_gemm_prefetch")
 
 
+def dflash_diag_set_gemm_pre_stages(stages: int) -> int:
+    return _chk(lib().dflash_diag_set_gemm_pre_stages(int(stages)), "dflash_diag_set_gemm_pre_stages")
+
+
 def dflash_diag_gemm_prefetch() -> int:
     return lib().dflash_diag_gemm_prefetch()
+
+
+def dflash_diag_set_o_beside_attention(on: bool) -> int:
+    return _chk(lib().dflash_diag_set_o_beside_attention(1 if on else 0), "dflash_diag_set_o_beside_attention")
 
 
 def dflash_diag_set_inject_partition(whole_tiles: bool) -> int:

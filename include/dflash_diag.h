@@ -198,6 +198,12 @@ int dflash_diag_set_gemm_prefetch(int tiles);
 /* The current setting of dflash_diag_set_gemm_prefetch. */
 int dflash_diag_gemm_prefetch(void);
 
+/* Shared-memory ring stages each CTA of the tensor-core GEMM fills with weight
+ * tiles before waiting for the previous kernel (process-wide, 0..64; 0 = the whole
+ * ring, the default).  A shallower pre-wait burst leaves the previous kernel's
+ * finishing memory round trips less contended. */
+int dflash_diag_set_gemm_pre_stages(int stages);
+
 /* Whether the draft step folds each RMSNorm into the GEMM that consumes its
  * output (process-wide, default 1; applies to calls enqueued afterwards).  When
  * on and the token tile is at most 64 wide, the producer of the residual stream
@@ -208,6 +214,12 @@ int dflash_diag_gemm_prefetch(void);
  * the HBM roofline, where the folded form measured slower) unless on = 2, which
  * folds it too.  0 = one RMSNorm kernel before each of them. */
 int dflash_diag_set_norm_fold(int on);
+
+/* Placement of the O-projection GEMM of each draft layer (process-wide, default 1):
+ * 1 = on the SMs the preceding attention kernel does not occupy (when it occupies
+ * at most three quarters of them), with those CTAs prefetching their whole weight
+ * range into L2 while the attention runs; 0 = on every SM like the other GEMMs. */
+int dflash_diag_set_o_beside_attention(int on);
 
 /* Work partition of dflash_inject_kv's GEMM (process-wide, applies to calls
  * enqueued afterwards).  1 (default): whole output tiles in one launch (no tile is
