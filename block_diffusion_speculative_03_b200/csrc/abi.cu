@@ -19,7 +19,9 @@ using namespace df;
 namespace df {
 static bool g_pdl = true;
 // RMSNorm folded into the GEMMs that consume the normalised rows (draft step,
-// token tiles up to kFoldMaxNT wide); dflash_diag_set_norm_fold switches it.
+// token tiles up to kFoldMaxNT wide; wider tiles give the two normalising warps
+// more work per stage than the weight stream leaves them, measured slower than a
+// separate norm kernel); dflash_diag_set_norm_fold switches it.
 static bool g_fold = true;
 // Partition of dflash_inject_kv's GEMM: whole output tiles (every K/V element one
 // in-order sum over all of K), or split-K per slab of tile rows.  Whole tiles are
@@ -30,7 +32,7 @@ static bool g_inject_whole = true;
 static bool g_fold_head = false;
 // O-projection on the SMs the attention does not hold (see layers_bf16).
 static bool g_o_beside_attention = true;
-constexpr int kFoldMaxNT = 64;
+constexpr int kFoldMaxNT = 16;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
 void ensure_carveout(const void* fn) {

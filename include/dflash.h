@@ -210,7 +210,7 @@ int dflash_inject_kv(dflash_handle* h, dflash_cache* c, const void* ctx, const i
  * draft layer's K/V cache), taken straight from the target's verification output.
  * Computes exactly dflash_fuse_context followed by dflash_inject_kv of the same
  * rows (the same rounding points: ctx = R(RMSNorm(R(y)) * g_fc) is what the K/V
- * projections read), but with small batches of rows (at most 64 per call) the
+ * projections read), but with small batches of rows (at most 16 per call) the
  * RMSNorm is folded into the injection GEMM: the W_fc GEMM also writes its rows'
  * partial sums of squares, and the injection GEMM normalises its token tiles in
  * shared memory, so no separate normalisation kernel runs and the feature is not

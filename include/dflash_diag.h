@@ -206,13 +206,14 @@ int dflash_diag_set_gemm_pre_stages(int stages);
 
 /* Whether the draft step folds each RMSNorm into the GEMM that consumes its
  * output (process-wide, default 1; applies to calls enqueued afterwards).  When
- * on and the token tile is at most 64 wide, the producer of the residual stream
- * (the embedding, the O-projection and the down-projection) also writes per-tile
- * partial sums of squares of its rows, and the QKV and gate/up GEMMs
- * read x itself and normalise each token tile in shared memory.  The final norm
- * before the LM head stays a kernel of its own (the LM head streams its weights at
- * the HBM roofline, where the folded form measured slower) unless on = 2, which
- * folds it too.  0 = one RMSNorm kernel before each of them. */
+ * on and the token tile is at most 16 wide (batch 1 at gamma 16), the producer
+ * of the residual stream (the embedding, the O-projection and the
+ * down-projection) also writes per-tile partial sums of squares of its rows, and
+ * the QKV and gate/up GEMMs read x itself and normalise each token tile in shared
+ * memory.  The final norm before the LM head stays a kernel of its own (the LM
+ * head streams its weights at the HBM roofline, where the folded form measured
+ * slower) unless on = 2, which folds it too.  0 = one RMSNorm kernel before each
+ * of them. */
 int dflash_diag_set_norm_fold(int on);
 
 /* Placement of the O-projection GEMM of each draft layer (process-wide, default 1):
