@@ -67,7 +67,9 @@ def parse_args():
     ap.add_argument("--o-beside", type=int, default=None,
                     help="1: O-projection on the SMs the attention leaves free (default), 0: on all SMs")
     ap.add_argument("--pre-stages", type=int, default=None,
-                    help="ring stages each GEMM CTA fills with weights before its dependency wait (0 = all)")
+                    help="ring stages each GEMM CTA fills with weights before its dependency wait (0 = all; library default 6)")
+    ap.add_argument("--last-arriver", action="store_true",
+                    help="split GEMM tiles finished by the contributor that counts in last (default: by the first)")
     ap.add_argument("--l2-prefetch", type=int, default=None,
                     help="weight tiles each GEMM CTA prefetches into L2 before its dependency wait")
     return ap.parse_args()
@@ -474,6 +476,7 @@ def run_gpu(args):
         D.dflash_diag_set_gemm_pre_stages(args.pre_stages)
     if args.o_beside is not None:
         D.dflash_diag_set_o_beside_attention(bool(args.o_beside))
+    D.dflash_diag_set_split_finisher(args.last_arriver)
     pre_ms = []
     for rep in range(3):
         cache.set_len(zeros)
@@ -729,7 +732,9 @@ def run_gpu(args):
             "step_options": {"conditioning": args.conditioning,
                              "pre_step": ("fuse_context + ingest_fused_input" if args.conditioning == "input-fusion"
                                           else "two calls" if args.separate_pre_step else "fuse_inject (one call)"),
-                             "norm_fold": not args.no_fold, "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch()},
+                             "norm_fold": not args.no_fold, "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch(),
+                             "split_tile_finisher": "last arriver" if args.last_arriver else "first contributor",
+                             "gemm_pre_stages": args.pre_stages if args.pre_stages is not None else "library default (6)"},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
                                                                               else ", programmatic dependent launch"),
             "clocks": clocks,

@@ -304,6 +304,7 @@ void capture_hf(dflash_handle* h, int Mlm, cudaStream_t st) {
 void gemm_common(dflash_handle* h, GemmParams& p) {
     p.l2_prefetch = gemm_l2_prefetch();
     p.pre_stages = gemm_pre_stages();
+    p.last_arriver = gemm_last_arriver();
     p.partial = h->gpart;
     p.counters = h->gcnt;
     p.status = h->status;
@@ -1196,6 +1197,7 @@ int dflash_diag_gemm_bf16_traced(const void* X, const void* W, float* Y, int M, 
     p.partial = (float*)((uint8_t*)scratch + counters);
     p.status = nullptr;
     p.trace = (long long*)trace;
+    p.last_arriver = gemm_last_arriver();
     p.ctas = grid > 0 ? std::min(grid, kMaxCtas) : 0;
     int e = launch_gemm_tc(p, nt, std::min(sms, kMaxCtas), S(stream));
     return e == 0 ? DFLASH_OK : DFLASH_CUDA;
@@ -1359,6 +1361,11 @@ int dflash_diag_gemm_prefetch(void) { return gemm_l2_prefetch(); }
 int dflash_diag_set_gemm_pre_stages(int stages) {
     if (stages < 0 || stages > 64) return DFLASH_INVALID_ARG;
     set_gemm_pre_stages(stages);
+    return DFLASH_OK;
+}
+
+int dflash_diag_set_split_finisher(int last_arriver) {
+    set_gemm_last_arriver(last_arriver);
     return DFLASH_OK;
 }
 

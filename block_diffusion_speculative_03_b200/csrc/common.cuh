@@ -88,6 +88,32 @@ DF_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
     }
 }
 
+// Global load with gpu-scope acquire semantics (pairs with a writer's
+// fence + atomic).
+DF_DEV int ld_acquire_gpu(const int* ptr) {
+    int v;
+    asm volatile("ld.global.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Bounded wait until a count that other CTAs raise reaches `target`; the
+// same limit and abort behaviour as mbar_wait.  One thread polls.
+DF_DEV bool count_wait(const int* ctr, int target, volatile int* abort_flag, int* status) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_gpu(ctr) >= target) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                if (status) atomicCAS(status, 0, DFLASH_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 // Step trace of the small kernels (null in normal use): thread 0 of every block
 // stamps %globaltimer (ns) into tr[2 * block + which], which = 0 once past the
 // dependency wait, 1 at exit.

@@ -52,6 +52,9 @@ struct GemmParams {
                                  //    in-order accumulation over all of K, whatever M and the grid
     int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
     int pre_stages;              // ring stages filled with weights before the wait (0: the whole ring)
+    int last_arriver;            // split tiles: 1 = finished by whichever contributor counts in last;
+                                 //    0 = by the contributor holding the tile's first k-blocks, which
+                                 //    waits for the others' partials and stores none of its own
     float* partial;              // [2 * ctas][NT][128] fp32 split-tile partials
     int* counters;               // [n_tiles * m_tiles], zero between launches
     int* status;                 // handle status word (DFLASH_TIMEOUT)
@@ -135,6 +138,8 @@ void set_gemm_l2_prefetch(int tiles);
 // Ring stages each CTA fills with weight tiles before its dependency wait (0 = all).
 int gemm_pre_stages();
 void set_gemm_pre_stages(int stages);
+int gemm_last_arriver();
+void set_gemm_last_arriver(int on);
 
 // Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
 // ctas) and launches on `stream`.  Returns a cudaError_t; cudaErrorInvalidValue

@@ -422,20 +422,33 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                                                                      : make_float2(1.f, 0.f);
                 }
             }
-            const bool ok = mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
+            // Split tiles.  By default a split tile is finished by its first
+            // contributor, the CTA holding the tile's k-blocks from 0: its range ends
+            // inside the tile, so the tile is its last segment, while every other
+            // contributor's range starts inside the tile, so each publishes its partial
+            // in its first segment and never waits on another CTA (no cycle of waits;
+            // the grid is at most one CTA per SM, so all CTAs become resident).  The
+            // finisher stores no partial of its own: one thread waits for the count of
+            // published partials, before the accumulator wait so that the round trip
+            // overlaps the CTA's last MMAs.  With p.last_arriver every contributor
+            // publishes and counts, and the one that counts last finishes.
+            const bool whole = (kb0 == 0 && kb1 == KB);
+            const bool fin_first = !whole && !p.last_arriver && kb0 == 0;
+            int first = cta, nc = 1;
+            if (!whole) {
+                const uint32_t t32 = (uint32_t)t, K32 = (uint32_t)KB, U32 = (uint32_t)U, P32 = (uint32_t)P;
+                first = (int)sk32_owner(t32 * K32, U32, P32);
+                nc = (int)sk32_owner((t32 + 1) * K32 - 1, U32, P32) - first + 1;
+            }
+            bool ok = true;
+            if (fin_first && e == 0) ok = count_wait(&p.counters[t], nc - 1, abort_flag, p.status);
+            ok = ok && mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
             if (named_bar_or(1, 128, !ok)) break;   // leave together: later named barriers stay matched
             if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
             tc_fence_after();
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
-            const bool whole = (kb0 == 0 && kb1 == KB);
             bool finish = true;
-            int first = cta, nc = 1;
-            if (!whole) {
-                {
-                    const uint32_t t32 = (uint32_t)t, K32 = (uint32_t)KB, U32 = (uint32_t)U, P32 = (uint32_t)P;
-                    first = (int)sk32_owner(t32 * K32, U32, P32);
-                    nc = (int)sk32_owner((t32 + 1) * K32 - 1, U32, P32) - first + 1;
-                }
+            if (!whole && !fin_first) {
                 float* dst = p.partial + (size_t)sk32_slot(cta, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += 16) {
@@ -446,18 +459,26 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                 }
                 // Release the CTA's partial and count it: the barrier orders every
                 // thread's stores before one thread's gpu-scope fence and atomic; the
-                // last arriver's fence (acquire side) and the barrier after it make the
-                // other contributors' partials visible to all its threads.
+                // finisher's acquire (a fence after the atomic for the last arriver)
+                // and the barrier after it make the partials visible to all its threads.
                 named_bar_sync(1, 128);
-                if (e == 0) {
-                    __threadfence();
-                    const int old = atomicAdd(&p.counters[t], 1);
-                    const bool last = old == nc - 1;
-                    if (last) __threadfence();
-                    *s_flag = last ? 1 : 0;
+                if (p.last_arriver) {
+                    if (e == 0) {
+                        __threadfence();
+                        const int old = atomicAdd(&p.counters[t], 1);
+                        const bool last = old == nc - 1;
+                        if (last) __threadfence();
+                        *s_flag = last ? 1 : 0;
+                    }
+                    named_bar_sync(1, 128);
+                    finish = (*s_flag != 0);
+                } else {
+                    if (e == 0) {
+                        __threadfence();
+                        atomicAdd(&p.counters[t], 1);
+                    }
+                    finish = false;
                 }
-                named_bar_sync(1, 128);
-                finish = (*s_flag != 0);
             }
             if (finish) {
 #pragma unroll 1
@@ -697,9 +718,12 @@ static int launch_nt(GemmParams& p, cudaStream_t stream) {
 }
 
 static int g_l2_prefetch = 0;
-static int g_pre_stages = 0;
+static int g_pre_stages = 6;   // measured: 6 of the ring's stages before the wait beat the whole ring
+static int g_last_arriver = 0;
 int gemm_pre_stages() { return g_pre_stages; }
 void set_gemm_pre_stages(int stages) { g_pre_stages = stages < 0 ? 0 : stages; }
+int gemm_last_arriver() { return g_last_arriver; }
+void set_gemm_last_arriver(int on) { g_last_arriver = on != 0; }
 int gemm_l2_prefetch() { return g_l2_prefetch; }
 void set_gemm_l2_prefetch(int tiles) { g_l2_prefetch = tiles < 0 ? 0 : (tiles > 256 ? 256 : tiles); }
 

@@ -200,9 +200,18 @@ int dflash_diag_gemm_prefetch(void);
 
 /* Shared-memory ring stages each CTA of the tensor-core GEMM fills with weight
  * tiles before waiting for the previous kernel (process-wide, 0..64; 0 = the whole
- * ring, the default).  A shallower pre-wait burst leaves the previous kernel's
+ * ring; default 6).  A shallower pre-wait burst leaves the previous kernel's
  * finishing memory round trips less contended. */
 int dflash_diag_set_gemm_pre_stages(int stages);
+
+/* How the tensor-core GEMM finishes an output tile whose k-blocks are split
+ * over several CTAs (process-wide; applies to launches enqueued afterwards).
+ * 0 (the default): the CTA holding the tile's first k-blocks finishes it; it
+ * waits (bounded) for the other contributors' published partials and adds them
+ * in contributor order.  1: every contributor publishes its partial and counts
+ * it with an atomic, and the one that counts last finishes.  Both add the
+ * partials in the same order, so the results are bit-identical. */
+int dflash_diag_set_split_finisher(int last_arriver);
 
 /* Whether the draft step folds each RMSNorm into the GEMM that consumes its
  * output (process-wide, default 1; applies to calls enqueued afterwards).  When

@@ -44,8 +44,8 @@ def test_gemm_matches_fp64(M, N, K):
 
 @pytest.mark.parametrize("grid", [1, 3, 7, 64])
 def test_gemm_split_tiles_and_repeat_calls(grid):
-    # few CTAs over many k-blocks: every tile is split across CTAs and resolved
-    # by the last arriver; repeated calls check the counters are left at zero
+    # few CTAs over many k-blocks: every tile is split across CTAs and finished
+    # by one of them; repeated calls check the counters are left at zero
     M, N, K = 16, 512, 2048
     ref, outs = _run(M, N, K, grid=grid, calls=3)
     for got in outs:
@@ -59,3 +59,22 @@ def test_gemm_result_does_not_depend_on_partition_much():
     _, (b,) = _run(M, N, K, grid=5)
     _close(ref, a, K)
     _close(ref, b, K)
+
+
+@pytest.mark.parametrize("M,N,K,grid", [(16, 512, 2048, 7), (16, 128, 12288, 0), (33, 1000, 4096, 0),
+                                        (200, 640, 1024, 64), (16, 4096, 4096, 0), (5, 384, 704, 100)])
+def test_split_tile_finishers_agree_bitwise(M, N, K, grid):
+    """A split tile finished by its first contributor (waiting for the others'
+    partials) and by its last arriver adds the same partials in the same order:
+    identical bits, every call.  (16, 128, 12288) on the full grid splits one tile
+    over all CTAs, so the first contributor waits for every other one."""
+    try:
+        D.dflash_diag_set_split_finisher(True)
+        _, last = _run(M, N, K, grid=grid, calls=2)
+        D.dflash_diag_set_split_finisher(False)
+        ref, first = _run(M, N, K, grid=grid, calls=2)
+    finally:
+        D.dflash_diag_set_split_finisher(False)
+    _close(ref, first[0], K)
+    for got in last + first[1:]:
+        assert torch.equal(got, first[0])
