@@ -59,25 +59,6 @@ DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2
     }
 }
 
-// The tile's share of each written row's sum of squares (sq: this thread's
-// feature, CH rows): over the 32 lanes of a warp (butterfly), then the four
-// warps in quadrant order, so every run adds in the same order.  Called by all
-// 128 epilogue threads (two named barriers); red: [4][CH] shared floats.
-template <int CH>
-DF_DEV void tile_ssq(float* sq, float* red, int q, int lane, int e, int mbase, int n_tile, const GemmParams& p) {
-#pragma unroll
-    for (int i = 0; i < CH; ++i)
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], off);
-    if (lane == 0)
-#pragma unroll
-        for (int i = 0; i < CH; ++i) red[q * CH + i] = sq[i];
-    named_bar_sync(1, 128);
-    if (e < CH && mbase + e < p.M)
-        p.ssq_out[(size_t)n_tile * p.ssq_ld + mbase + e] = ((red[e] + red[CH + e]) + red[2 * CH + e]) + red[3 * CH + e];
-    named_bar_sync(1, 128);
-}
-
 template <int NT>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     k_gemm_tc(const __grid_constant__ GemmParams p) {
@@ -89,6 +70,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     uint8_t* sA = smem;
     uint8_t* sB = smem + S * C::A_BYTES;
     float* xch = (float*)(sB + S * C::B_BYTES);
+    __nv_bfloat16* const xout = (__nv_bfloat16*)xch;   // epilogue outputs, token-major [CH][128] bf16
     uint64_t* full = (uint64_t*)(xch + C::XCH_FLOATS);
     uint64_t* empty = full + S;
     uint64_t* accf = empty + S;
@@ -99,11 +81,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     int* s_flag = (int*)(tmem_slot + 2);
     int* tok_b = s_flag + 1;          // [NT]
     int* tok_pos = tok_b + NT;        // [NT]
-    float* lmred = (float*)(tok_pos + NT);   // [4][CH][3]
-    float* inv_s = lmred + 4 * CH * 3;       // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
+    float* inv_s = (float*)(tok_pos + NT);   // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
     uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + 2 * NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
     __nv_bfloat16* sgain = (__nv_bfloat16*)(((uintptr_t)(ready + S) + 15) & ~(uintptr_t)15);   // [GAIN_MAX]
-    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 4 * CH * 3 * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
                       C::MISC_BYTES, "misc");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -526,62 +507,77 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                                 if (mbase + i < p.M) o[(size_t)(mbase + i) * p.ldo + lr] = v[i];
                         break;
                     }
-                    case EPI_BF16: {
-                        __nv_bfloat16* o = (__nv_bfloat16*)p.out;
-                        float sq[CH];
-#pragma unroll
-                        for (int i = 0; i < CH; ++i) {
-                            sq[i] = 0.f;
-                            if (row_ok && mbase + i < p.M) {
-                                const __nv_bfloat16 yb = f2bf(v[i]);
-                                o[(size_t)(mbase + i) * p.ldo + lr] = yb;
-                                const float yf = bf2f(yb);
-                                sq[i] = yf * yf;
-                            }
-                        }
-                        if (p.ssq_out) tile_ssq<CH>(sq, lmred, q, lane, e, mbase, n_tile, p);
-                        break;
-                    }
+                    case EPI_BF16:
                     case EPI_RESID: {
-                        // All residual loads of the chunk first, then the stores,
-                        // so the loads are not serialised behind the stores.
+                        // The rounded outputs go through shared memory token-major, so
+                        // that they leave in 16-byte stores and each token's sum of
+                        // squares over the tile's features is one short butterfly.
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
-                        float rv[CH];
-                        if constexpr (PRE) {
+                        if (p.epi == EPI_RESID) {
+                            float rv[CH];
+                            if constexpr (PRE) {
 #pragma unroll
-                            for (int i = 0; i < CH; ++i) rv[i] = pre_x[i];
+                                for (int i = 0; i < CH; ++i) rv[i] = pre_x[i];
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < CH; ++i)
+                                    rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+                            }
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) xout[i * 128 + row] = f2bf(rv[i] + v[i]);
                         } else {
 #pragma unroll
-                            for (int i = 0; i < CH; ++i)
-                                rv[i] = (row_ok && mbase + i < p.M) ? bf2f(o[(size_t)(mbase + i) * p.ldo + lr]) : 0.f;
+                            for (int i = 0; i < CH; ++i) xout[i * 128 + row] = f2bf(v[i]);
                         }
-                        float sq[CH];
+                        named_bar_sync(1, 128);
+                        const int nrows = p.amat[mi].rows, rbase = (n_tile - p.amat[mi].tile0) * 128;
 #pragma unroll
-                        for (int i = 0; i < CH; ++i) {
-                            sq[i] = 0.f;
-                            if (row_ok && mbase + i < p.M) {
-                                const __nv_bfloat16 xb = f2bf(rv[i] + v[i]);
-                                o[(size_t)(mbase + i) * p.ldo + lr] = xb;
-                                const float xf = bf2f(xb);
-                                sq[i] = xf * xf;
+                        for (int k = 0; k < CH / 8; ++k) {
+                            const int c = e + 128 * k, i = c >> 4, r0 = (c & 15) * 8;
+                            const int m = mbase + i, f = rbase + r0;
+                            const bool in = m < p.M && f < nrows;   // rows come in multiples of 8
+                            const uint4 w = *(const uint4*)(xout + i * 128 + r0);
+                            if (in) *(uint4*)(o + (size_t)m * p.ldo + f) = w;
+                            if (p.ssq_out) {
+                                // the 8 features in order, then the 16 pieces of the token
+                                // in a fixed butterfly
+                                float sq = 0.f;
+                                if (in) {
+                                    const __nv_bfloat16* b8 = (const __nv_bfloat16*)&w;
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j) {
+                                        const float xf = bf2f(b8[j]);
+                                        sq = fmaf(xf, xf, sq);
+                                    }
+                                }
+#pragma unroll
+                                for (int off = 8; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                                if ((c & 15) == 0 && m < p.M) p.ssq_out[(size_t)n_tile * p.ssq_ld + m] = sq;
                             }
                         }
-                        if (p.ssq_out) tile_ssq<CH>(sq, lmred, q, lane, e, mbase, n_tile, p);
+                        named_bar_sync(1, 128);
                         break;
                     }
                     case EPI_SWIGLU: {
+                        // Rows 0..63 of the tile are gate rows, 64..127 the matching up
+                        // rows.  The up values cross through the upper half of the
+                        // exchange buffer, the bf16 products through its lower half.
+                        if (row >= 64)
 #pragma unroll
-                        for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
+                            for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
                         named_bar_sync(1, 128);
-                        if (row < 64) {
-                            __nv_bfloat16* o = (__nv_bfloat16*)p.out;
-                            const int f = n_tile * 64 + row;
+                        if (row < 64)
 #pragma unroll
                             for (int i = 0; i < CH; ++i)
-                                if (mbase + i < p.M) {
-                                    const float up = xch[(row + 64) * (CH + 1) + i];
-                                    o[(size_t)(mbase + i) * p.ldo + f] = f2bf(silu(v[i]) * up);
-                                }
+                                xout[i * 64 + row] = f2bf(silu(v[i]) * xch[(row + 64) * (CH + 1) + i]);
+                        named_bar_sync(1, 128);
+                        __nv_bfloat16* o = (__nv_bfloat16*)p.out;
+#pragma unroll
+                        for (int k = 0; k < CH / 16; ++k) {
+                            const int c = e + 128 * k, i = c >> 3, r0 = (c & 7) * 8;
+                            const int m = mbase + i;
+                            if (m < p.M)
+                                *(uint4*)(o + (size_t)m * p.ldo + n_tile * 64 + r0) = *(const uint4*)(xout + i * 64 + r0);
                         }
                         named_bar_sync(1, 128);
                         break;
@@ -599,50 +595,68 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
 #pragma unroll
                         for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
                         named_bar_sync(1, 128);
+                        // rotate-half RoPE of every column (the partner feature of the same
+                        // head from the exchange buffer), rounded to bf16 in registers
                         const int prow = (i_in < half) ? row + half : row - half;
-                        if (row_ok) {
-                            // cos/sin of every column first (independent loads), then the stores
-                            float2 cs[CH];
-                            if constexpr (PRE) {
+                        float2 cs[CH];
+                        if constexpr (PRE) {
 #pragma unroll
-                                for (int i = 0; i < CH; ++i) cs[i] = pre_cs[i];
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < CH; ++i) {
-                                    const int b = tok_b[c0 + i];
-                                    cs[i] = (rotate && b >= 0)
-                                                ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
-                                                : make_float2(1.f, 0.f);
-                                }
-                            }
+                            for (int i = 0; i < CH; ++i) cs[i] = pre_cs[i];
+                        } else {
 #pragma unroll
                             for (int i = 0; i < CH; ++i) {
                                 const int b = tok_b[c0 + i];
-                                if (b < 0) continue;
-                                const int pos = tok_pos[c0 + i];
-                                float x = v[i];
-                                if (rotate) {
-                                    const float pr = xch[prow * (CH + 1) + i];
-                                    x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
-                                }
-                                if (is_q) {
-                                    ((__nv_bfloat16*)p.out)[(size_t)(mbase + i) * p.ldo + lr] = f2bf(x);
-                                } else {
-                                    const int g = lr / d;
-                                    p.slab[(size_t)b * p.s_req + (size_t)layer * p.s_layer + (size_t)kind * p.s_kind +
-                                           (size_t)g * p.s_kv + (size_t)pos * d + i_in] = f2bf(x);
-                                }
+                                cs[i] = (rotate && row_ok && b >= 0)
+                                            ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
+                                            : make_float2(1.f, 0.f);
+                            }
+                        }
+                        __nv_bfloat16 y[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) {
+                            float x = v[i];
+                            if (rotate) {
+                                const float pr = xch[prow * (CH + 1) + i];
+                                x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
+                            }
+                            y[i] = f2bf(x);
+                        }
+                        named_bar_sync(1, 128);
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) xout[i * 128 + row] = y[i];
+                        named_bar_sync(1, 128);
+                        // 8 features of one token per 16-byte store: a q row, or a K/V cache
+                        // row of the token's request and position
+                        const int nrows = p.amat[mi].rows, rbase = (n_tile - p.amat[mi].tile0) * 128;
+#pragma unroll
+                        for (int k = 0; k < CH / 8; ++k) {
+                            const int c = e + 128 * k, i = c >> 4, r0 = (c & 15) * 8;
+                            const int b = tok_b[c0 + i], f = rbase + r0;
+                            if (b >= 0 && f < nrows) {
+                                const uint4 w = *(const uint4*)(xout + i * 128 + r0);
+                                __nv_bfloat16* dst =
+                                    is_q ? (__nv_bfloat16*)p.out + (size_t)(mbase + i) * p.ldo + f
+                                         : p.slab + (size_t)b * p.s_req + (size_t)layer * p.s_layer +
+                                               (size_t)kind * p.s_kind + (size_t)(f / d) * p.s_kv +
+                                               (size_t)tok_pos[c0 + i] * d + (f % d);
+                                *(uint4*)dst = w;
                             }
                         }
                         named_bar_sync(1, 128);
                         break;
                     }
                     case EPI_LMHEAD: {
+                        // Optional logits (the drafting rows only), then the top-2 of each
+                        // token column over the tile's 128 vocabulary rows: the columns
+                        // cross shared memory, G = 128 / CH threads scan CH rows each in
+                        // row order, and a butterfly over the G threads merges them (ties
+                        // of the top value go to the lower id, whatever the order).
                         const int vid = lr;   // vocab id (lm_head is one matrix)
+                        if (p.logits && row_ok) {
 #pragma unroll 1
-                        for (int i = 0; i < CH; ++i) {
-                            const int m = mbase + i;
-                            if (p.logits && row_ok && m < p.M) {
+                            for (int i = 0; i < CH; ++i) {
+                                const int m = mbase + i;
+                                if (m >= p.M) break;
                                 int lrow = m;
                                 if (p.lm_gamma) {
                                     const int j = m % p.lm_gamma;
@@ -650,30 +664,28 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                                 }
                                 if (lrow >= 0) p.logits[(size_t)lrow * p.vocab + vid] = v[i];
                             }
-                            float a1 = row_ok ? v[i] : -INFINITY, a2 = -INFINITY;
-                            int ai = row_ok ? vid : 0x7fffffff;
+                        }
 #pragma unroll
-                            for (int off = 16; off > 0; off >>= 1) {
-                                const float b1 = __shfl_xor_sync(0xffffffffu, a1, off);
-                                const int bi = __shfl_xor_sync(0xffffffffu, ai, off);
-                                const float b2 = __shfl_xor_sync(0xffffffffu, a2, off);
-                                top2_merge(a1, ai, a2, b1, bi, b2);
-                            }
-                            if (lane == 0) {
-                                lmred[(q * CH + i) * 3 + 0] = a1;
-                                lmred[(q * CH + i) * 3 + 1] = __int_as_float(ai);
-                                lmred[(q * CH + i) * 3 + 2] = a2;
-                            }
-                        }
+                        for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = row_ok ? v[i] : -INFINITY;
                         named_bar_sync(1, 128);
-                        if (e < CH && mbase + e < p.M) {
-                            float a1 = lmred[e * 3 + 0], a2 = lmred[e * 3 + 2];
-                            int ai = __float_as_int(lmred[e * 3 + 1]);
-                            for (int qq = 1; qq < 4; ++qq)
-                                top2_merge(a1, ai, a2, lmred[(qq * CH + e) * 3 + 0],
-                                           __float_as_int(lmred[(qq * CH + e) * 3 + 1]), lmred[(qq * CH + e) * 3 + 2]);
-                            p.records[(size_t)(mbase + e) * p.n_tiles + n_tile] = make_float4(a1, __int_as_float(ai), a2, 0.0f);
+                        constexpr int G = 128 / CH;
+                        const int i = e / G, j = e % G, vbase = n_tile * 128;
+                        float a1 = -INFINITY, a2 = -INFINITY;
+                        int ai = 0x7fffffff;
+#pragma unroll
+                        for (int k = 0; k < CH; ++k) {
+                            const int r = j + G * k;
+                            top2_merge(a1, ai, a2, xch[r * (CH + 1) + i], vbase + r, -INFINITY);
                         }
+#pragma unroll
+                        for (int off = G / 2; off > 0; off >>= 1) {
+                            const float b1 = __shfl_xor_sync(0xffffffffu, a1, off);
+                            const int bi = __shfl_xor_sync(0xffffffffu, ai, off);
+                            const float b2 = __shfl_xor_sync(0xffffffffu, a2, off);
+                            top2_merge(a1, ai, a2, b1, bi, b2);
+                        }
+                        if (j == 0 && mbase + i < p.M)
+                            p.records[(size_t)(mbase + i) * p.n_tiles + n_tile] = make_float4(a1, __int_as_float(ai), a2, 0.0f);
                         named_bar_sync(1, 128);
                         break;
                     }
@@ -740,6 +752,18 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
             nt_total += p.amat[i].ntiles;
         }
         p.n_tiles = nt_total;
+    }
+    // The bf16 epilogues write 8 features of a token per 16-byte store: output rows,
+    // row strides and K/V cache strides must keep 8-element pieces 16-byte aligned.
+    if (p.epi != EPI_F32 && p.epi != EPI_LMHEAD) {
+        const bool q_out = p.epi != EPI_INJECT;
+        if (q_out && (((uintptr_t)p.out & 15) != 0 || p.ldo % 8 != 0)) return (int)cudaErrorInvalidValue;
+        for (int i = 0; i < p.n_amat; ++i)
+            if (p.amat[i].rows % 8 != 0) return (int)cudaErrorInvalidValue;
+        if ((p.epi == EPI_QKV || p.epi == EPI_INJECT) &&
+            (((uintptr_t)p.slab & 15) != 0 || p.d % 8 != 0 || p.s_req % 8 != 0 || p.s_layer % 8 != 0 ||
+             p.s_kind % 8 != 0 || p.s_kv % 8 != 0))
+            return (int)cudaErrorInvalidValue;
     }
     p.units = (long long)p.n_tiles * p.m_tiles * p.KB;
     if (p.units * (long long)kGemmMaxGrid >= (1LL << 32)) return (int)cudaErrorInvalidValue;   // 32-bit partition arithmetic
