@@ -61,6 +61,7 @@ def parse_args():
     ap.add_argument("--separate-pre-step", action="store_true",
                     help="fuse_context + inject_kv as two calls instead of one fuse_inject call")
     ap.add_argument("--no-fold", action="store_true", help="separate RMSNorm kernels in the draft step")
+    ap.add_argument("--fold-head", action="store_true", help="fold the final RMSNorm into the LM head too")
     ap.add_argument("--inject-whole", type=int, default=None, help="1: injection GEMM over whole tiles, 0: split-K slabs")
     ap.add_argument("--trace-dump", default=None,
                     help="write the traced step's raw per-block stamps and launch records to this .npz file")
@@ -467,7 +468,7 @@ def run_gpu(args):
     starts = torch.arange(0, B * T, T, dtype=torch.int32, device=dev)
     # library switches (process-wide) before any call, the prefill included
     D.dflash_diag_set_launch_mode(not args.no_pdl)
-    D.dflash_diag_set_norm_fold(not args.no_fold)
+    D.dflash_diag_set_norm_fold(0 if args.no_fold else 2 if args.fold_head else 1)
     if args.inject_whole is not None:
         D.dflash_diag_set_inject_partition(bool(args.inject_whole))
     if args.l2_prefetch is not None:
@@ -732,7 +733,8 @@ def run_gpu(args):
             "step_options": {"conditioning": args.conditioning,
                              "pre_step": ("fuse_context + ingest_fused_input" if args.conditioning == "input-fusion"
                                           else "two calls" if args.separate_pre_step else "fuse_inject (one call)"),
-                             "norm_fold": not args.no_fold, "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch(),
+                             "norm_fold": "off" if args.no_fold else "with the LM head" if args.fold_head else "on",
+                             "gemm_l2_prefetch_tiles": D.dflash_diag_gemm_prefetch(),
                              "split_tile_finisher": "last arriver" if args.last_arriver else "first contributor",
                              "gemm_pre_stages": args.pre_stages if args.pre_stages is not None else "library default (6)"},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl

@@ -275,16 +275,33 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                 const bool copy_out = p.norm_out && t / m_tiles == 0;
                 if (m_tile != cur_mt) {
                     // inverse RMS of the m-tile's rows from the producer's per-tile
-                    // partial sums, added in tile order (the same in every CTA); each
-                    // warp keeps its own copy, so the two warps never wait for each other
-                    // inside the stage loop
+                    // partial sums; each warp keeps its own copy, so the two warps never
+                    // wait for each other inside the stage loop.  A row's tiles are split
+                    // into G contiguous runs, one per lane, each added in tile order from
+                    // loads issued 16 at a time, then the G runs meet in a fixed butterfly:
+                    // the same order in every CTA, and one or two round trips of latency
+                    // instead of one per tile.
                     __syncwarp();
-                    for (int r = lane; r < NT; r += 32) {
+                    constexpr int G = NT < 32 ? 32 / NT : 1;   // lanes per row
+                    const int T = p.ssq_tiles, per = (T + G - 1) / G;
+                    for (int r0 = 0; r0 < NT; r0 += 32 / G) {
+                        const int r = r0 + lane / G, g = lane % G;
                         const int m = m_tile * NT + r;
                         float ss = 0.f;
-                        if (m < p.M)
-                            for (int j = 0; j < p.ssq_tiles; ++j) ss += __ldcg(p.ssq_in + (size_t)j * p.ssq_ld + m);
-                        inv_w[r] = 1.0f / sqrtf(ss / (float)p.norm_h + p.eps);
+                        if (r < NT && m < p.M) {
+                            const int j1 = min(T, (g + 1) * per);
+                            for (int j = g * per; j < j1; j += 16) {
+                                float part[16];
+#pragma unroll
+                                for (int k = 0; k < 16; ++k)
+                                    part[k] = j + k < j1 ? __ldcg(p.ssq_in + (size_t)(j + k) * p.ssq_ld + m) : 0.f;
+#pragma unroll
+                                for (int k = 0; k < 16; ++k) ss += part[k];
+                            }
+                        }
+#pragma unroll
+                        for (int off = 1; off < G; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                        if (r < NT && g == 0) inv_w[r] = 1.0f / sqrtf(ss / (float)p.norm_h + p.eps);
                     }
                     __syncwarp();
                     cur_mt = m_tile;
