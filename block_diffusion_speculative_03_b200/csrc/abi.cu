@@ -31,7 +31,7 @@ static bool g_inject_whole = true;
 // Whether the final norm is folded into the LM-head GEMM too (see draft_bf16).
 static bool g_fold_head = false;
 // O-projection on the SMs the attention does not hold (see layers_bf16).
-static bool g_o_beside_attention = true;
+static bool g_o_beside_attention = false;
 constexpr int kFoldMaxNT = 16;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -1362,6 +1362,17 @@ int dflash_diag_set_gemm_pre_stages(int stages) {
     if (stages < 0 || stages > 64) return DFLASH_INVALID_ARG;
     set_gemm_pre_stages(stages);
     return DFLASH_OK;
+}
+
+int dflash_diag_set_gemm_max_cluster(int max_cluster) {
+    if (max_cluster < 0 || max_cluster > 4) return DFLASH_INVALID_ARG;
+    set_gemm_max_cluster(max_cluster);
+    return DFLASH_OK;
+}
+
+int dflash_diag_gemm_max_active_clusters(int cluster_size) {
+    if (cluster_size < 2 || cluster_size > 8) return 0;
+    return gemm_max_active_clusters(cluster_size);
 }
 
 int dflash_diag_set_split_finisher(int last_arriver) {

@@ -41,6 +41,23 @@ DF_DEV void mbar_init(uint64_t* bar, uint32_t count) {
 DF_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 DF_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Thread-block cluster barrier (every thread of every CTA of the cluster), and
+// distributed shared memory: the address of the same variable in CTA `rank` of
+// the cluster, and a 16-byte store into it that completes `bytes` on that
+// CTA's mbarrier.
+DF_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+DF_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+DF_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+DF_DEV void st_async_v4(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+                 : "memory");
+}
+
 DF_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");

@@ -52,6 +52,9 @@ struct GemmParams {
                                  //    in-order accumulation over all of K, whatever M and the grid
     int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
     int pre_stages;              // ring stages filled with weights before the wait (0: the whole ring)
+    int cluster;                 // >= 2: CTAs in thread-block clusters of this size, each cluster owning
+                                 //    whole tiles, split tiles reduced through distributed shared
+                                 //    memory (set by the launcher for 16-token tiles when it pays)
     int last_arriver;            // split tiles: 1 = finished by whichever contributor counts in last;
                                  //    0 = by the contributor holding the tile's first k-blocks, which
                                  //    waits for the others' partials and stores none of its own
@@ -140,6 +143,9 @@ int gemm_pre_stages();
 void set_gemm_pre_stages(int stages);
 int gemm_last_arriver();
 void set_gemm_last_arriver(int on);
+int gemm_max_cluster();
+void set_gemm_max_cluster(int c);
+int gemm_max_active_clusters(int c);   // resident clusters of c CTAs of the cluster-mode 16-token kernel
 
 // Host launcher (gemm_tc.cu).  Fills the derived fields (KB, tiles, units,
 // ctas) and launches on `stream`.  Returns a cudaError_t; cudaErrorInvalidValue

@@ -8,6 +8,8 @@
 // epilogue while the next tile accumulates in the other buffer; warps 6 and 7,
 // when the GEMM consumes RMS-normalised rows, rewrite each token tile in shared
 // memory as R(x * inv_rms * gain) between its arrival and the MMA.
+#include <algorithm>
+
 #include "gemm.cuh"
 
 namespace df {
@@ -17,7 +19,7 @@ constexpr long long kGemmMaxGrid = 160;
 
 // Tile configuration per token width NT: one CTA per SM with the deepest ring
 // that fits (two CTAs per SM with half the ring measured slower at batch 1).
-template <int NT>
+template <int NT, bool CLU = false>
 struct GemmCfg {
     static constexpr int THREADS = 256;
     static constexpr bool TWO_PER_SM = false;
@@ -28,11 +30,17 @@ struct GemmCfg {
     static constexpr int XCH_FLOATS = 128 * (CH + 1);
     static constexpr int GAIN_MAX = 4096;                // RMSNorm gain elements staged in shared memory
     static constexpr int MISC_BYTES = 6144 + GAIN_MAX * 2;
+    // Cluster mode (its own instance, so the whole-grid kernel keeps the deeper ring):
+    // the partials of up to 3 peers of the cluster land here, rows padded to NT + 4
+    // floats so 16-byte reads of a row are conflict-free.
+    static constexpr int LAND_SLOTS = CLU ? 3 : 0;
+    static constexpr int LAND_LD = NT + 4;
+    static constexpr int LAND_BYTES = LAND_SLOTS * 128 * LAND_LD * 4;
     static constexpr int SMEM_CAP = TWO_PER_SM ? (233472 / 2 - 2048) : 232448;
-    static constexpr int BUDGET = SMEM_CAP - 1024 - XCH_FLOATS * 4 - MISC_BYTES;
+    static constexpr int BUDGET = SMEM_CAP - 1024 - XCH_FLOATS * 4 - LAND_BYTES - MISC_BYTES;
     static constexpr int STAGES_RAW = BUDGET / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
-    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCH_FLOATS * 4 + MISC_BYTES;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCH_FLOATS * 4 + LAND_BYTES + MISC_BYTES;
     static constexpr uint32_t TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
     static constexpr int MIN_BLOCKS = TWO_PER_SM ? 2 : 1;
 };
@@ -59,10 +67,10 @@ DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
+template <int NT, bool CLU>
+__global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::MIN_BLOCKS)
     k_gemm_tc(const __grid_constant__ GemmParams p) {
-    using C = GemmCfg<NT>;
+    using C = GemmCfg<NT, CLU>;
     constexpr int S = C::STAGES;
     constexpr int CH = C::CH;
     extern __shared__ uint8_t smem_raw[];
@@ -71,12 +79,14 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     uint8_t* sB = smem + S * C::A_BYTES;
     float* xch = (float*)(sB + S * C::B_BYTES);
     __nv_bfloat16* const xout = (__nv_bfloat16*)xch;   // epilogue outputs, token-major [CH][128] bf16
-    uint64_t* full = (uint64_t*)(xch + C::XCH_FLOATS);
+    float* land = xch + C::XCH_FLOATS;                 // [LAND_SLOTS][128][LAND_LD] peers' partials
+    uint64_t* full = (uint64_t*)(land + C::LAND_BYTES / 4);
     uint64_t* empty = full + S;
     uint64_t* accf = empty + S;
     uint64_t* acce = accf + 2;
     uint64_t* drain = acce + 2;
-    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+    uint64_t* landb = drain + 1;      // cluster mode: the peers' partials have landed
+    uint32_t* tmem_slot = (uint32_t*)(landb + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* s_flag = (int*)(tmem_slot + 2);
     int* tok_b = s_flag + 1;          // [NT]
@@ -84,13 +94,41 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     float* inv_s = (float*)(tok_pos + NT);   // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
     uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + 2 * NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
     __nv_bfloat16* sgain = (__nv_bfloat16*)(((uintptr_t)(ready + S) + 15) & ~(uintptr_t)15);   // [GAIN_MAX]
-    static_assert((2 * S + 5) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+    static_assert((2 * S + 6) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
                       C::MISC_BYTES, "misc");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 8 : nullptr;
     const long long clk0 = clock64();
     if (trace && threadIdx.x == 0) trace[0] = (long long)globaltimer_ns();
+
+    // Work partition.  Whole grid: CTA p owns k-block units [pU/P, (p+1)U/P) of all
+    // output tiles.  Cluster mode (CL >= 2): cluster q of Q owns whole tiles
+    // [qT/Q, (q+1)T/Q), and its CL CTAs split that cluster's units the same way,
+    // so every split tile's contributors are CTAs of one cluster.
+    const long long U = p.units;
+    const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
+    const int CL = (CLU && p.cluster >= 2) ? p.cluster : 0;
+    long long ubase = 0, Uloc = U;
+    int Ploc = P, rloc = cta, cbase = 0;
+    if constexpr (C::LAND_SLOTS > 0) {
+        if (CL) {
+            const int q = cta / CL, Q = P / CL;
+            const long long T = U / KB;
+            const long long t0 = T * q / Q, t1 = T * (q + 1) / Q;
+            ubase = t0 * KB;
+            Uloc = (t1 - t0) * KB;
+            Ploc = CL;
+            rloc = cta % CL;
+            cbase = q * CL;
+        }
+    }
+    long long u_begin = ubase + sk_begin(rloc, Uloc, Ploc), u_end = ubase + sk_begin(rloc + 1, Uloc, Ploc);
+    if (p.whole_tiles && !CL) {   // tile-granular ranges: no tile is split, no partials
+        const long long T = U / KB;
+        u_begin = (T * cta / P) * KB;
+        u_end = (T * (cta + 1) / P) * KB;
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -102,6 +140,16 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
         }
         for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 2);   // one arrival per normaliser warp
         mbar_init(drain, 1);
+        mbar_init(landb, 1);
+        if (CL) {
+            // The CTA's last segment is a split tile it finishes when it starts at the
+            // tile's k-block 0 and ends inside it: expect its peers' partials.
+            const long long tl = (u_end - 1) / KB;
+            if (u_begin <= tl * KB && u_end < (tl + 1) * KB) {
+                const int nc = sk_owner((tl + 1) * KB - 1 - ubase, Uloc, Ploc) - sk_owner(tl * KB - ubase, Uloc, Ploc) + 1;
+                mbar_arrive_expect_tx(landb, (uint32_t)((nc - 1) * 128 * NT * 4));
+            }
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -113,14 +161,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    const long long U = p.units;
-    const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
-    long long u_begin = sk_begin(cta, U, P), u_end = sk_begin(cta + 1, U, P);
-    if (p.whole_tiles) {   // tile-granular ranges: no tile is split, no partials
-        const long long T = U / KB;
-        u_begin = (T * cta / P) * KB;
-        u_end = (T * (cta + 1) / P) * KB;
+    if (CL) {
+        // every peer's landing barrier is initialised before any partial is sent
+        cluster_arrive();
+        cluster_wait();
     }
 
     griddep_launch();
@@ -430,23 +474,50 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
             // published partials, before the accumulator wait so that the round trip
             // overlaps the CTA's last MMAs.  With p.last_arriver every contributor
             // publishes and counts, and the one that counts last finishes.
+            // In cluster mode the peers' partials arrive in this CTA's shared memory
+            // (distributed shared-memory stores completing on landb), so the finisher
+            // waits on its own barrier; whole-grid mode counts published partials in
+            // global memory.
             const bool whole = (kb0 == 0 && kb1 == KB);
-            const bool fin_first = !whole && !p.last_arriver && kb0 == 0;
+            const bool fin_first = !whole && (CL || !p.last_arriver) && kb0 == 0;
             int first = cta, nc = 1;
             if (!whole) {
-                const uint32_t t32 = (uint32_t)t, K32 = (uint32_t)KB, U32 = (uint32_t)U, P32 = (uint32_t)P;
-                first = (int)sk32_owner(t32 * K32, U32, P32);
-                nc = (int)sk32_owner((t32 + 1) * K32 - 1, U32, P32) - first + 1;
+                const uint32_t t32 = (uint32_t)(t * KB - ubase), K32 = (uint32_t)KB, U32 = (uint32_t)Uloc,
+                               P32 = (uint32_t)Ploc;
+                first = (int)sk32_owner(t32, U32, P32);
+                nc = (int)sk32_owner(t32 + K32 - 1, U32, P32) - first + 1;
+                first += cbase;
             }
             bool ok = true;
-            if (fin_first && e == 0) ok = count_wait(&p.counters[t], nc - 1, abort_flag, p.status);
+            if (fin_first) {
+                if (CL)
+                    ok = mbar_wait(landb, 0, abort_flag, p.status);
+                else if (e == 0)
+                    ok = count_wait(&p.counters[t], nc - 1, abort_flag, p.status);
+            }
             ok = ok && mbar_wait(&accf[buf], use & 1, abort_flag, p.status);
             if (named_bar_or(1, 128, !ok)) break;   // leave together: later named barriers stay matched
             if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
             tc_fence_after();
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
             bool finish = true;
-            if (!whole && !fin_first) {
+            if (!whole && !fin_first && CL) {
+                // Send the partial (all NT columns of this thread's row) into the
+                // finisher's landing slot for this rank, 16 bytes per store.
+                const uint32_t fr = (uint32_t)(first - cbase);
+                const uint32_t slot = (uint32_t)(rloc - (first - cbase) - 1);
+                const uint32_t raddr = mapa_shared(smem_u32(land + ((size_t)slot * 128 + row) * C::LAND_LD), fr);
+                const uint32_t rbar = mapa_shared(smem_u32(landb), fr);
+#pragma unroll 1
+                for (int c0 = 0; c0 < NT; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tb + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        st_async_v4(raddr + (uint32_t)(c0 + i) * 4, v[i], v[i + 1], v[i + 2], v[i + 3], rbar);
+                }
+                finish = false;
+            } else if (!whole && !fin_first) {
                 float* dst = p.partial + (size_t)sk32_slot(cta, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += 16) {
@@ -484,7 +555,25 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                     float v[CH];
 #pragma unroll
                     for (int h = 0; h < CH; h += 16) tmem_ld16(tb + c0 + h, v + h);
-                    if (!whole) {
+                    if (!whole && CL) {
+                        // this CTA first, then the peers' partials in rank order
+                        float acc[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) acc[i] = 0.0f + v[i];
+                        for (int b = 1; b < nc; ++b) {
+                            const float* src = land + ((size_t)(b - 1) * 128 + row) * C::LAND_LD + c0;
+#pragma unroll
+                            for (int i = 0; i < CH; i += 4) {
+                                const float4 w = *reinterpret_cast<const float4*>(src + i);
+                                acc[i] += w.x;
+                                acc[i + 1] += w.y;
+                                acc[i + 2] += w.z;
+                                acc[i + 3] += w.w;
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) v[i] = acc[i];
+                    } else if (!whole) {
                         float acc[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) acc[i] = 0.0f;
@@ -710,7 +799,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
                         break;
                     }
                 }
-                if (!whole && e == 0) p.counters[t] = 0;
+                if (!whole && !CL && e == 0) p.counters[t] = 0;
             }
             tc_fence_before();
             mbar_arrive(&acce[buf]);
@@ -726,24 +815,115 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, GemmCfg<NT>::MIN_BLOCKS)
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+    if (CL) {
+        // no CTA leaves while a peer may still store into its shared memory
+        cluster_arrive();
+        cluster_wait();
+    }
     if (trace && threadIdx.x == 0) {
         trace[6] = (long long)globaltimer_ns();
         trace[7] = clock64() - clk0;
     }
 }
 
-template <int NT>
+template <int NT, bool CLU>
+static cudaError_t set_smem_attr() {
+    static bool done = false;
+    if (done) return cudaSuccess;
+    cudaError_t e =
+        cudaFuncSetAttribute(k_gemm_tc<NT, CLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<NT, CLU>::SMEM);
+    done = e == cudaSuccess;
+    return e;
+}
+
+template <int NT, bool CLU>
 static int launch_nt(GemmParams& p, cudaStream_t stream) {
-    using C = GemmCfg<NT>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return (int)e;
-        attr_done = true;
+    using C = GemmCfg<NT, CLU>;
+    cudaError_t e = set_smem_attr<NT, CLU>();
+    if (e != cudaSuccess) return (int)e;
+    if (CLU) {
+        ensure_carveout((const void*)k_gemm_tc<NT, CLU>);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.ctas);
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = (size_t)C::SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)p.cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, k_gemm_tc<NT, CLU>, p);
+    } else {
+        e = launch_k(k_gemm_tc<NT, CLU>, dim3(p.ctas), dim3(C::THREADS), (size_t)C::SMEM, stream, p);
     }
-    cudaError_t e = launch_k(k_gemm_tc<NT>, dim3(p.ctas), dim3(C::THREADS), (size_t)C::SMEM, stream, p);
     if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
+}
+
+// Clusters of c CTAs of the 16-token kernel that can be resident at once (the
+// clusters of one launch must fit a GPC each), cached; 0 if none.
+static int max_active_clusters16(int c) {
+    static int cached[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    if (c < 2 || c > 8) return 0;
+    if (cached[c] >= 0) return cached[c];
+    int n = 0;
+    if (set_smem_attr<16, true>() == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(c * 8);
+        cfg.blockDim = dim3(GemmCfg<16, true>::THREADS);
+        cfg.dynamicSmemBytes = (size_t)GemmCfg<16, true>::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, (const void*)k_gemm_tc<16, true>, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cached[c] = n;
+    return n;
+}
+
+// Cluster mode pays when the cluster partition's longest CTA range (whole tiles per
+// cluster, split over its CTAs) is shorter than the whole-grid range plus the
+// global-memory split-tile fix-up, which costs about kFixupUnits weight tiles of
+// streaming at the end of every launch.  Off by default: on a 148-SM B200, 74 / 45 /
+// 33 clusters of 2 / 3 / 4 CTAs are resident, which fits none of the 16-token
+// projections of the drafters here well enough (QKV's 48 tiles need 48 clusters of
+// 3; the O-projection's 32 tiles on 128 CTAs with the shallower ring measured
+// slower than the whole-grid kernel).
+constexpr long long kFixupUnits = 6;
+static int g_max_cluster = 0;
+int gemm_max_cluster() { return g_max_cluster; }
+void set_gemm_max_cluster(int c) {
+    constexpr int cmax = GemmCfg<16, true>::LAND_SLOTS + 1;
+    g_max_cluster = c < 0 ? 0 : (c > cmax ? cmax : c);
+}
+int gemm_max_active_clusters(int c) { return max_active_clusters16(c); }
+
+static void pick_cluster(GemmParams& p, int num_sms) {
+    p.cluster = 0;
+    if (g_max_cluster < 2 || p.whole_tiles) return;
+    const long long T = (long long)p.n_tiles * p.m_tiles, KB = p.KB;
+    long long best = (T * KB + num_sms - 1) / num_sms + kFixupUnits;
+    for (int c = 2; c <= g_max_cluster; ++c) {
+        if (KB < c) break;
+        const long long Q = std::min<long long>(max_active_clusters16(c), std::min<long long>(T, num_sms / c));
+        if (Q < 1) continue;
+        const long long cost = (((T + Q - 1) / Q) * KB + c - 1) / c;
+        if (cost < best) {
+            best = cost;
+            p.cluster = c;
+            p.ctas = (int)(Q * c);
+        }
+    }
 }
 
 static int g_l2_prefetch = 0;
@@ -784,16 +964,19 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
     }
     p.units = (long long)p.n_tiles * p.m_tiles * p.KB;
     if (p.units * (long long)kGemmMaxGrid >= (1LL << 32)) return (int)cudaErrorInvalidValue;   // 32-bit partition arithmetic
+    const bool auto_grid = p.ctas <= 0;
     if (p.ctas <= 0 || p.ctas > num_sms) p.ctas = num_sms;
     if ((long long)p.ctas > p.units) p.ctas = (int)p.units;
     if (p.whole_tiles && (long long)p.ctas > p.units / p.KB) p.ctas = (int)(p.units / p.KB);
     if (p.units == 0) return 0;
+    p.cluster = 0;
+    if (nt == 16 && auto_grid) pick_cluster(p, num_sms);
     switch (nt) {
-    case 16: return launch_nt<16>(p, stream);
-    case 32: return launch_nt<32>(p, stream);
-    case 64: return launch_nt<64>(p, stream);
-    case 128: return launch_nt<128>(p, stream);
-    case 256: return launch_nt<256>(p, stream);
+    case 16: return p.cluster >= 2 ? launch_nt<16, true>(p, stream) : launch_nt<16, false>(p, stream);
+    case 32: return launch_nt<32, false>(p, stream);
+    case 64: return launch_nt<64, false>(p, stream);
+    case 128: return launch_nt<128, false>(p, stream);
+    case 256: return launch_nt<256, false>(p, stream);
     default: return (int)cudaErrorInvalidValue;
     }
 }

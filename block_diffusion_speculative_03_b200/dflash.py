@@ -109,6 +109,8 @@ def lib():
         "dflash_diag_gemm_prefetch": (i32, []),
         "dflash_diag_set_gemm_pre_stages": (i32, [i32]),
         "dflash_diag_set_split_finisher": (i32, [i32]),
+        "dflash_diag_set_gemm_max_cluster": (i32, [i32]),
+        "dflash_diag_gemm_max_active_clusters": (i32, [i32]),
         "dflash_diag_set_norm_fold": (i32, [i32]),
         "dflash_diag_set_inject_partition": (i32, [i32]),
         "dflash_diag_set_o_beside_attention": (i32, [i32]),
@@ -146,7 +148,8 @@ def exported_symbols() -> list:
             "dflash_diag_gemm_bf16", "dflash_diag_partition", "dflash_diag_synth_target", "dflash_diag_arch",
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_set_gemm_prefetch", "dflash_diag_gemm_prefetch",
-            "dflash_diag_set_gemm_pre_stages", "dflash_diag_set_split_finisher",
+            "dflash_diag_set_gemm_pre_stages", "dflash_diag_set_split_finisher", "dflash_diag_set_gemm_max_cluster",
+            "dflash_diag_gemm_max_active_clusters",
             "dflash_diag_set_norm_fold", "dflash_diag_set_inject_partition",
             "dflash_diag_set_o_beside_attention",
             "dflash_diag_wait_selftest",
@@ -362,6 +365,14 @@ def dflash_diag_set_gemm_pre_stages(stages: int) -> int:
 
 def dflash_diag_set_split_finisher(last_arriver: bool) -> int:
     return _chk(lib().dflash_diag_set_split_finisher(int(bool(last_arriver))), "dflash_diag_set_split_finisher")
+
+
+def dflash_diag_set_gemm_max_cluster(max_cluster: int) -> int:
+    return _chk(lib().dflash_diag_set_gemm_max_cluster(int(max_cluster)), "dflash_diag_set_gemm_max_cluster")
+
+
+def dflash_diag_gemm_max_active_clusters(cluster_size: int) -> int:
+    return int(lib().dflash_diag_gemm_max_active_clusters(int(cluster_size)))
 
 
 def dflash_diag_gemm_prefetch() -> int:

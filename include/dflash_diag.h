@@ -204,6 +204,21 @@ int dflash_diag_gemm_prefetch(void);
  * finishing memory round trips less contended. */
 int dflash_diag_set_gemm_pre_stages(int stages);
 
+/* Largest thread-block cluster the tensor-core GEMM may use for 16-token tiles
+ * (process-wide, 0..4; default 0 = never, as measured faster on B200 for the
+ * drafter shapes here; 1 = never).  In cluster mode each cluster
+ * owns whole output tiles and its CTAs split their k-blocks; a split tile's
+ * partial accumulators travel to the CTA that finishes it through distributed
+ * shared memory instead of global memory.  The launcher takes the cluster size
+ * (2..max) whose partition is shorter than the whole-grid partition plus its
+ * global-memory fix-up, if any. */
+int dflash_diag_set_gemm_max_cluster(int max_cluster);
+
+/* How many clusters of `cluster_size` CTAs (2..8) of the cluster-mode GEMM kernel
+ * can be resident at once on the current device (a cluster must fit one GPC);
+ * 0 if none or out of range.  The launcher's choice of cluster size uses this. */
+int dflash_diag_gemm_max_active_clusters(int cluster_size);
+
 /* How the tensor-core GEMM finishes an output tile whose k-blocks are split
  * over several CTAs (process-wide; applies to launches enqueued afterwards).
  * 0 (the default): the CTA holding the tile's first k-blocks finishes it; it

@@ -75,6 +75,27 @@ def test_split_tile_finishers_agree_bitwise(M, N, K, grid):
         ref, first = _run(M, N, K, grid=grid, calls=2)
     finally:
         D.dflash_diag_set_split_finisher(False)
+        D.dflash_diag_set_gemm_max_cluster(0)
     _close(ref, first[0], K)
     for got in last + first[1:]:
         assert torch.equal(got, first[0])
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 6144, 4096), (16, 4096, 4096), (16, 24576, 4096), (5, 1024, 12288),
+                                   (16, 128, 256), (1, 384, 704), (9, 640, 1024)])
+def test_cluster_partition_matches_fp64_and_repeats(M, N, K):
+    """16-token tiles in thread-block clusters (tiles owned by clusters, split
+    tiles reduced through distributed shared memory; on a single tile the whole
+    cluster contributes to it) against the fp64 product and against the
+    whole-grid partition, with identical bits on repeated calls."""
+    try:
+        D.dflash_diag_set_gemm_max_cluster(4)
+        ref, clu = _run(M, N, K, calls=3)
+        D.dflash_diag_set_gemm_max_cluster(0)
+        _, (grid,) = _run(M, N, K)
+    finally:
+        D.dflash_diag_set_gemm_max_cluster(0)
+    for got in clu + [grid]:
+        assert not torch.isnan(got).any()
+        _close(ref, got, K)
+    assert torch.equal(clu[0], clu[1]) and torch.equal(clu[1], clu[2])
