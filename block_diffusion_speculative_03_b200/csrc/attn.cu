@@ -456,18 +456,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         rpo[s2] = s2 < nsplit ? cluster.map_shared_rank(po, s2) : po;
         rpml[s2] = s2 < nsplit ? cluster.map_shared_rank(pml, s2) : pml;
     }
-    // One round of distributed-shared-memory reads per output chunk: each thread
-    // fetches every split's (base, sum) of its row and O chunk together, and forms
-    // the row's merge weights itself (exact powers of two times 1 / the merged sum).
+    // One round of distributed-shared-memory reads per output piece: columns
+    // [c, c+4) and [c + D/2, c + D/2 + 4) of a row, so the lanes of a half-warp read
+    // contiguous 256-byte runs.  Each thread fetches every split's (base, sum) of its
+    // row and its 8 O columns together, and forms the row's merge weights itself
+    // (exact powers of two times 1 / the merged sum).  At up to 16 rows per CTA every
+    // thread has one piece.
     const int nr = r_hi - r_lo;
-    for (int idx = tid; idx < nr * (D / 4); idx += kAttnThreads) {
-        const int rr = idx / (D / 4), c = (idx % (D / 4)) * 4, r = r_lo + rr;
+    for (int idx = tid; idx < nr * (D / 8); idx += kAttnThreads) {
+        const int rr = idx / (D / 8), c = (idx % (D / 8)) * 4, r = r_lo + rr;
         float2 ml[kAttnMaxSplits];
-        float4 v[kAttnMaxSplits];
+        float4 va[kAttnMaxSplits], vb[kAttnMaxSplits];
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
-            ml[s2] = s2 < nsplit ? rpml[s2][r] : make_float2(0.f, 0.f);
-            v[s2] = s2 < nsplit ? *reinterpret_cast<const float4*>(rpo[s2] + r * PO_LD + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s2 < nsplit) {
+                ml[s2] = rpml[s2][r];
+                va[s2] = *reinterpret_cast<const float4*>(rpo[s2] + r * PO_LD + c);
+                vb[s2] = *reinterpret_cast<const float4*>(rpo[s2] + r * PO_LD + c + D / 2);
+            } else {
+                ml[s2] = make_float2(0.f, 0.f);
+                va[s2] = vb[s2] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
         float M = -INFINITY;
 #pragma unroll
@@ -482,21 +491,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
             L += wv[s2] * ml[s2].y;
         }
         const float inv = L > 0.f ? 1.0f / L : 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
             if (s2 < nsplit) {
                 const float w = wv[s2] * inv;
-                acc.x += w * v[s2].x;
-                acc.y += w * v[s2].y;
-                acc.z += w * v[s2].z;
-                acc.w += w * v[s2].w;
+                acc[0] += w * va[s2].x;
+                acc[1] += w * va[s2].y;
+                acc[2] += w * va[s2].z;
+                acc[3] += w * va[s2].w;
+                acc[4] += w * vb[s2].x;
+                acc[5] += w * vb[s2].y;
+                acc[6] += w * vb[s2].z;
+                acc[7] += w * vb[s2].w;
             }
         }
         const int j = r / p.G, hh = r % p.G;
         __nv_bfloat16* dst = p.out + ((size_t)(b * p.gamma + j) * p.nq + (size_t)(g * p.G + hh)) * D + c;
-        *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc.x, acc.y);
-        *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
+        *reinterpret_cast<uint2*>(dst + D / 2) = make_uint2(pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
     }
     if (trace && tid == 0) trace[7] = (long long)globaltimer_ns();
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
