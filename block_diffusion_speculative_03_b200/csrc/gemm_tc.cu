@@ -52,9 +52,6 @@ DF_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
 // GEMM's last tiles, where 64-bit divisions cost.
 DF_DEV uint32_t sk32_begin(uint32_t p, uint32_t U, uint32_t P) { return p * U / P; }
 DF_DEV uint32_t sk32_owner(uint32_t u, uint32_t U, uint32_t P) { return ((u + 1) * P - 1) / U; }
-DF_DEV int sk32_slot(uint32_t p, uint32_t tile, uint32_t KB, uint32_t U, uint32_t P) {
-    return (int)(2 * p + (tile == sk32_begin(p, U, P) / KB ? 0 : 1));
-}
 
 // Top-2 merge: a <- top2(a ∪ b); ties of the top value go to the lower id.
 DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
@@ -103,14 +100,24 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     if (trace && threadIdx.x == 0) trace[0] = (long long)globaltimer_ns();
 
     // Work partition.  Whole grid: CTA p owns k-block units [pU/P, (p+1)U/P) of all
-    // output tiles.  Cluster mode (CL >= 2): cluster q of Q owns whole tiles
-    // [qT/Q, (q+1)T/Q), and its CL CTAs split that cluster's units the same way,
-    // so every split tile's contributors are CTAs of one cluster.
+    // output tiles.  Grouped (several token tiles): CTA p = g * m_tiles + m takes token
+    // tile m of group g's share of the (weight tile, k-block) units, so the m_tiles
+    // CTAs of a group read each weight tile at about the same time (one HBM read, the
+    // others L2 hits) instead of at unrelated offsets.  Cluster mode (CL >= 2):
+    // cluster q of Q owns whole tiles [qT/Q, (q+1)T/Q), and its CL CTAs split that
+    // cluster's units the same way, so every split tile's contributors are CTAs of
+    // one cluster.  rloc is the CTA's index within its partition (group, rank).
     const long long U = p.units;
     const int P = p.ctas, cta = blockIdx.x, KB = p.KB, m_tiles = p.m_tiles;
     const int CL = (CLU && p.cluster >= 2) ? p.cluster : 0;
-    long long ubase = 0, Uloc = U;
-    int Ploc = P, rloc = cta, cbase = 0;
+    // (only the widest token tile ever has several: narrower widths are picked for M <= NT)
+    const int GM = (NT == 256 && p.grouped && !CL) ? m_tiles : 1;   // CTAs per group
+    const int gm = cta % GM;                                             // the group's token tile
+    long long ubase = 0, Uloc = U / GM;
+    int Ploc = P / GM, rloc = cta / GM, cbase = 0;
+    // global tile of partition unit u, and the CTA of partition index i
+    auto tile_of = [&](long long u) -> long long { return GM > 1 ? (u / KB) * m_tiles + gm : u / KB; };
+    auto cta_of = [&](int i) -> int { return (cbase + i) * GM + gm; };
     if constexpr (C::LAND_SLOTS > 0) {
         if (CL) {
             const int q = cta / CL, Q = P / CL;
@@ -125,9 +132,9 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     }
     long long u_begin = ubase + sk_begin(rloc, Uloc, Ploc), u_end = ubase + sk_begin(rloc + 1, Uloc, Ploc);
     if (p.whole_tiles && !CL) {   // tile-granular ranges: no tile is split, no partials
-        const long long T = U / KB;
-        u_begin = (T * cta / P) * KB;
-        u_end = (T * (cta + 1) / P) * KB;
+        const long long T = Uloc / KB;
+        u_begin = (T * rloc / Ploc) * KB;
+        u_end = (T * (rloc + 1) / Ploc) * KB;
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -179,7 +186,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             const int s_pre = (p.pre_stages > 0 && p.pre_stages < S) ? p.pre_stages : S;
             const int n_ahead = s_pre + p.l2_prefetch;
             for (long long u = u_begin, idx = 0; u < u_end && idx < n_ahead;) {
-                const long long t = u / KB;
+                const long long t = tile_of(u);
                 const int kb0 = (int)(u % KB);
                 const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
                 const int n_tile = (int)(t / m_tiles);
@@ -214,7 +221,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             long long issued = 0;
             bool ok = true;
             for (long long u = u_begin; u < u_end && ok;) {
-                const long long t = u / KB;
+                const long long t = tile_of(u);
                 const int kb0 = (int)(u % KB);
                 const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
                 const int n_tile = (int)(t / m_tiles), m_tile = (int)(t % m_tiles);
@@ -311,7 +318,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             uint32_t round = 0;
             bool ok = true;
             for (long long u = u_begin; u < u_end && ok;) {
-                const long long t = u / KB;
+                const long long t = tile_of(u);
                 const int kb0 = (int)(u % KB);
                 const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
                 const int m_tile = (int)(t % m_tiles);
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
         int seg = 0;
         int tok_mt = -1;                        // m-tile whose token map tok_b / tok_pos holds
         for (long long u = u_begin; u < u_end;) {
-            const long long t = u / KB;
+            const long long t = tile_of(u);
             const int kb0 = (int)(u % KB);
             const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
             const int n_tile = (int)(t / m_tiles), m_tile = (int)(t % m_tiles);
@@ -480,14 +487,25 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             // global memory.
             const bool whole = (kb0 == 0 && kb1 == KB);
             const bool fin_first = !whole && (CL || !p.last_arriver) && kb0 == 0;
-            int first = cta, nc = 1;
+            // contributors: partition indices firsti .. firsti + nc - 1 (CTAs cta_of(i));
+            // tn: the tile's weight-tile index in partition units (its k-block 0 at tn * KB)
+            const long long tn = GM > 1 ? t / m_tiles : t;
+            int first = cta, firsti = rloc, nc = 1;
             if (!whole) {
-                const uint32_t t32 = (uint32_t)(t * KB - ubase), K32 = (uint32_t)KB, U32 = (uint32_t)Uloc,
+                const uint32_t t32 = (uint32_t)(tn * KB - ubase), K32 = (uint32_t)KB, U32 = (uint32_t)Uloc,
                                P32 = (uint32_t)Ploc;
-                first = (int)sk32_owner(t32, U32, P32);
-                nc = (int)sk32_owner(t32 + K32 - 1, U32, P32) - first + 1;
-                first += cbase;
+                firsti = (int)sk32_owner(t32, U32, P32);
+                nc = (int)sk32_owner(t32 + K32 - 1, U32, P32) - firsti + 1;
+                first = cta_of(firsti);
             }
+            // partial slot of the CTA with partition index i for this tile: its first
+            // segment (slot 2 * CTA) or its last (2 * CTA + 1)
+            // (32-bit arithmetic: the launcher keeps every unit index below 2^32)
+            auto slot_of = [&](int i) -> int {
+                const uint32_t first_tn =
+                    ((uint32_t)ubase + sk32_begin((uint32_t)i, (uint32_t)Uloc, (uint32_t)Ploc)) / (uint32_t)KB;
+                return 2 * cta_of(i) + (first_tn == (uint32_t)tn ? 0 : 1);
+            };
             bool ok = true;
             if (fin_first) {
                 if (CL)
@@ -518,7 +536,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                 }
                 finish = false;
             } else if (!whole && !fin_first) {
-                float* dst = p.partial + (size_t)sk32_slot(cta, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
+                float* dst = p.partial + (size_t)slot_of(rloc) * NT * 128;
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += 16) {
                     float v[16];
@@ -582,10 +600,9 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                             float pv[MAXB][CH];
 #pragma unroll
                             for (int bi = 0; bi < MAXB; ++bi) {
-                                const int pc = first + b0 + bi;
-                                if (b0 + bi < nc && pc != cta) {
-                                    const float* src =
-                                        p.partial + (size_t)sk32_slot(pc, (uint32_t)t, KB, (uint32_t)U, P) * NT * 128;
+                                const int pi = firsti + b0 + bi;
+                                if (b0 + bi < nc && pi != rloc) {
+                                    const float* src = p.partial + (size_t)slot_of(pi) * NT * 128;
 #pragma unroll
                                     for (int i = 0; i < CH; ++i) pv[bi][i] = __ldcg(src + (c0 + i) * 128 + row);
                                 }
@@ -593,7 +610,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
 #pragma unroll
                             for (int bi = 0; bi < MAXB; ++bi) {
                                 if (b0 + bi < nc) {
-                                    const bool own = first + b0 + bi == cta;
+                                    const bool own = firsti + b0 + bi == rloc;
 #pragma unroll
                                     for (int i = 0; i < CH; ++i) acc[i] += own ? v[i] : pv[bi][i];
                                 }
@@ -971,6 +988,19 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
     if (p.units == 0) return 0;
     p.cluster = 0;
     if (nt == 16 && auto_grid) pick_cluster(p, num_sms);
+    // Several token tiles: groups of m_tiles CTAs, one per token tile, when that keeps
+    // at least 90 % of the grid busy and every group has work (a unit; with whole
+    // tiles, a weight tile).
+    p.grouped = 0;
+    if (nt == 256 && auto_grid && p.cluster < 2 && p.m_tiles > 1) {
+        int G = p.ctas / p.m_tiles;
+        if (p.whole_tiles && G > p.n_tiles) G = p.n_tiles;
+        if (G >= 1 && (long long)G * p.m_tiles * 10 >= (long long)p.ctas * 9 &&
+            (long long)p.n_tiles * p.KB >= G) {
+            p.grouped = 1;
+            p.ctas = G * p.m_tiles;
+        }
+    }
     switch (nt) {
     case 16: return p.cluster >= 2 ? launch_nt<16, true>(p, stream) : launch_nt<16, false>(p, stream);
     case 32: return launch_nt<32, false>(p, stream);
