@@ -221,6 +221,16 @@ DF_DEV uint64_t make_l2_policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+DF_DEV uint64_t make_l2_policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+DF_DEV uint64_t make_l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 // ---------------------------------------------------------------------------
 // tcgen05 (TMEM allocation, MMA, commit, loads)
 // ---------------------------------------------------------------------------

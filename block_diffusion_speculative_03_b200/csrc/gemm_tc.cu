@@ -178,7 +178,12 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t pol_w = make_l2_policy_evict_first();
+            // Weights are read once: evict first.  In grouped mode the m_tiles CTAs of a
+            // group read each weight tile within a short time of each other, so it stays
+            // at normal priority until the last of them has it, and the token tiles, read
+            // by every group, are kept ahead of it.
+            const uint64_t pol_w = GM > 1 ? make_l2_policy_evict_normal() : make_l2_policy_evict_first();
+            const uint64_t pol_b = make_l2_policy_evict_last();
             // Weights never depend on the previous kernel: start streaming the
             // first S weight tiles into the ring, and the next l2_prefetch ones
             // into L2, before waiting for it to finish.
@@ -243,7 +248,10 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         }
                     }
                     const int bm = kb / p.kb_per_b;
-                    tma_load_2d(b, &p.tb[bm], &full[stage], (kb - bm * p.kb_per_b) * 64, m_tile * NT);
+                    if (GM > 1)   // every group reads all token tiles: keep them in L2 ahead of the weights
+                        tma_load_2d_hint(b, &p.tb[bm], &full[stage], (kb - bm * p.kb_per_b) * 64, m_tile * NT, pol_b);
+                    else
+                        tma_load_2d(b, &p.tb[bm], &full[stage], (kb - bm * p.kb_per_b) * 64, m_tile * NT);
                     ++issued;
                     if (++stage == S) { stage = 0; ++round; }
                 }
