@@ -90,7 +90,8 @@ def env_int(name, default):
 # outputs)), from one ncu capture of a single GEMM launch of the step's shape
 # class (M = 16 tokens, weights larger than L2).  It describes the kernel sources
 # it was taken on: once they change, the figure is void and the line reports null.
-GEMM_TRAFFIC = {"ratio": None, "sources_sha256": None}
+GEMM_TRAFFIC = {"ratio": 1.0041,
+                "sources_sha256": "0636b0903ee71329c1a34168e1d85dac1e4b140eae3e7974dc368dc22d772a2c"}
 
 
 def gemm_sources_sha256():
