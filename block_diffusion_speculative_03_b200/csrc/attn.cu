@@ -406,24 +406,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
         float lrow = l;
 #pragma unroll
         for (int k = 1; k < CS; ++k) lrow += xch[(rl + k * RW) & 127];
-        // the lane's O (its key slice's share of the row) into po[rl]
+        // the lane's O (its key slice's share of the row) into po[rl], 32 columns per
+        // tensor-memory load
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            float v[16];
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            float v[32];
             if (ok && ntiles >= 1) {
-                tmem_ld16w(tO + lanes + c0, v);
+                tmem_ld32w(tO + lanes + c0, v);
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
+            for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4*>(po + rl * PO_LD + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         }
         named_bar_sync(1, 128);
         // add the CS slices of each row into its first-window lane; the row's CS
-        // threads take D/CS columns each
-#pragma unroll 1
+        // threads take D/CS columns each (loads of several columns in flight at once)
+#pragma unroll 4
         for (int c = cs * (D / CS); c < (cs + 1) * (D / CS); c += 4) {
             float4 a = *reinterpret_cast<const float4*>(po + row * PO_LD + c);
 #pragma unroll
