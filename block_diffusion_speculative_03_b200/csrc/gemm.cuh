@@ -119,14 +119,6 @@ __host__ __device__ inline int sk_first_cta(long long tile, int KB, long long U,
 __host__ __device__ inline int sk_n_contrib(long long tile, int KB, long long U, int P) {
     return sk_owner((tile + 1) * KB - 1, U, P) - sk_owner(tile * KB, U, P) + 1;
 }
-// Partial slot of CTA p's segment of `tile`: a CTA has at most two split
-// segments, its first (slot 2p) and its last (slot 2p+1); every segment in
-// between covers a whole tile and needs no partial.
-__host__ __device__ inline int sk_slot(int p, long long tile, int KB, long long U, int P) {
-    long long first_tile = sk_begin(p, U, P) / KB;
-    return 2 * p + (tile == first_tile ? 0 : 1);
-}
-
 // Tokens per MMA tile for M rows.
 inline int pick_nt(int M) {
     if (M <= 16) return 16;
