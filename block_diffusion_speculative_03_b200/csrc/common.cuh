@@ -40,6 +40,9 @@ DF_DEV void mbar_init(uint64_t* bar, uint32_t count) {
 }
 DF_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 DF_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Global-memory data this thread has observed (generic proxy) becomes visible to
+// its subsequent bulk copies (async proxy).
+DF_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // Thread-block cluster barrier (every thread of every CTA of the cluster), and
 // distributed shared memory: the address of the same variable in CTA `rank` of
@@ -55,6 +58,14 @@ DF_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 DF_DEV void st_async_v4(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
                  ::"r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+                 : "memory");
+}
+
+// Untiled bulk copy from global memory into this CTA's shared memory (both
+// addresses 16-byte aligned, bytes a multiple of 16), completing `bytes` on bar.
+DF_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
 

@@ -526,6 +526,27 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             if (trace && e == 0) trace[4] = (long long)globaltimer_ns();
             tc_fence_after();
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * NT);
+            // Whole-grid finisher: the tile is its last segment, so once its accumulator
+            // is ready its ring is idle (every stage consumed, no load in flight): the
+            // peers' partials land there in one round trip of bulk copies instead of
+            // rounds of register loads.
+            const bool land_ring =
+                NT <= 32 && fin_first && !CL && nc > 1 && (nc - 1) * NT * 512 <= S * C::A_BYTES;
+            if (land_ring) {
+                if (e == 0) {
+                    fence_proxy_async_global();   // the partials seen through the count's acquire
+                    mbar_arrive_expect_tx(landb, (uint32_t)((nc - 1) * NT * 512));
+                    for (int b = 1; b < nc; ++b)
+                        bulk_load(sA + (size_t)(b - 1) * NT * 512, p.partial + (size_t)slot_of(firsti + b) * NT * 128,
+                                  (uint32_t)(NT * 512), landb);
+                }
+                const bool lok = mbar_wait(landb, 0, abort_flag, p.status);
+                if (!lok && e == 0) {
+                    volatile int never = 0;   // let the copies land before the CTA can leave
+                    mbar_wait(landb, 0, &never, nullptr);
+                }
+                if (named_bar_or(1, 128, !lok)) break;
+            }
             bool finish = true;
             if (!whole && !fin_first && CL) {
                 // Send the partial (all NT columns of this thread's row) into the
@@ -596,6 +617,19 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                                 acc[i + 2] += w.z;
                                 acc[i + 3] += w.w;
                             }
+                        }
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) v[i] = acc[i];
+                    } else if (!whole && land_ring) {
+                        // this CTA first (it is the first contributor), then the landed
+                        // partials in contributor order
+                        float acc[CH];
+#pragma unroll
+                        for (int i = 0; i < CH; ++i) acc[i] = 0.0f + v[i];
+                        for (int b = 1; b < nc; ++b) {
+                            const float* src = reinterpret_cast<const float*>(sA) + (size_t)(b - 1) * NT * 128;
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) acc[i] += src[(c0 + i) * 128 + row];
                         }
 #pragma unroll
                         for (int i = 0; i < CH; ++i) v[i] = acc[i];
