@@ -32,6 +32,7 @@ static bool g_inject_whole = true;
 static bool g_fold_head = false;
 // O-projection on the SMs the attention does not hold (see layers_bf16).
 static bool g_o_beside_attention = false;
+static int g_o_late_deficit = 9;   // units fewer for the O-projection CTAs that start after the attention (measured: 0, 3, 9)
 constexpr int kFoldMaxNT = 16;
 void set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
@@ -905,12 +906,16 @@ static int layers_bf16(dflash_handle* h, dflash_cache* cc, int gamma, bool inges
                 p.ssq_ld = ssq_ld;
             }
             Timed t(h, TK_GEMM_O, st);
-            // The attention holds attn_blocks SMs until it ends; O-projection CTAs
-            // placed there would start a whole attention later than the rest and
-            // finish last.  Run the O-projection on the other SMs only, and let those
-            // CTAs, idle until the attention is done, prefetch their whole weight
-            // range into L2 (the attention leaves HBM nearly idle).
+            // The attention holds attn_blocks SMs until it ends: the O-projection's
+            // CTAs that land there (the highest block indices: CTAs are dispatched in
+            // order) start when it ends, without the weight stages the others loaded
+            // during it, so they take g_o_late_deficit fewer k-block units.  (Optional:
+            // run the O-projection on the other SMs only, prefetching into L2.)
             const bool beside = g_o_beside_attention && attn_blocks * 4 <= h->num_sms * 3;
+            if (!beside && attn_blocks < h->num_sms) {
+                p.late_from = h->num_sms - attn_blocks;
+                p.late_deficit = g_o_late_deficit;
+            }
             int r = beside ? run_gemm(h, p, nt, st, TK_GEMM_O, h->num_sms - attn_blocks, 64)
                            : run_gemm(h, p, nt, st, TK_GEMM_O);
             if (r) return r;
@@ -1377,6 +1382,12 @@ int dflash_diag_gemm_max_active_clusters(int cluster_size) {
 
 int dflash_diag_set_split_finisher(int last_arriver) {
     set_gemm_last_arriver(last_arriver);
+    return DFLASH_OK;
+}
+
+int dflash_diag_set_o_late_deficit(int units) {
+    if (units < 0 || units > 64) return DFLASH_INVALID_ARG;
+    g_o_late_deficit = units;
     return DFLASH_OK;
 }
 

@@ -52,6 +52,9 @@ struct GemmParams {
                                  //    in-order accumulation over all of K, whatever M and the grid
     int l2_prefetch;             // weight tiles past the shared-memory ring prefetched into L2 before the wait
     int pre_stages;              // ring stages filled with weights before the wait (0: the whole ring)
+    int late_from, late_deficit; // whole-grid partition: CTAs [late_from, ctas) start late (their SMs
+                                 //    are held by the previous kernel) and take late_deficit fewer
+                                 //    k-block units each (0: equal shares)
     int grouped;                 // 1: CTAs in groups of m_tiles, one per token tile, splitting the
                                  //    (weight tile, k-block) units between groups (set by the launcher)
     int cluster;                 // >= 2: CTAs in thread-block clusters of this size, each cluster owning

@@ -53,6 +53,22 @@ DF_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
 DF_DEV uint32_t sk32_begin(uint32_t p, uint32_t U, uint32_t P) { return p * U / P; }
 DF_DEV uint32_t sk32_owner(uint32_t u, uint32_t U, uint32_t P) { return ((u + 1) * P - 1) / U; }
 
+// Weighted whole-grid partition: CTAs [L, P) take d units fewer than CTAs [0, L).
+// With E = U + (P - L) d, begin(p) = floor((p E - max(0, p - L) d P) / P), so the
+// early CTAs own E / P units each and the late ones (U - L d) / P; the launcher
+// keeps U - L d >= P and P E < 2^32.  owner(u) is the largest p with begin(p) <= u.
+DF_DEV uint32_t skw32_begin(uint32_t p, uint32_t U, uint32_t P, uint32_t L, uint32_t d) {
+    const uint32_t E = U + (P - L) * d;
+    return (p * E - (p > L ? p - L : 0u) * d * P) / P;
+}
+DF_DEV uint32_t skw32_owner(uint32_t u, uint32_t U, uint32_t P, uint32_t L, uint32_t d) {
+    const uint32_t E = U + (P - L) * d;
+    const uint32_t pe = ((u + 1) * P - 1) / E;
+    if (pe < L) return pe;
+    const uint32_t pl = ((u + 1) * P - L * d * P - 1) / (U - L * d);
+    return pl < P - 1 ? pl : P - 1;
+}
+
 // Top-2 merge: a <- top2(a ∪ b); ties of the top value go to the lower id.
 DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2) {
     if (b1 > a1 || (b1 == a1 && bi < ai)) {
@@ -130,7 +146,14 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             cbase = q * CL;
         }
     }
+    // weighted shares (whole grid only)
+    const bool WT = p.late_deficit > 0 && GM == 1 && !CL && !p.whole_tiles;
+    const uint32_t wL = (uint32_t)p.late_from, wd = (uint32_t)p.late_deficit;
     long long u_begin = ubase + sk_begin(rloc, Uloc, Ploc), u_end = ubase + sk_begin(rloc + 1, Uloc, Ploc);
+    if (WT) {
+        u_begin = skw32_begin((uint32_t)cta, (uint32_t)U, (uint32_t)P, wL, wd);
+        u_end = skw32_begin((uint32_t)cta + 1, (uint32_t)U, (uint32_t)P, wL, wd);
+    }
     if (p.whole_tiles && !CL) {   // tile-granular ranges: no tile is split, no partials
         const long long T = Uloc / KB;
         u_begin = (T * rloc / Ploc) * KB;
@@ -502,16 +525,22 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             if (!whole) {
                 const uint32_t t32 = (uint32_t)(tn * KB - ubase), K32 = (uint32_t)KB, U32 = (uint32_t)Uloc,
                                P32 = (uint32_t)Ploc;
-                firsti = (int)sk32_owner(t32, U32, P32);
-                nc = (int)sk32_owner(t32 + K32 - 1, U32, P32) - firsti + 1;
+                if (WT) {
+                    firsti = (int)skw32_owner(t32, U32, P32, wL, wd);
+                    nc = (int)skw32_owner(t32 + K32 - 1, U32, P32, wL, wd) - firsti + 1;
+                } else {
+                    firsti = (int)sk32_owner(t32, U32, P32);
+                    nc = (int)sk32_owner(t32 + K32 - 1, U32, P32) - firsti + 1;
+                }
                 first = cta_of(firsti);
             }
             // partial slot of the CTA with partition index i for this tile: its first
             // segment (slot 2 * CTA) or its last (2 * CTA + 1)
             // (32-bit arithmetic: the launcher keeps every unit index below 2^32)
             auto slot_of = [&](int i) -> int {
-                const uint32_t first_tn =
-                    ((uint32_t)ubase + sk32_begin((uint32_t)i, (uint32_t)Uloc, (uint32_t)Ploc)) / (uint32_t)KB;
+                const uint32_t b0 = WT ? skw32_begin((uint32_t)i, (uint32_t)Uloc, (uint32_t)Ploc, wL, wd)
+                                       : sk32_begin((uint32_t)i, (uint32_t)Uloc, (uint32_t)Ploc);
+                const uint32_t first_tn = ((uint32_t)ubase + b0) / (uint32_t)KB;
                 return 2 * cta_of(i) + (first_tn == (uint32_t)tn ? 0 : 1);
             };
             bool ok = true;
@@ -1030,6 +1059,14 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
     if (p.units == 0) return 0;
     p.cluster = 0;
     if (nt == 16 && auto_grid) pick_cluster(p, num_sms);
+    // Weighted shares only on the whole grid, when every late CTA keeps a unit and the
+    // 32-bit partition arithmetic holds.
+    if (p.late_deficit > 0) {
+        const long long L = p.late_from, d = p.late_deficit, P = p.ctas;
+        const long long E = p.units + (P - L) * d;
+        if (p.whole_tiles || p.cluster >= 2 || L <= 0 || L >= P || p.units - L * d < P || P * E >= (1LL << 32))
+            p.late_deficit = 0;
+    }
     // Several token tiles: groups of m_tiles CTAs, one per token tile, when that keeps
     // at least 90 % of the grid busy and every group has work (a unit; with whole
     // tiles, a weight tile).
@@ -1041,6 +1078,7 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
             (long long)p.n_tiles * p.KB >= G) {
             p.grouped = 1;
             p.ctas = G * p.m_tiles;
+            p.late_deficit = 0;
         }
     }
     switch (nt) {
