@@ -72,7 +72,7 @@ def parse_args():
     ap.add_argument("--gemm-cluster", type=int, default=None,
                     help="largest thread-block cluster for 16-token GEMMs (0 = whole-grid split-K only, the library default)")
     ap.add_argument("--o-late-deficit", type=int, default=None,
-                    help="k-block units fewer for O-projection CTAs that start after the attention (library default 6)")
+                    help="k-block units fewer for O-projection CTAs that start after the attention (library default 9)")
     ap.add_argument("--last-arriver", action="store_true",
                     help="split GEMM tiles finished by the contributor that counts in last (default: by the first)")
     ap.add_argument("--l2-prefetch", type=int, default=None,
@@ -747,7 +747,7 @@ def run_gpu(args):
                              "split_tile_finisher": "last arriver" if args.last_arriver else "first contributor",
                              "gemm_pre_stages": args.pre_stages if args.pre_stages is not None else "library default (6)",
                              "gemm_max_cluster": args.gemm_cluster if args.gemm_cluster is not None else "library default (0)",
-                             "o_late_deficit": args.o_late_deficit if args.o_late_deficit is not None else "library default (6)",
+                             "o_late_deficit": args.o_late_deficit if args.o_late_deficit is not None else "library default (9)",
                              "gemm_resident_clusters": {str(c): D.dflash_diag_gemm_max_active_clusters(c) for c in (2, 3, 4)}},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
                                                                               else ", programmatic dependent launch"),

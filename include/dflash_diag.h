@@ -228,7 +228,7 @@ int dflash_diag_gemm_max_active_clusters(int cluster_size);
  * partials in the same order, so the results are bit-identical. */
 int dflash_diag_set_split_finisher(int last_arriver);
 
-/* k-block units (0..64, default 6) fewer for each O-projection CTA that lands on
+/* k-block units (0..64, default 9) fewer for each O-projection CTA that lands on
  * an SM the attention still holds (process-wide; applies to calls enqueued
  * afterwards).  Those CTAs start when the attention ends, without the weight
  * stages the others loaded during it; 0 gives every CTA an equal share. */
