@@ -73,6 +73,9 @@ def parse_args():
                     help="largest thread-block cluster for 16-token GEMMs (0 = whole-grid split-K only, the library default)")
     ap.add_argument("--o-late-deficit", type=int, default=None,
                     help="k-block units fewer for O-projection CTAs that start after the attention (library default 9)")
+    ap.add_argument("--gemm-tail", type=int, nargs=2, default=None, metavar=("CTAS", "UNITS"),
+                    help="the last CTAS CTAs of the other whole-grid GEMMs take UNITS fewer k-block units "
+                         "(library default 24 3)")
     ap.add_argument("--last-arriver", action="store_true",
                     help="split GEMM tiles finished by the contributor that counts in last (default: by the first)")
     ap.add_argument("--l2-prefetch", type=int, default=None,
@@ -485,6 +488,8 @@ def run_gpu(args):
     D.dflash_diag_set_split_finisher(args.last_arriver)
     if args.o_late_deficit is not None:
         D.dflash_diag_set_o_late_deficit(args.o_late_deficit)
+    if args.gemm_tail is not None:
+        D.dflash_diag_set_gemm_tail(*args.gemm_tail)
     if args.gemm_cluster is not None:
         D.dflash_diag_set_gemm_max_cluster(args.gemm_cluster)
     pre_ms = []
@@ -748,6 +753,7 @@ def run_gpu(args):
                              "gemm_pre_stages": args.pre_stages if args.pre_stages is not None else "library default (6)",
                              "gemm_max_cluster": args.gemm_cluster if args.gemm_cluster is not None else "library default (0)",
                              "o_late_deficit": args.o_late_deficit if args.o_late_deficit is not None else "library default (9)",
+                             "gemm_tail": args.gemm_tail if args.gemm_tail is not None else "library default (24, 3)",
                              "gemm_resident_clusters": {str(c): D.dflash_diag_gemm_max_active_clusters(c) for c in (2, 3, 4)}},
             "launch_mode": ("eager" if args.eager else "cuda-graph replay") + (", plain launches" if args.no_pdl
                                                                               else ", programmatic dependent launch"),

@@ -312,8 +312,20 @@ void gemm_common(dflash_handle* h, GemmParams& p) {
     p.ctas = 0;
 }
 
+// The last CTAs of a launch land on the SMs the previous kernel's last CTAs held and
+// start after them: the last g_tail_ctas CTAs of the step's other whole-grid GEMMs
+// take g_tail_deficit fewer k-block units.  The shift also moves the split points
+// of every tile, and that dominates: 24 CTAs x 3 units measured best on the
+// Qwen3-8B-shaped drafter (neighbouring settings were slower, and the
+// Qwen3-4B-shaped one is slower with it).
+static int g_tail_ctas = 24, g_tail_deficit = 3;
+
 int run_gemm(dflash_handle* h, GemmParams& p, int nt, cudaStream_t st, int kind, int ctas = 0, int l2_prefetch = -1) {
     gemm_common(h, p);
+    if (p.late_deficit == 0 && g_tail_ctas > 0 && g_tail_deficit > 0 && ctas == 0 && kind != TK_SIMT_F32) {
+        p.late_from = std::min(h->num_sms, kMaxCtas) - g_tail_ctas;
+        p.late_deficit = g_tail_deficit;
+    }
     if (ctas > 0) p.ctas = ctas;
     if (l2_prefetch >= 0) p.l2_prefetch = l2_prefetch;
     // GEMM trace: 8 stamps per CTA (gemm.cuh), past the wait at 1, exit at 6;
@@ -1382,6 +1394,13 @@ int dflash_diag_gemm_max_active_clusters(int cluster_size) {
 
 int dflash_diag_set_split_finisher(int last_arriver) {
     set_gemm_last_arriver(last_arriver);
+    return DFLASH_OK;
+}
+
+int dflash_diag_set_gemm_tail(int ctas, int units) {
+    if (ctas < 0 || ctas > 64 || units < 0 || units > 64) return DFLASH_INVALID_ARG;
+    g_tail_ctas = ctas;
+    g_tail_deficit = units;
     return DFLASH_OK;
 }
 

@@ -111,6 +111,7 @@ def lib():
         "dflash_diag_set_split_finisher": (i32, [i32]),
         "dflash_diag_set_gemm_max_cluster": (i32, [i32]),
         "dflash_diag_set_o_late_deficit": (i32, [i32]),
+        "dflash_diag_set_gemm_tail": (i32, [i32, i32]),
         "dflash_diag_gemm_max_active_clusters": (i32, [i32]),
         "dflash_diag_set_norm_fold": (i32, [i32]),
         "dflash_diag_set_inject_partition": (i32, [i32]),
@@ -150,7 +151,7 @@ def exported_symbols() -> list:
             "dflash_diag_timing_enable", "dflash_diag_timing_read", "dflash_diag_timing_disable",
             "dflash_diag_timed_name", "dflash_diag_set_launch_mode", "dflash_diag_set_gemm_prefetch", "dflash_diag_gemm_prefetch",
             "dflash_diag_set_gemm_pre_stages", "dflash_diag_set_split_finisher", "dflash_diag_set_gemm_max_cluster",
-            "dflash_diag_set_o_late_deficit",
+            "dflash_diag_set_o_late_deficit", "dflash_diag_set_gemm_tail",
             "dflash_diag_gemm_max_active_clusters",
             "dflash_diag_set_norm_fold", "dflash_diag_set_inject_partition",
             "dflash_diag_set_o_beside_attention",
@@ -379,6 +380,10 @@ def dflash_diag_gemm_max_active_clusters(cluster_size: int) -> int:
 
 def dflash_diag_set_o_late_deficit(units: int) -> int:
     return _chk(lib().dflash_diag_set_o_late_deficit(int(units)), "dflash_diag_set_o_late_deficit")
+
+
+def dflash_diag_set_gemm_tail(ctas: int, units: int) -> int:
+    return _chk(lib().dflash_diag_set_gemm_tail(int(ctas), int(units)), "dflash_diag_set_gemm_tail")
 
 
 def dflash_diag_gemm_prefetch() -> int:

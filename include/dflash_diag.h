@@ -228,6 +228,13 @@ int dflash_diag_gemm_max_active_clusters(int cluster_size);
  * partials in the same order, so the results are bit-identical. */
 int dflash_diag_set_split_finisher(int last_arriver);
 
+/* The last `ctas` CTAs (0..64) of the draft step's other whole-grid GEMMs take
+ * `units` (0..64) fewer k-block units each (process-wide; default 24, 3; 0, 0 for
+ * equal shares).  They land on the SMs the previous kernel's last CTAs held and
+ * start after them; the shift also moves every tile's split points, which is the
+ * larger effect and depends on the shapes. */
+int dflash_diag_set_gemm_tail(int ctas, int units);
+
 /* k-block units (0..64, default 9) fewer for each O-projection CTA that lands on
  * an SM the attention still holds (process-wide; applies to calls enqueued
  * afterwards).  Those CTAs start when the attention ends, without the weight
