@@ -133,18 +133,43 @@ __global__ void k_ingest_end(const int* __restrict__ row_count, int rows, int B,
 template <typename T>
 __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* __restrict__ y, int H, float eps,
                           int grp, int gstride, int goff, long long* tr) {
-    griddep_wait();
-    griddep_launch();
-    trace_mark(tr, 0);
     constexpr int VEC = 16 / sizeof(T);          // elements per 16-byte access
+    constexpr int KEEP = 4;                      // vectors of x and g a thread keeps in registers
     const int o = blockIdx.x;
     const int in = (o / grp) * gstride + goff + o % grp;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)in * H);
     const uint4* gr = reinterpret_cast<const uint4*>(g);
     uint4* yr = reinterpret_cast<uint4*>(y + (size_t)o * H);
     const int nv = H / VEC;
+    // the gain is a weight: fetch it before waiting for the kernel that writes x
+    uint4 gk[KEEP], xk[KEEP];
+#pragma unroll
+    for (int j = 0; j < KEEP; ++j) {
+        const int i = threadIdx.x + j * blockDim.x;
+        if (i < nv) gk[j] = gr[i];
+    }
+    griddep_wait();
+    griddep_launch();
+    trace_mark(tr, 0);
     float ss = 0.f;
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+#pragma unroll
+    for (int j = 0; j < KEEP; ++j) {
+        const int i = threadIdx.x + j * blockDim.x;
+        if (i < nv) xk[j] = xr[i];
+    }
+#pragma unroll
+    for (int j = 0; j < KEEP; ++j) {
+        const int i = threadIdx.x + j * blockDim.x;
+        if (i < nv) {
+            const T* e = reinterpret_cast<const T*>(&xk[j]);
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) {
+                const float v = ldf(e + k);
+                ss += v * v;
+            }
+        }
+    }
+    for (int i = threadIdx.x + KEEP * blockDim.x; i < nv; i += blockDim.x) {   // rows wider than the kept part
         const uint4 u = xr[i];
         const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
@@ -164,8 +189,7 @@ __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* _
     }
     __syncthreads();
     const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-        const uint4 u = xr[i], gu = gr[i];
+    auto norm_store = [&](int i, const uint4& u, const uint4& gu) {
         const T* e = reinterpret_cast<const T*>(&u);
         const T* ge = reinterpret_cast<const T*>(&gu);
         uint4 out;
@@ -173,7 +197,13 @@ __global__ void k_rmsnorm(const T* __restrict__ x, const T* __restrict__ g, T* _
 #pragma unroll
         for (int k = 0; k < VEC; ++k) stf(oe + k, ldf(e + k) * inv * ldf(ge + k));
         yr[i] = out;
+    };
+#pragma unroll
+    for (int j = 0; j < KEEP; ++j) {
+        const int i = threadIdx.x + j * blockDim.x;
+        if (i < nv) norm_store(i, xk[j], gk[j]);
     }
+    for (int i = threadIdx.x + KEEP * blockDim.x; i < nv; i += blockDim.x) norm_store(i, xr[i], gr[i]);
     trace_mark(tr, 1);
 }
 
