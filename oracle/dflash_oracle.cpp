@@ -470,11 +470,22 @@ void oracle_layer_oproj(const oracle_config* c, const oracle_weights* w, int l, 
 
 // a6, second half: m = R(silu(h2 . Wg^T) * (h2 . Wu^T)) for the normalised rows
 // h2 [gamma][H] (m [gamma][I] optional), then x_out = R(x + m . Wd^T).
+// The down-projection and residual add of layer l from the SwiGLU output m
+// [gamma][intermediate]: x_out = R(x + m . Wd^T).
+void oracle_layer_down(const oracle_config* c, const oracle_weights* w, int l, const double* m, const double* x,
+                       int gamma, double* x_out) {
+    g_acc32 = c->acc32;
+    int S = c->storage, H = c->hidden, I = c->intermediate;
+    std::vector<double> y((size_t)gamma * H);
+    linear(m, gamma, I, w->w_down[l], H, S, y.data());
+    for (size_t i = 0; i < y.size(); ++i) x_out[i] = R(x[i] + y[i], S);
+}
+
 void oracle_layer_mlp(const oracle_config* c, const oracle_weights* w, int l, const double* h2, const double* x,
                       int gamma, double* m_out, double* x_out) {
     g_acc32 = c->acc32;
     int S = c->storage, H = c->hidden, I = c->intermediate;
-    std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I), y((size_t)gamma * H);
+    std::vector<double> gt((size_t)gamma * I), up((size_t)gamma * I), mm((size_t)gamma * I);
     linear(h2, gamma, H, w->w_gate[l], I, S, gt.data());
     linear(h2, gamma, H, w->w_up[l], I, S, up.data());
     for (size_t i = 0; i < mm.size(); ++i) {
@@ -483,8 +494,7 @@ void oracle_layer_mlp(const oracle_config* c, const oracle_weights* w, int l, co
         mm[i] = R(silu * up[i], S);
     }
     if (m_out) std::memcpy(m_out, mm.data(), sizeof(double) * mm.size());
-    linear(mm.data(), gamma, I, w->w_down[l], H, S, y.data());
-    for (size_t i = 0; i < y.size(); ++i) x_out[i] = R(x[i] + y[i], S);
+    oracle_layer_down(c, w, l, mm.data(), x, gamma, x_out);
 }
 
 // ---------------------------------------------------------------------------

@@ -66,6 +66,7 @@ def lib():
                                              C.c_int, dp]
         L.oracle_layer_oproj.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, dp]
         L.oracle_layer_mlp.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, dp, dp]
+        L.oracle_layer_down.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, dp, dp, C.c_int, dp]
         L.oracle_embed_block.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), C.c_int, C.c_int, dp]
         L.oracle_final_norm.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, dp]
         L.oracle_lm_head.argtypes = [C.POINTER(_Cfg), C.POINTER(_W), dp, C.c_int, ip, dp, dp]
@@ -312,6 +313,14 @@ class OracleDrafter:
         lib().oracle_layer_mlp(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(h2), _dp(x), x.shape[0], _dp(m),
                                _dp(out))
         return m, out
+
+    def layer_down(self, layer: int, m: np.ndarray, x: np.ndarray) -> np.ndarray:
+        """x_out [rows, hidden] = R(x + m . Wd^T) from the SwiGLU output m [rows, intermediate]."""
+        m = np.ascontiguousarray(m, dtype=np.float64)
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty_like(x)
+        lib().oracle_layer_down(C.byref(self.cfg), C.byref(self.w), int(layer), _dp(m), _dp(x), x.shape[0], _dp(out))
+        return out
 
     def final_norm(self, x: np.ndarray) -> np.ndarray:
         """hf rows of the mask positions 1..gamma-1 of x [gamma, hidden]."""

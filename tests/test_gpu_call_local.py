@@ -159,7 +159,10 @@ class Rig:
                 check_state(st["h2"][l], od.norm_rows("g_post", l, st["x_mid"][l]), "h2" + tag)
                 m_o, x_o = od.layer_mlp(l, st["h2"][l], st["x_mid"][l])
                 check_state(st["act"][l], m_o, "act" + tag)
-                check_state(xs[l + 1], x_o, "x" + tag)
+                check_state(xs[l + 1], od.layer_down(l, st["act"][l], st["x_mid"][l]), "x" + tag)
+                # the MLP from h2 runs two GEMMs through a bf16 intermediate: its flips
+                # carry into the down-projection, so only the error bound is held here
+                check_state(xs[l + 1], x_o, "mlp" + tag, min_same=0.0)
                 # the whole layer from its input: bf16 flips inside the layer cascade
                 # through the MLP (fp64 vs fp32 accumulation alone leaves ~70 % of the
                 # outputs identical), so only the error bound is held here

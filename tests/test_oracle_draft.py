@@ -308,7 +308,7 @@ def test_piecewise_draft_equals_one_call(dtype):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_layer_stages_compose_to_the_layer(dtype):
-    # norm -> qkv -> attention -> O-proj -> norm -> MLP, one stage at a time (the form
+    # norm -> qkv -> attention -> O-proj -> norm -> MLP (= SwiGLU, then down), one stage at a time (the form
     # the per-stage GPU parity tests feed the GPU's own inputs to), equals one layer call
     w = micro(dtype)
     W = I.make_weights(w)
@@ -321,5 +321,6 @@ def test_layer_stages_compose_to_the_layer(dtype):
         o = od.layer_attention(cache, l, q, k, v)
         xm = od.layer_oproj(l, o, x)
         m, x2 = od.layer_mlp(l, od.norm_rows("g_post", l, xm), xm)
+        assert np.array_equal(x2, od.layer_down(l, m, xm))
         assert np.array_equal(x2, od.draft_layer(cache, l, x))
         x = x2
