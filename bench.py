@@ -283,6 +283,46 @@ def step_algorithmic_bytes(w, B, gamma, ctx_len, conditioning="kv-injection"):
     return draft + ab["gemm_inject"]
 
 
+def algorithmic_flops(w, B, gamma, ctx_len):
+    """Multiply-add FLOPs of one launch of each kernel kind (the same kinds as
+    algorithmic_bytes)."""
+    H, d = w.hidden, w.head_dim
+    Nq, Nkv, I, V = w.n_q_heads * d, w.n_kv_heads * d, w.intermediate, w.vocab
+    M, Mlm = B * gamma, B * (gamma - 1)
+    return {
+        "gemm_qkv": 2 * M * H * (Nq + 2 * Nkv),
+        "gemm_o": 2 * M * Nq * H,
+        "gemm_swiglu": 2 * M * H * 2 * I,
+        "gemm_down": 2 * M * I * H,
+        "gemm_lmhead": 2 * Mlm * H * V,
+        "gemm_fuse": 2 * M * w.n_sel * w.target_hidden * H,
+        "gemm_inject": 2 * M * H * w.n_layers * 2 * Nkv,
+        "attention": 4 * B * w.n_q_heads * gamma * (ctx_len + gamma) * d,
+        "rmsnorm": 0,
+    }
+
+
+def step_launch_counts(w, conditioning="kv-injection"):
+    """Launches of each kernel kind in one step (those algorithmic_bytes counts)."""
+    L = w.n_layers
+    n = {"gemm_qkv": L, "gemm_o": L, "gemm_swiglu": L, "gemm_down": L, "attention": L,
+         "gemm_lmhead": 1, "gemm_fuse": 1, "gemm_inject": 1}
+    if conditioning == "input-fusion":
+        n["gemm_inject"] = 0
+        n["gemm_qkv"] += L
+        for k in ("gemm_o", "gemm_swiglu", "gemm_down", "attention"):
+            n[k] += L - 1
+    return n
+
+
+def kernelwise_roof_ms(w, B, gamma, ctx_len, conditioning, hbm_gbs, tflops):
+    """Sum over the step's launches of max(bytes at the HBM peak, FLOPs at the tensor
+    peak): a launch cannot beat its own slower bound."""
+    ab, af = algorithmic_bytes(w, B, gamma, ctx_len), algorithmic_flops(w, B, gamma, ctx_len)
+    return sum(c * max(ab[k] / (hbm_gbs * 1e9), af[k] / (tflops * 1e12))
+               for k, c in step_launch_counts(w, conditioning).items()) * 1e3
+
+
 def step_flops(w, B, gamma, ctx_len):
     H, d = w.hidden, w.head_dim
     Nq, Nkv, I, V = w.n_q_heads * d, w.n_kv_heads * d, w.intermediate, w.vocab
@@ -608,6 +648,8 @@ def run_gpu(args):
     ab = algorithmic_bytes(w, B, g, T)
     step_bytes = step_algorithmic_bytes(w, B, g, T, args.conditioning)
     t_roof_ms = step_bytes / (hbm_peak * 1e9) * 1e3
+    t_flops_ms = step_flops(w, B, g, T) / (tc_peak * 1e12) * 1e3
+    t_kw_ms = kernelwise_roof_ms(w, B, g, T, args.conditioning, hbm_peak, tc_peak)
 
     # ---- traced pass: the same step captured in one CUDA graph with the library's
     # step trace on (every kernel stamps %globaltimer per block past its dependency
@@ -733,7 +775,13 @@ def run_gpu(args):
             "roofline": roofline,
             "step_roofline": {"algorithmic_bytes": step_bytes, "flops": step_flops(w, B, g, T),
                               "t_roof_ms": round(t_roof_ms, 4), "frac": round(t_roof_ms / ms_step, 4),
-                              "peak_gbs": hbm_peak, "peak_source": peak_src},
+                              "peak_gbs": hbm_peak, "peak_source": peak_src,
+                              # the mixed bound: the step cannot beat its bytes at the HBM peak
+                              # nor its FLOPs at the (sustained) bf16 tensor peak
+                              "t_flops_ms": round(t_flops_ms, 4), "peak_tflops": tc_peak,
+                              "t_roof_mixed_ms": round(max(t_roof_ms, t_flops_ms), 4),
+                              "frac_mixed": round(max(t_roof_ms, t_flops_ms) / ms_step, 4),
+                              "t_roof_kernelwise_ms": round(t_kw_ms, 4), "frac_kernelwise": round(t_kw_ms / ms_step, 4)},
             "per_kernel": per_kernel,
             "traced_step": ({"ms_per_step": round(traced["traced_ms_per_step"], 4),
                              "traced_launches": traced["launches"],

@@ -60,3 +60,25 @@ def test_trace_attribution_partitions_the_traced_span():
     assert [(o[1], o[2]) for o in out] == [(100, 400), (300, 2100), (2050, 2700), (2400, 3600)]
     assert [o[3] for o in out] == [300, 1700, 600, 900]
     assert sum(o[3] for o in out) == 3600 - 100
+
+
+def test_step_flops_and_kernelwise_roofline_are_consistent():
+    """The per-kind FLOPs times the step's launch counts add up to the step's FLOPs
+    (both conditionings' draft parts), and the kernel-wise bound (each launch at its
+    slower of bytes and FLOPs) is at least the step's byte bound and its FLOP bound."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_diffusion_speculative_03_b200 import inputs as I
+    for name in ("qwen3_8b", "llama31_8b", "long_ctx", "tiny"):
+        w = I.preset(name)
+        B, g, T = w.batch, w.gamma, w.context[0]
+        af = bench.algorithmic_flops(w, B, g, T)
+        n = bench.step_launch_counts(w)
+        assert sum(af[k] * c for k, c in n.items()) == bench.step_flops(w, B, g, T)
+        ab = bench.algorithmic_bytes(w, B, g, T)
+        assert sum(ab[k] * c for k, c in n.items()) == bench.step_algorithmic_bytes(w, B, g, T)
+        bw, tf = 6541.0, 1385.0
+        kw = bench.kernelwise_roof_ms(w, B, g, T, "kv-injection", bw, tf)
+        t_bytes = bench.step_algorithmic_bytes(w, B, g, T) / (bw * 1e9) * 1e3
+        t_flops = bench.step_flops(w, B, g, T) / (tf * 1e12) * 1e3
+        assert kw >= max(t_bytes, t_flops) * (1 - 1e-12)
