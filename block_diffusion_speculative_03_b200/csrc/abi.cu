@@ -76,6 +76,22 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t r
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// 2-D bf16 tensor map of row-major rows (no swizzle): `inner` elements per row, `rows`
+// rows of `stride` elements, box {box_inner, box_rows}, zero fill out of bounds.
+bool encode_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                      uint32_t box_inner, uint32_t box_rows) {
+    PFN_encodeTiled_t enc = get_encode();
+    if (!enc || rows == 0 || inner == 0) return false;
+    if (((uintptr_t)base & 15) || ((stride * 2) & 15) || ((box_inner * 2) & 15)) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {stride * 2};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 }  // namespace df
 
 namespace {

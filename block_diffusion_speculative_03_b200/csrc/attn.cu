@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_tc(const __grid_consta
     constexpr int KC = 64 / CS;    // keys of a tile per softmax thread
     constexpr int PO_LD = C::PO_LD;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* smem = smem_align_up<uint8_t>(smem_raw, 1024);
     uint8_t* sK = smem;                            // [S][KV_BYTES]
     uint8_t* sV = sK + S * C::KV_BYTES;            // [S][KV_BYTES]
     uint64_t* bars = (uint64_t*)(smem + C::RING);

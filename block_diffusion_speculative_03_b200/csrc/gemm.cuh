@@ -40,6 +40,9 @@ struct GemmAMat {
 struct GemmParams {
     CUtensorMap ta[kMaxAMats];   // weight maps, box {64, 128} (SwiGLU: {64, 64})
     CUtensorMap tb[kMaxBMaps];   // activation maps, box {64, NT}
+    CUtensorMap tx;              // EPI_RESID, NT >= 64: the residual rows out[M][ldo], box {128, 32}, no
+                                 //    swizzle (set by the launcher; has_tx says whether it is valid)
+    int has_tx;
     GemmAMat amat[kMaxAMats];
     int n_amat;
     int swiglu;                  // A = rows [64t, 64t+64) of ta[0] then of ta[1]
@@ -130,6 +133,11 @@ inline int pick_nt(int M) {
     if (M <= 128) return 128;
     return 256;
 }
+
+// Row-major bf16 tensor map without swizzle (box {box_inner, box_rows}); false when the
+// driver's encoder is unavailable or the layout is not 16-byte aligned.
+bool encode_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                      uint32_t box_inner, uint32_t box_rows);
 
 // Weight tiles each CTA prefetches into L2 (beyond its shared-memory ring)
 // before its dependency wait; process-wide, set by dflash_diag_set_gemm_prefetch.

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     constexpr int S = C::STAGES;
     constexpr int CH = C::CH;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* smem = smem_align_up<uint8_t>(smem_raw, 1024);
     uint8_t* sA = smem;
     uint8_t* sB = smem + S * C::A_BYTES;
     float* xch = (float*)(sB + S * C::B_BYTES);
@@ -99,17 +99,20 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     uint64_t* acce = accf + 2;
     uint64_t* drain = acce + 2;
     uint64_t* landb = drain + 1;      // cluster mode: the peers' partials have landed
-    uint32_t* tmem_slot = (uint32_t*)(landb + 1);
+    uint64_t* landc = landb + 1;      // [3] chunked landing of the peers' partials (NT >= 64)
+    uint32_t* tmem_slot = (uint32_t*)(landc + 3);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* s_flag = (int*)(tmem_slot + 2);
     int* tok_b = s_flag + 1;          // [NT]
     int* tok_pos = tok_b + NT;        // [NT]
     float* inv_s = (float*)(tok_pos + NT);   // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
-    uint64_t* ready = (uint64_t*)(((uintptr_t)(inv_s + 2 * NT) + 7) & ~(uintptr_t)7);   // [S] normalised B stages
-    __nv_bfloat16* sgain = (__nv_bfloat16*)(((uintptr_t)(ready + S) + 15) & ~(uintptr_t)15);   // [GAIN_MAX]
-    static_assert((2 * S + 6) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+    uint64_t* ready = smem_align_up<uint64_t>(inv_s + 2 * NT, 8);   // [S] normalised B stages
+    __nv_bfloat16* sgain = smem_align_up<__nv_bfloat16>(ready + S, 16);   // [GAIN_MAX]
+    static_assert((2 * S + 9) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
                       C::MISC_BYTES, "misc");
 
+    // shared-window addresses of what the epilogues read back
+    const uint32_t xch_a = smem_u32(xch), tok_b_a = smem_u32(tok_b), tok_pos_a = smem_u32(tok_pos);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 8 : nullptr;
     const long long clk0 = clock64();
@@ -171,6 +174,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
         for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 2);   // one arrival per normaliser warp
         mbar_init(drain, 1);
         mbar_init(landb, 1);
+        for (int j = 0; j < 3; ++j) mbar_init(&landc[j], 1);
         if (CL) {
             // The CTA's last segment is a split tile it finishes when it starts at the
             // tile's k-block 0 and ends inside it: expect its peers' partials.
@@ -498,7 +502,8 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     const int half = p.d >> 1, ih = (lr % p.d) % half;
 #pragma unroll
                     for (int i = 0; i < CH; ++i)
-                        pre_cs[i] = (rot && row_ok && tok_b[i] >= 0) ? __ldg(&p.rope[(size_t)tok_pos[i] * half + ih])
+                        pre_cs[i] = (rot && row_ok && lds_s32(tok_b_a + i * 4u) >= 0)
+                                        ? __ldg(&p.rope[(size_t)lds_s32(tok_pos_a + i * 4u) * half + ih])
                                                                      : make_float2(1.f, 0.f);
                 }
             }
@@ -576,6 +581,74 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                 }
                 if (named_bar_or(1, 128, !lok)) break;
             }
+            // Wider tiles (NT >= 64) finished in the CTA's last segment: the ring is idle
+            // then (every stage consumed, no load in flight), so what each CH-token chunk
+            // of the epilogue reads from global memory lands there by bulk copies, up to
+            // three chunks ahead of the chunk being finished, instead of every chunk
+            // waiting on rounds of dependent register loads: the peers' partials (the CH
+            // columns of a chunk are contiguous in a column-major partial) and the
+            // epilogue's inputs, the residual rows of the chunk's tokens (EPI_RESID) or
+            // their RoPE rows (rotated sections of EPI_QKV / EPI_INJECT).
+            static_assert(NT < 64 || CH == 32, "one chunk token per lane of the issuing warp");
+            constexpr int LC_BYTES = CH * 128 * 4;          // one chunk of one partial
+            constexpr int RING_BYTES = S * C::STAGE_BYTES;
+            const bool rot_tile = p.epi == EPI_QKV ? mi <= 1 : (p.epi == EPI_INJECT && (mi & 1) == 0);
+            const int n_peer = fin_first ? nc - 1 : 0;
+            const int aux_row = p.epi == EPI_RESID ? (p.has_tx ? 128 * 2 : -1)
+                                                   : (rot_tile ? (p.d >> 1) * 8 : 0);   // bytes per token
+            const int lbuf = n_peer * LC_BYTES + CH * max(aux_row, 0);                            // bytes per chunk
+            const bool last_seg = u + (kb1 - kb0) == u_end;
+            const int lc_depth = (NT >= 64 && !CL && last_seg && (fin_first || whole) && aux_row >= 0 && lbuf > 0 &&
+                                  lbuf <= RING_BYTES)
+                                     ? min(3, min(NT / CH, RING_BYTES / lbuf))
+                                     : 0;
+            const int lcd = lc_depth > 0 ? lc_depth : 1;   // buffers (a divisor when the mode is off)
+            int lc_issued = 0;                             // chunks issued (the same count in every thread)
+            // Issued by the 32 threads of warp e < 32: thread e < n_peer copies its peer's
+            // chunk; the residual rows come as one 32 x 128 tensor tile; the RoPE rows of
+            // the chunk's tokens as one copy per run of consecutive positions of a request
+            // (thread e copies the run that starts at token e).
+            const float* lc_psrc = (lc_depth > 0 && e < n_peer)
+                                       ? p.partial + (size_t)slot_of(firsti + 1 + e) * NT * 128 : nullptr;
+            auto lc_issue = [&](int c) {
+                uint64_t* bar = &landc[c % lcd];
+                uint8_t* dst = smem + (size_t)(c % lcd) * lbuf;
+                uint8_t* aux = dst + (size_t)n_peer * LC_BYTES;
+                const void* src = nullptr;
+                uint32_t bytes = 0;
+                uint32_t tile_bytes = 0;
+                if (p.epi == EPI_RESID) {
+                    tile_bytes = CH * 128 * 2;
+                } else if (rot_tile) {
+                    const int tk = c * CH + e;
+                    const int b = lds_s32(tok_b_a + tk * 4u), pos = lds_s32(tok_pos_a + tk * 4u);
+                    const int pb = __shfl_up_sync(0xffffffffu, b, 1), ppos = __shfl_up_sync(0xffffffffu, pos, 1);
+                    const bool valid = b >= 0;
+                    const bool start = valid && !(e > 0 && pb == b && ppos + 1 == pos);
+                    const uint32_t starts = __ballot_sync(0xffffffffu, start), valids = __ballot_sync(0xffffffffu, valid);
+                    if (start) {
+                        const uint32_t stops = (starts | ~valids) & ~((2u << e) - 1u);   // lanes after e that end the run
+                        const int f = stops ? __ffs(stops) - 1 : 32;
+                        src = p.rope + (size_t)pos * (p.d >> 1);
+                        bytes = (uint32_t)((f - e) * aux_row);
+                    }
+                }
+                const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + tile_bytes + (uint32_t)(n_peer * LC_BYTES);
+                if (e == 0) mbar_arrive_expect_tx(bar, total);
+                __syncwarp();
+                if (bytes) bulk_load(aux + (size_t)e * aux_row, src, bytes, bar);
+                if (tile_bytes && e == 0)
+                    tma_load_2d(aux, &p.tx, bar, (n_tile - p.amat[mi].tile0) * 128, m_tile * NT + c * CH);
+                if (e < n_peer) bulk_load(dst + (size_t)e * LC_BYTES, lc_psrc + (size_t)c * CH * 128, (uint32_t)LC_BYTES, bar);
+            };
+            if (lc_depth > 0) {
+                if (e < 32) {
+                    fence_proxy_async_global();   // the partials seen through the count's acquire
+                    for (int c = 0; c < lc_depth; ++c) lc_issue(c);
+                }
+                lc_issued = lc_depth;
+            }
+            bool lost = false;
             bool finish = true;
             if (!whole && !fin_first && CL) {
                 // Send the partial (all NT columns of this thread's row) into the
@@ -616,7 +689,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         *s_flag = last ? 1 : 0;
                     }
                     named_bar_sync(1, 128);
-                    finish = (*s_flag != 0);
+                    finish = (lds_s32(smem_u32(s_flag)) != 0);
                 } else {
                     if (e == 0) {
                         __threadfence();
@@ -631,16 +704,42 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     float v[CH];
 #pragma unroll
                     for (int h = 0; h < CH; h += 16) tmem_ld16(tb + c0 + h, v + h);
-                    if (!whole && CL) {
+                    if (lc_depth > 0) {
+                        // this CTA first (the first contributor), then the landed chunks of
+                        // the partials in contributor order
+                        const int ci = c0 / CH;
+                        const bool lok = mbar_wait(&landc[ci % lcd], (uint32_t)((ci / lcd) & 1), abort_flag, p.status);
+                        if (named_bar_or(1, 128, !lok)) {
+                            if (e == 0) {
+                                volatile int never = 0;   // let the copies in flight land before the CTA can leave
+                                for (int c = ci; c < lc_issued; ++c)
+                                    mbar_wait(&landc[c % lcd], (uint32_t)((c / lcd) & 1), &never, nullptr);
+                            }
+                            lost = true;
+                            break;
+                        }
+                        if (n_peer > 0) {
+                            uint32_t src = smem_u32(smem + (size_t)(ci % lcd) * lbuf) + (uint32_t)row * 4u;
+                            float acc[CH];
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) acc[i] = 0.0f + v[i];
+                            for (int b = 0; b < n_peer; ++b, src += CH * 128 * 4) {
+#pragma unroll
+                                for (int i = 0; i < CH; ++i) acc[i] += lds_f32(src + i * 512u);
+                            }
+#pragma unroll
+                            for (int i = 0; i < CH; ++i) v[i] = acc[i];
+                        }
+                    } else if (!whole && CL) {
                         // this CTA first, then the peers' partials in rank order
                         float acc[CH];
 #pragma unroll
                         for (int i = 0; i < CH; ++i) acc[i] = 0.0f + v[i];
                         for (int b = 1; b < nc; ++b) {
-                            const float* src = land + ((size_t)(b - 1) * 128 + row) * C::LAND_LD + c0;
+                            const uint32_t src = smem_u32(land + ((size_t)(b - 1) * 128 + row) * C::LAND_LD + c0);
 #pragma unroll
                             for (int i = 0; i < CH; i += 4) {
-                                const float4 w = *reinterpret_cast<const float4*>(src + i);
+                                const float4 w = lds_f32x4(src + i * 4u);
                                 acc[i] += w.x;
                                 acc[i + 1] += w.y;
                                 acc[i + 2] += w.z;
@@ -656,9 +755,9 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
 #pragma unroll
                         for (int i = 0; i < CH; ++i) acc[i] = 0.0f + v[i];
                         for (int b = 1; b < nc; ++b) {
-                            const float* src = reinterpret_cast<const float*>(sA) + (size_t)(b - 1) * NT * 128;
+                            const uint32_t src = smem_u32(sA) + (uint32_t)(((b - 1) * NT * 128 + c0 * 128 + row) * 4);
 #pragma unroll
-                            for (int i = 0; i < CH; ++i) acc[i] += src[(c0 + i) * 128 + row];
+                            for (int i = 0; i < CH; ++i) acc[i] += lds_f32(src + i * 512u);
                         }
 #pragma unroll
                         for (int i = 0; i < CH; ++i) v[i] = acc[i];
@@ -712,6 +811,13 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                             if constexpr (PRE) {
 #pragma unroll
                                 for (int i = 0; i < CH; ++i) rv[i] = pre_x[i];
+                            } else if (lc_depth > 0) {
+                                // the chunk's residual rows landed after the partials
+                                const uint32_t xs = smem_u32(smem + (size_t)((c0 / CH) % lcd) * lbuf + (size_t)n_peer * LC_BYTES) +
+                                                    (uint32_t)row * 2u;
+#pragma unroll
+                                for (int i = 0; i < CH; ++i)
+                                    rv[i] = (row_ok && mbase + i < p.M) ? lds_bf16_as_f32(xs + i * 256u) : 0.f;
                             } else {
 #pragma unroll
                                 for (int i = 0; i < CH; ++i)
@@ -730,7 +836,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                             const int c = e + 128 * k, i = c >> 4, r0 = (c & 15) * 8;
                             const int m = mbase + i, f = rbase + r0;
                             const bool in = m < p.M && f < nrows;   // rows come in multiples of 8
-                            const uint4 w = *(const uint4*)(xout + i * 128 + r0);
+                            const uint4 w = lds_u32x4(xch_a + (uint32_t)(i * 128 + r0) * 2u);
                             if (in) *(uint4*)(o + (size_t)m * p.ldo + f) = w;
                             if (p.ssq_out) {
                                 // the 8 features in order, then the 16 pieces of the token
@@ -763,7 +869,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         if (row < 64)
 #pragma unroll
                             for (int i = 0; i < CH; ++i)
-                                xout[i * 64 + row] = f2bf(silu(v[i]) * xch[(row + 64) * (CH + 1) + i]);
+                                xout[i * 64 + row] = f2bf(silu(v[i]) * lds_f32(xch_a + (uint32_t)((row + 64) * (CH + 1) + i) * 4u));
                         named_bar_sync(1, 128);
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
 #pragma unroll
@@ -771,7 +877,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                             const int c = e + 128 * k, i = c >> 3, r0 = (c & 7) * 8;
                             const int m = mbase + i;
                             if (m < p.M)
-                                *(uint4*)(o + (size_t)m * p.ldo + n_tile * 64 + r0) = *(const uint4*)(xout + i * 64 + r0);
+                                *(uint4*)(o + (size_t)m * p.ldo + n_tile * 64 + r0) = lds_u32x4(xch_a + (uint32_t)(i * 64 + r0) * 2u);
                         }
                         named_bar_sync(1, 128);
                         break;
@@ -796,12 +902,20 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         if constexpr (PRE) {
 #pragma unroll
                             for (int i = 0; i < CH; ++i) cs[i] = pre_cs[i];
+                        } else if (lc_depth > 0 && rotate) {
+                            // the chunk's RoPE rows landed after the partials
+                            const uint32_t rs = smem_u32(smem + (size_t)((c0 / CH) % lcd) * lbuf + (size_t)n_peer * LC_BYTES) +
+                                                (uint32_t)(i_in % half) * 8u;
+#pragma unroll
+                            for (int i = 0; i < CH; ++i)
+                                cs[i] = (row_ok && lds_s32(tok_b_a + (c0 + i) * 4u) >= 0) ? lds_f32x2(rs + (uint32_t)(i * half) * 8u)
+                                                                                          : make_float2(1.f, 0.f);
                         } else {
 #pragma unroll
                             for (int i = 0; i < CH; ++i) {
-                                const int b = tok_b[c0 + i];
+                                const int b = lds_s32(tok_b_a + (c0 + i) * 4u);
                                 cs[i] = (rotate && row_ok && b >= 0)
-                                            ? __ldg(&p.rope[(size_t)tok_pos[c0 + i] * half + (i_in % half)])
+                                            ? __ldg(&p.rope[(size_t)lds_s32(tok_pos_a + (c0 + i) * 4u) * half + (i_in % half)])
                                             : make_float2(1.f, 0.f);
                             }
                         }
@@ -810,7 +924,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         for (int i = 0; i < CH; ++i) {
                             float x = v[i];
                             if (rotate) {
-                                const float pr = xch[prow * (CH + 1) + i];
+                                const float pr = lds_f32(xch_a + (uint32_t)(prow * (CH + 1) + i) * 4u);
                                 x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
                             }
                             y[i] = f2bf(x);
@@ -825,14 +939,14 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
 #pragma unroll
                         for (int k = 0; k < CH / 8; ++k) {
                             const int c = e + 128 * k, i = c >> 4, r0 = (c & 15) * 8;
-                            const int b = tok_b[c0 + i], f = rbase + r0;
+                            const int b = lds_s32(tok_b_a + (c0 + i) * 4u), f = rbase + r0;
                             if (b >= 0 && f < nrows) {
-                                const uint4 w = *(const uint4*)(xout + i * 128 + r0);
+                                const uint4 w = lds_u32x4(xch_a + (uint32_t)(i * 128 + r0) * 2u);
                                 __nv_bfloat16* dst =
                                     is_q ? (__nv_bfloat16*)p.out + (size_t)(mbase + i) * p.ldo + f
                                          : p.slab + (size_t)b * p.s_req + (size_t)layer * p.s_layer +
                                                (size_t)kind * p.s_kind + (size_t)(f / d) * p.s_kv +
-                                               (size_t)tok_pos[c0 + i] * d + (f % d);
+                                               (size_t)lds_s32(tok_pos_a + (c0 + i) * 4u) * d + (f % d);
                                 *(uint4*)dst = w;
                             }
                         }
@@ -869,7 +983,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
 #pragma unroll
                         for (int k = 0; k < CH; ++k) {
                             const int r = j + G * k;
-                            top2_merge(a1, ai, a2, xch[r * (CH + 1) + i], vbase + r, -INFINITY);
+                            top2_merge(a1, ai, a2, lds_f32(xch_a + (uint32_t)(r * (CH + 1) + i) * 4u), vbase + r, -INFINITY);
                         }
 #pragma unroll
                         for (int off = G / 2; off > 0; off >>= 1) {
@@ -886,7 +1000,17 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     default:
                         break;
                     }
+                    if (lc_depth > 0) {
+                        // the chunk's buffer is free once every thread is done with it: the
+                        // chunk lc_depth ahead lands there
+                        named_bar_sync(1, 128);
+                        if (lc_issued < NT / CH) {
+                            if (e < 32) lc_issue(lc_issued);
+                            ++lc_issued;
+                        }
+                    }
                 }
+                if (lost) break;
                 if (!whole && !CL && e == 0) p.counters[t] = 0;
             }
             tc_fence_before();
@@ -1050,6 +1174,11 @@ int launch_gemm_tc(GemmParams& p, int nt, int num_sms, cudaStream_t stream) {
              p.s_kind % 8 != 0 || p.s_kv % 8 != 0))
             return (int)cudaErrorInvalidValue;
     }
+    // Residual rows for the chunked landing of wide tiles: 32 tokens x 128 features
+    // per copy (the kernel falls back to register loads without it).
+    p.has_tx = 0;
+    if (p.epi == EPI_RESID && nt >= 64 && p.n_amat == 1)
+        p.has_tx = encode_bf16_rows(&p.tx, p.out, (uint64_t)p.amat[0].rows, (uint64_t)p.M, (uint64_t)p.ldo, 128, 32) ? 1 : 0;
     p.units = (long long)p.n_tiles * p.m_tiles * p.KB;
     if (p.units * (long long)kGemmMaxGrid >= (1LL << 32)) return (int)cudaErrorInvalidValue;   // 32-bit partition arithmetic
     const bool auto_grid = p.ctas <= 0;

@@ -62,12 +62,18 @@ def test_gemm_result_does_not_depend_on_partition_much():
 
 
 @pytest.mark.parametrize("M,N,K,grid", [(16, 512, 2048, 7), (16, 128, 12288, 0), (33, 1000, 4096, 0),
-                                        (200, 640, 1024, 64), (16, 4096, 4096, 0), (5, 384, 704, 100)])
+                                        (200, 640, 1024, 64), (16, 4096, 4096, 0), (5, 384, 704, 100),
+                                        (256, 6144, 4096, 0), (256, 4096, 4096, 0), (256, 2048, 4096, 0),
+                                        (256, 1024, 4096, 0), (128, 1024, 4096, 0), (64, 2048, 4096, 0),
+                                        (250, 4096, 14336, 0)])
 def test_split_tile_finishers_agree_bitwise(M, N, K, grid):
     """A split tile finished by its first contributor (waiting for the others'
     partials) and by its last arriver adds the same partials in the same order:
     identical bits, every call.  (16, 128, 12288) on the full grid splits one tile
-    over all CTAs, so the first contributor waits for every other one."""
+    over all CTAs, so the first contributor waits for every other one.  The 64- to
+    256-token tiles cover the chunked landing of wide partials at every depth (about
+    3, 5, 10 and 18 contributors per tile: three, two and one chunk ahead, and the
+    register path past the ring's capacity)."""
     try:
         D.dflash_diag_set_split_finisher(True)
         _, last = _run(M, N, K, grid=grid, calls=2)
