@@ -80,6 +80,20 @@ DF_DEV void top2_merge(float& a1, int& ai, float& a2, float b1, int bi, float b2
     }
 }
 
+// What the producer warp copies into the idle ring for the finishing epilogue of a
+// wide tile (posted by the epilogue once the tile's accumulator and the peers'
+// partials are ready; depth 0: nothing).
+struct LandPlan {
+    int depth;                 // chunk buffers in flight (0: no landing)
+    int nchunks;               // CH-token chunks of the tile
+    int lbuf;                  // bytes per chunk buffer
+    int n_peer;                // peers' partial chunks per buffer (first, 16 KB each)
+    int aux;                   // 0 none, 1 residual rows (tensor tile), 2 RoPE rows of the chunk's tokens
+    int aux_row;               // aux bytes per token
+    int tx_x, tx_y0;           // residual tile coordinates of chunk 0
+    const float* psrc[12];     // the peers' partials of this tile
+};
+
 template <int NT, bool CLU>
 __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::MIN_BLOCKS)
     k_gemm_tc(const __grid_constant__ GemmParams p) {
@@ -99,8 +113,10 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     uint64_t* acce = accf + 2;
     uint64_t* drain = acce + 2;
     uint64_t* landb = drain + 1;      // cluster mode: the peers' partials have landed
-    uint64_t* landc = landb + 1;      // [3] chunked landing of the peers' partials (NT >= 64)
-    uint32_t* tmem_slot = (uint32_t*)(landc + 3);
+    uint64_t* landc = landb + 1;      // [3] chunked landing: chunk buffer filled (NT >= 64)
+    uint64_t* lfree = landc + 3;      // [3] chunked landing: chunk buffer consumed by the epilogue
+    uint64_t* land_go = lfree + 3;    // chunked landing: the plan is posted
+    uint32_t* tmem_slot = (uint32_t*)(land_go + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* s_flag = (int*)(tmem_slot + 2);
     int* tok_b = s_flag + 1;          // [NT]
@@ -108,7 +124,9 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
     float* inv_s = (float*)(tok_pos + NT);   // [2][NT] inverse RMS of the current m-tile's rows, per normaliser warp
     uint64_t* ready = smem_align_up<uint64_t>(inv_s + 2 * NT, 8);   // [S] normalised B stages
     __nv_bfloat16* sgain = smem_align_up<__nv_bfloat16>(ready + S, 16);   // [GAIN_MAX]
-    static_assert((2 * S + 9) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 <=
+    LandPlan* plan = smem_align_up<LandPlan>(sgain + C::GAIN_MAX, 16);
+    static_assert((2 * S + 13) * 8 + 16 + 2 * NT * 4 + 2 * NT * 4 + 8 + S * 8 + 16 + C::GAIN_MAX * 2 + 16 +
+                          (int)sizeof(LandPlan) <=
                       C::MISC_BYTES, "misc");
 
     // shared-window addresses of what the epilogues read back
@@ -174,7 +192,11 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
         for (int s2 = 0; s2 < S; ++s2) mbar_init(&ready[s2], 2);   // one arrival per normaliser warp
         mbar_init(drain, 1);
         mbar_init(landb, 1);
-        for (int j = 0; j < 3; ++j) mbar_init(&landc[j], 1);
+        for (int j = 0; j < 3; ++j) {
+            mbar_init(&landc[j], 1);
+            mbar_init(&lfree[j], 128);
+        }
+        mbar_init(land_go, 1);
         if (CL) {
             // The CTA's last segment is a split tile it finishes when it starts at the
             // tile's k-block 0 and ends inside it: expect its peers' partials.
@@ -290,6 +312,54 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                 for (long long i = first; i < issued; ++i) {
                     volatile int never = 0;
                     mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), &never, nullptr);
+                }
+            } else if (NT >= 64 && u_begin < u_end && mbar_wait(land_go, 0, abort_flag, p.status)) {
+                // Finishing inputs of the last tile: chunk c into buffer c % depth, once
+                // the epilogue has consumed the chunk that buffer held.
+                const LandPlan pl = *plan;
+                if (pl.depth > 0) {
+                    fence_proxy_async_global();   // the partials, seen through the epilogue's acquire
+                    int nis = 0;
+                    for (int c = 0; c < pl.nchunks; ++c) {
+                        if (c >= pl.depth &&
+                            !mbar_wait(&lfree[c % pl.depth], (uint32_t)((c / pl.depth - 1) & 1), abort_flag, p.status))
+                            break;
+                        uint64_t* bar = &landc[c % pl.depth];
+                        uint8_t* dst = smem + (size_t)(c % pl.depth) * pl.lbuf;
+                        uint8_t* aux = dst + (size_t)pl.n_peer * (CH * 128 * 4);
+                        uint32_t total = (uint32_t)(pl.n_peer * CH * 128 * 4);
+                        if (pl.aux == 1) total += CH * 128 * 2;
+                        if (pl.aux == 2)
+                            for (int i = 0; i < CH; ++i) total += lds_s32(tok_b_a + (c * CH + i) * 4u) >= 0 ? pl.aux_row : 0;
+                        mbar_arrive_expect_tx(bar, total);
+                        for (int b = 0; b < pl.n_peer; ++b)
+                            bulk_load(dst + (size_t)b * (CH * 128 * 4), pl.psrc[b] + (size_t)c * CH * 128,
+                                      (uint32_t)(CH * 128 * 4), bar);
+                        if (pl.aux == 1) tma_load_2d(aux, &p.tx, bar, pl.tx_x, pl.tx_y0 + c * CH);
+                        if (pl.aux == 2) {
+                            // one copy per run of consecutive positions of one request
+                            const int half = p.d >> 1;
+                            for (int i = 0; i < CH;) {
+                                const int b = lds_s32(tok_b_a + (c * CH + i) * 4u), pos = lds_s32(tok_pos_a + (c * CH + i) * 4u);
+                                int j = i + 1;
+                                if (b >= 0)
+                                    while (j < CH && lds_s32(tok_b_a + (c * CH + j) * 4u) == b &&
+                                           lds_s32(tok_pos_a + (c * CH + j) * 4u) == pos + (j - i))
+                                        ++j;
+                                if (b >= 0)
+                                    bulk_load(aux + (size_t)i * pl.aux_row, p.rope + (size_t)pos * half,
+                                              (uint32_t)((j - i) * pl.aux_row), bar);
+                                i = j;
+                            }
+                        }
+                        ++nis;
+                    }
+                    // every issued copy lands before the CTA can leave (the latest chunk of each buffer)
+                    for (int b = 0; b < pl.depth && b < nis; ++b) {
+                        const int last = b + pl.depth * ((nis - 1 - b) / pl.depth);
+                        volatile int never = 0;
+                        mbar_wait(&landc[b], (uint32_t)((last / pl.depth) & 1), &never, nullptr);
+                    }
                 }
             }
         }
@@ -589,7 +659,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
             // columns of a chunk are contiguous in a column-major partial) and the
             // epilogue's inputs, the residual rows of the chunk's tokens (EPI_RESID) or
             // their RoPE rows (rotated sections of EPI_QKV / EPI_INJECT).
-            static_assert(NT < 64 || CH == 32, "one chunk token per lane of the issuing warp");
+            static_assert(NT < 64 || CH == 32, "32-token chunks");
             constexpr int LC_BYTES = CH * 128 * 4;          // one chunk of one partial
             constexpr int RING_BYTES = S * C::STAGE_BYTES;
             const bool rot_tile = p.epi == EPI_QKV ? mi <= 1 : (p.epi == EPI_INJECT && (mi & 1) == 0);
@@ -603,50 +673,24 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                                      ? min(3, min(NT / CH, RING_BYTES / lbuf))
                                      : 0;
             const int lcd = lc_depth > 0 ? lc_depth : 1;   // buffers (a divisor when the mode is off)
-            int lc_issued = 0;                             // chunks issued (the same count in every thread)
-            // Issued by the 32 threads of warp e < 32: thread e < n_peer copies its peer's
-            // chunk; the residual rows come as one 32 x 128 tensor tile; the RoPE rows of
-            // the chunk's tokens as one copy per run of consecutive positions of a request
-            // (thread e copies the run that starts at token e).
-            const float* lc_psrc = (lc_depth > 0 && e < n_peer)
-                                       ? p.partial + (size_t)slot_of(firsti + 1 + e) * NT * 128 : nullptr;
-            auto lc_issue = [&](int c) {
-                uint64_t* bar = &landc[c % lcd];
-                uint8_t* dst = smem + (size_t)(c % lcd) * lbuf;
-                uint8_t* aux = dst + (size_t)n_peer * LC_BYTES;
-                const void* src = nullptr;
-                uint32_t bytes = 0;
-                uint32_t tile_bytes = 0;
-                if (p.epi == EPI_RESID) {
-                    tile_bytes = CH * 128 * 2;
-                } else if (rot_tile) {
-                    const int tk = c * CH + e;
-                    const int b = lds_s32(tok_b_a + tk * 4u), pos = lds_s32(tok_pos_a + tk * 4u);
-                    const int pb = __shfl_up_sync(0xffffffffu, b, 1), ppos = __shfl_up_sync(0xffffffffu, pos, 1);
-                    const bool valid = b >= 0;
-                    const bool start = valid && !(e > 0 && pb == b && ppos + 1 == pos);
-                    const uint32_t starts = __ballot_sync(0xffffffffu, start), valids = __ballot_sync(0xffffffffu, valid);
-                    if (start) {
-                        const uint32_t stops = (starts | ~valids) & ~((2u << e) - 1u);   // lanes after e that end the run
-                        const int f = stops ? __ffs(stops) - 1 : 32;
-                        src = p.rope + (size_t)pos * (p.d >> 1);
-                        bytes = (uint32_t)((f - e) * aux_row);
+            if (NT >= 64 && last_seg) {
+                // Post the landing plan to the producer warp (every CTA, once, at its last
+                // segment; depth 0 when nothing lands).
+                if (e < 32) {
+                    if (lc_depth > 0 && e < n_peer) plan->psrc[e] = p.partial + (size_t)slot_of(firsti + 1 + e) * NT * 128;
+                    __syncwarp();
+                    if (e == 0) {
+                        plan->depth = lc_depth;
+                        plan->nchunks = NT / CH;
+                        plan->lbuf = lbuf;
+                        plan->n_peer = n_peer;
+                        plan->aux = p.epi == EPI_RESID ? 1 : (rot_tile ? 2 : 0);
+                        plan->aux_row = max(aux_row, 0);
+                        plan->tx_x = (n_tile - p.amat[mi].tile0) * 128;
+                        plan->tx_y0 = m_tile * NT;
+                        mbar_arrive(land_go);
                     }
                 }
-                const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + tile_bytes + (uint32_t)(n_peer * LC_BYTES);
-                if (e == 0) mbar_arrive_expect_tx(bar, total);
-                __syncwarp();
-                if (bytes) bulk_load(aux + (size_t)e * aux_row, src, bytes, bar);
-                if (tile_bytes && e == 0)
-                    tma_load_2d(aux, &p.tx, bar, (n_tile - p.amat[mi].tile0) * 128, m_tile * NT + c * CH);
-                if (e < n_peer) bulk_load(dst + (size_t)e * LC_BYTES, lc_psrc + (size_t)c * CH * 128, (uint32_t)LC_BYTES, bar);
-            };
-            if (lc_depth > 0) {
-                if (e < 32) {
-                    fence_proxy_async_global();   // the partials seen through the count's acquire
-                    for (int c = 0; c < lc_depth; ++c) lc_issue(c);
-                }
-                lc_issued = lc_depth;
             }
             bool lost = false;
             bool finish = true;
@@ -709,12 +753,7 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         // the partials in contributor order
                         const int ci = c0 / CH;
                         const bool lok = mbar_wait(&landc[ci % lcd], (uint32_t)((ci / lcd) & 1), abort_flag, p.status);
-                        if (named_bar_or(1, 128, !lok)) {
-                            if (e == 0) {
-                                volatile int never = 0;   // let the copies in flight land before the CTA can leave
-                                for (int c = ci; c < lc_issued; ++c)
-                                    mbar_wait(&landc[c % lcd], (uint32_t)((c / lcd) & 1), &never, nullptr);
-                            }
+                        if (named_bar_or(1, 128, !lok)) {   // the producer lets its copies land
                             lost = true;
                             break;
                         }
@@ -815,9 +854,13 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                                 // the chunk's residual rows landed after the partials
                                 const uint32_t xs = smem_u32(smem + (size_t)((c0 / CH) % lcd) * lbuf + (size_t)n_peer * LC_BYTES) +
                                                     (uint32_t)row * 2u;
+                                // loaded unconditionally (the landed rows always exist), then
+                                // selected: a load under a condition serialises the chunk
 #pragma unroll
-                                for (int i = 0; i < CH; ++i)
-                                    rv[i] = (row_ok && mbase + i < p.M) ? lds_bf16_as_f32(xs + i * 256u) : 0.f;
+                                for (int i = 0; i < CH; ++i) {
+                                    const float xv = lds_bf16_as_f32(xs + i * 256u);
+                                    rv[i] = (row_ok && mbase + i < p.M) ? xv : 0.f;
+                                }
                             } else {
 #pragma unroll
                                 for (int i = 0; i < CH; ++i)
@@ -907,9 +950,11 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                             const uint32_t rs = smem_u32(smem + (size_t)((c0 / CH) % lcd) * lbuf + (size_t)n_peer * LC_BYTES) +
                                                 (uint32_t)(i_in % half) * 8u;
 #pragma unroll
-                            for (int i = 0; i < CH; ++i)
-                                cs[i] = (row_ok && lds_s32(tok_b_a + (c0 + i) * 4u) >= 0) ? lds_f32x2(rs + (uint32_t)(i * half) * 8u)
-                                                                                          : make_float2(1.f, 0.f);
+                            for (int i = 0; i < CH; ++i) {
+                                const int b = lds_s32(tok_b_a + (c0 + i) * 4u);
+                                const float2 r = lds_f32x2(rs + (uint32_t)(i * half) * 8u);   // unconditional, then selected
+                                cs[i] = (row_ok && b >= 0) ? r : make_float2(1.f, 0.f);
+                            }
                         } else {
 #pragma unroll
                             for (int i = 0; i < CH; ++i) {
@@ -923,10 +968,8 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
 #pragma unroll
                         for (int i = 0; i < CH; ++i) {
                             float x = v[i];
-                            if (rotate) {
-                                const float pr = lds_f32(xch_a + (uint32_t)(prow * (CH + 1) + i) * 4u);
-                                x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
-                            }
+                            const float pr = lds_f32(xch_a + (uint32_t)(prow * (CH + 1) + i) * 4u);   // unconditional
+                            if (rotate) x = (i_in < half) ? (x * cs[i].x - pr * cs[i].y) : (x * cs[i].x + pr * cs[i].y);
                             y[i] = f2bf(x);
                         }
                         named_bar_sync(1, 128);
@@ -940,13 +983,14 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                         for (int k = 0; k < CH / 8; ++k) {
                             const int c = e + 128 * k, i = c >> 4, r0 = (c & 15) * 8;
                             const int b = lds_s32(tok_b_a + (c0 + i) * 4u), f = rbase + r0;
+                            const int tpos = lds_s32(tok_pos_a + (c0 + i) * 4u);
+                            const uint4 w = lds_u32x4(xch_a + (uint32_t)(i * 128 + r0) * 2u);
                             if (b >= 0 && f < nrows) {
-                                const uint4 w = lds_u32x4(xch_a + (uint32_t)(i * 128 + r0) * 2u);
                                 __nv_bfloat16* dst =
                                     is_q ? (__nv_bfloat16*)p.out + (size_t)(mbase + i) * p.ldo + f
                                          : p.slab + (size_t)b * p.s_req + (size_t)layer * p.s_layer +
                                                (size_t)kind * p.s_kind + (size_t)(f / d) * p.s_kv +
-                                               (size_t)lds_s32(tok_pos_a + (c0 + i) * 4u) * d + (f % d);
+                                               (size_t)tpos * d + (f % d);
                                 *(uint4*)dst = w;
                             }
                         }
@@ -1000,15 +1044,9 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     default:
                         break;
                     }
-                    if (lc_depth > 0) {
-                        // the chunk's buffer is free once every thread is done with it: the
-                        // chunk lc_depth ahead lands there
-                        named_bar_sync(1, 128);
-                        if (lc_issued < NT / CH) {
-                            if (e < 32) lc_issue(lc_issued);
-                            ++lc_issued;
-                        }
-                    }
+                    // the chunk's buffer is free for the chunk lc_depth ahead once every
+                    // thread is done with it
+                    if (lc_depth > 0) mbar_arrive(&lfree[(c0 / CH) % lcd]);
                 }
                 if (lost) break;
                 if (!whole && !CL && e == 0) p.counters[t] = 0;
