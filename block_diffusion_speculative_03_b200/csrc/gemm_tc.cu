@@ -313,54 +313,62 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     volatile int never = 0;
                     mbar_wait(&full[i % S], (uint32_t)((i / S) & 1), &never, nullptr);
                 }
-            } else if (NT >= 64 && u_begin < u_end && mbar_wait(land_go, 0, abort_flag, p.status)) {
-                // Finishing inputs of the last tile: chunk c into buffer c % depth, once
-                // the epilogue has consumed the chunk that buffer held.
-                const LandPlan pl = *plan;
-                if (pl.depth > 0) {
-                    fence_proxy_async_global();   // the partials, seen through the epilogue's acquire
-                    int nis = 0;
-                    for (int c = 0; c < pl.nchunks; ++c) {
-                        if (c >= pl.depth &&
-                            !mbar_wait(&lfree[c % pl.depth], (uint32_t)((c / pl.depth - 1) & 1), abort_flag, p.status))
-                            break;
-                        uint64_t* bar = &landc[c % pl.depth];
-                        uint8_t* dst = smem + (size_t)(c % pl.depth) * pl.lbuf;
-                        uint8_t* aux = dst + (size_t)pl.n_peer * (CH * 128 * 4);
-                        uint32_t total = (uint32_t)(pl.n_peer * CH * 128 * 4);
-                        if (pl.aux == 1) total += CH * 128 * 2;
-                        if (pl.aux == 2)
-                            for (int i = 0; i < CH; ++i) total += lds_s32(tok_b_a + (c * CH + i) * 4u) >= 0 ? pl.aux_row : 0;
-                        mbar_arrive_expect_tx(bar, total);
-                        for (int b = 0; b < pl.n_peer; ++b)
-                            bulk_load(dst + (size_t)b * (CH * 128 * 4), pl.psrc[b] + (size_t)c * CH * 128,
-                                      (uint32_t)(CH * 128 * 4), bar);
-                        if (pl.aux == 1) tma_load_2d(aux, &p.tx, bar, pl.tx_x, pl.tx_y0 + c * CH);
-                        if (pl.aux == 2) {
-                            // one copy per run of consecutive positions of one request
-                            const int half = p.d >> 1;
-                            for (int i = 0; i < CH;) {
-                                const int b = lds_s32(tok_b_a + (c * CH + i) * 4u), pos = lds_s32(tok_pos_a + (c * CH + i) * 4u);
-                                int j = i + 1;
-                                if (b >= 0)
-                                    while (j < CH && lds_s32(tok_b_a + (c * CH + j) * 4u) == b &&
-                                           lds_s32(tok_pos_a + (c * CH + j) * 4u) == pos + (j - i))
-                                        ++j;
-                                if (b >= 0)
-                                    bulk_load(aux + (size_t)i * pl.aux_row, p.rope + (size_t)pos * half,
-                                              (uint32_t)((j - i) * pl.aux_row), bar);
-                                i = j;
-                            }
-                        }
-                        ++nis;
+            }
+        }
+        // Finishing inputs of the last tile of a wide-tile CTA, issued by the whole warp
+        // once the epilogue posts the plan: chunk c into buffer c % depth, once the
+        // epilogue has consumed the chunk that buffer held.
+        __syncwarp();
+        if (NT >= 64 && u_begin < u_end && !*abort_flag && mbar_wait(land_go, 0, abort_flag, p.status)) {
+            const LandPlan pl = *plan;
+            if (pl.depth > 0) {
+                fence_proxy_async_global();   // the partials, seen through the epilogue's acquire
+                int nis = 0;
+                for (int c = 0; c < pl.nchunks; ++c) {
+                    if (c >= pl.depth) {
+                        const bool fr = lane != 0 || mbar_wait(&lfree[c % pl.depth], (uint32_t)((c / pl.depth - 1) & 1),
+                                                               abort_flag, p.status);
+                        if (!__shfl_sync(0xffffffffu, (int)fr, 0)) break;
                     }
-                    // every issued copy lands before the CTA can leave (the latest chunk of each buffer)
+                    uint64_t* bar = &landc[c % pl.depth];
+                    uint8_t* dst = smem + (size_t)(c % pl.depth) * pl.lbuf;
+                    uint8_t* aux = dst + (size_t)pl.n_peer * (CH * 128 * 4);
+                    // RoPE rows: one copy per run of consecutive positions of one request,
+                    // issued by the lane of the run's first token
+                    const void* rsrc = nullptr;
+                    uint32_t rbytes = 0;
+                    if (pl.aux == 2) {
+                        const int tk = c * CH + lane;
+                        const int b = lds_s32(tok_b_a + tk * 4u), pos = lds_s32(tok_pos_a + tk * 4u);
+                        const int pb = __shfl_up_sync(0xffffffffu, b, 1), ppos = __shfl_up_sync(0xffffffffu, pos, 1);
+                        const bool valid = b >= 0;
+                        const bool start = valid && !(lane > 0 && pb == b && ppos + 1 == pos);
+                        const uint32_t starts = __ballot_sync(0xffffffffu, start), valids = __ballot_sync(0xffffffffu, valid);
+                        if (start) {
+                            const uint32_t stops = (starts | ~valids) & ~((2u << lane) - 1u);   // lanes after this one that end the run
+                            const int f = stops ? __ffs(stops) - 1 : 32;
+                            rsrc = p.rope + (size_t)pos * (p.d >> 1);
+                            rbytes = (uint32_t)((f - lane) * pl.aux_row);
+                        }
+                    }
+                    const uint32_t total = __reduce_add_sync(0xffffffffu, rbytes) + (uint32_t)(pl.n_peer * CH * 128 * 4) +
+                                           (pl.aux == 1 ? (uint32_t)(CH * 128 * 2) : 0u);
+                    if (lane == 0) mbar_arrive_expect_tx(bar, total);
+                    __syncwarp();
+                    if (lane < pl.n_peer)
+                        bulk_load(dst + (size_t)lane * (CH * 128 * 4), pl.psrc[lane] + (size_t)c * CH * 128,
+                                  (uint32_t)(CH * 128 * 4), bar);
+                    if (rbytes) bulk_load(aux + (size_t)lane * pl.aux_row, rsrc, rbytes, bar);
+                    if (pl.aux == 1 && lane == 0) tma_load_2d(aux, &p.tx, bar, pl.tx_x, pl.tx_y0 + c * CH);
+                    ++nis;
+                }
+                // every issued copy lands before the CTA can leave (the latest chunk of each buffer)
+                if (lane == 0)
                     for (int b = 0; b < pl.depth && b < nis; ++b) {
                         const int last = b + pl.depth * ((nis - 1 - b) / pl.depth);
                         volatile int never = 0;
                         mbar_wait(&landc[b], (uint32_t)((last / pl.depth) & 1), &never, nullptr);
                     }
-                }
             }
         }
     } else if (warp == 1) {
