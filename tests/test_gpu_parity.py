@@ -154,3 +154,25 @@ def test_small_bf16_wide_gqa_128_query_rows():
         anchors = pr.verify_and_accept(o_dr, w.gamma, plan[cyc], cyc)
         pr.check_cache()
     assert compared > 0
+
+
+@pytest.mark.parametrize("batch,gamma", [(3, 16), (5, 16), (13, 16), (7, 13)])
+def test_small_bf16_wide_token_tiles_ragged(batch, gamma):
+    # B x gamma = 48, 80, 208 and 91 rows: 64-, 128- and 256-token tiles whose last
+    # 32-token chunk is ragged, with split tiles finished from landed chunks of the
+    # peers' partials, of the residual rows and of the RoPE rows (runs of positions
+    # that break at request boundaries inside a chunk when gamma is 13)
+    import dataclasses
+    ctx = [300 - 17 * r for r in range(batch)]
+    w = dataclasses.replace(I.preset("small_bf16"), batch=batch, gamma=gamma, context=ctx, cycles=2)
+    pr = Pair(w)
+    pr.prefill()
+    anchors = I.make_anchors(w).numpy()
+    plan = I.plan_accept(w, w.cycles, gamma=gamma).numpy()
+    compared = 0
+    for cyc in range(w.cycles):
+        o_dr, g_dr, n = pr.draft(anchors, gamma)
+        compared += n
+        anchors = pr.verify_and_accept(o_dr, gamma, plan[cyc], cyc)
+        pr.check_cache()
+    assert compared > 0
