@@ -8,10 +8,13 @@
 // in TMEM.  Work units are k-blocks of 64 along K of every output tile; the
 // grid's CTAs take equal contiguous ranges of units (a range may start or end
 // inside a tile), so all SMs stream the same number of weight bytes whatever
-// the shape.  A tile split across CTAs is finished by the CTA that arrives
-// last on the tile's counter; it adds the fp32 partials in contributor order,
-// so the result does not depend on arrival order.  No CTA ever waits for
-// another.
+// the shape.  A tile split across CTAs is finished by its first contributor
+// (the CTA holding its k-block 0, for which the tile is the last segment): it
+// waits, bounded, for the others' published fp32 partials and adds them in
+// contributor order, so the result does not depend on arrival order (optionally
+// the last contributor to arrive finishes instead, adding in the same order).
+// Only a tile's first contributor ever waits, and only for CTAs that publish
+// before waiting on anything, so the waits form no cycle.
 #pragma once
 #include "common.cuh"
 
