@@ -911,16 +911,24 @@ __global__ void __launch_bounds__(GemmCfg<NT, CLU>::THREADS, GemmCfg<NT, CLU>::M
                     }
                     case EPI_SWIGLU: {
                         // Rows 0..63 of the tile are gate rows, 64..127 the matching up
-                        // rows.  The up values cross through the upper half of the
-                        // exchange buffer, the bf16 products through its lower half.
-                        if (row >= 64)
+                        // rows.  Both cross through the exchange buffer, so that all four
+                        // warps form products: thread e takes gate row e % 64 and half of
+                        // the chunk's tokens; the bf16 products then go through the buffer's
+                        // lower rows once every thread has read its pairs.
 #pragma unroll
-                            for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
+                        for (int i = 0; i < CH; ++i) xch[row * (CH + 1) + i] = v[i];
                         named_bar_sync(1, 128);
-                        if (row < 64)
+                        const int g = e & 63, i0 = (e >> 6) * (CH / 2);
+                        float prod[CH / 2];
 #pragma unroll
-                            for (int i = 0; i < CH; ++i)
-                                xout[i * 64 + row] = f2bf(silu(v[i]) * lds_f32(xch_a + (uint32_t)((row + 64) * (CH + 1) + i) * 4u));
+                        for (int j = 0; j < CH / 2; ++j) {
+                            const float gv = lds_f32(xch_a + (uint32_t)(g * (CH + 1) + i0 + j) * 4u);
+                            const float uv = lds_f32(xch_a + (uint32_t)((g + 64) * (CH + 1) + i0 + j) * 4u);
+                            prod[j] = silu(gv) * uv;
+                        }
+                        named_bar_sync(1, 128);
+#pragma unroll
+                        for (int j = 0; j < CH / 2; ++j) xout[(i0 + j) * 64 + g] = f2bf(prod[j]);
                         named_bar_sync(1, 128);
                         __nv_bfloat16* o = (__nv_bfloat16*)p.out;
 #pragma unroll
