@@ -82,3 +82,19 @@ def test_step_flops_and_kernelwise_roofline_are_consistent():
         t_bytes = bench.step_algorithmic_bytes(w, B, g, T) / (bw * 1e9) * 1e3
         t_flops = bench.step_flops(w, B, g, T) / (tf * 1e12) * 1e3
         assert kw >= max(t_bytes, t_flops) * (1 - 1e-12)
+
+
+def test_gemm_traffic_constant_matches_its_profile():
+    """The DRAM-traffic ratio the bench line multiplies by is the one the committed ncu
+    summary reports (the capture that `bench.py` cites), and it is a plausible ratio of
+    measured to algorithmic bytes (every weight byte read once, partials in L2)."""
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+    with open(os.path.join(ROOT, "profiles", "k_gemm_tc_m16_n24576_k4096.md")) as f:
+        text = f.read()
+    m = re.search(r"reports `roofline\.traffic` as ([0-9.]+)", text)
+    assert m, "the profile states the ratio the bench uses"
+    assert float(m.group(1)) == bench.GEMM_TRAFFIC["ratio"]
+    assert 1.0 <= bench.GEMM_TRAFFIC["ratio"] < 1.05
+    assert re.fullmatch(r"[0-9a-f]{64}", bench.GEMM_TRAFFIC["sources_sha256"])
